@@ -1,0 +1,458 @@
+#!/usr/bin/env python3
+"""Benchmark of the fused Dense-and-Sparse LUT GEMV, y = (Q + S) x.
+
+One step = one call of the fused kernel on one layer instance with one batch
+of activations.  Steps rotate over enough distinct layer instances that their
+total size is at least 4x the L2 cache, so every step streams its layer from
+HBM.  The K timed steps are CUDA-graph replays (one kernel node per step),
+bracketed by a barrier and a device synchronise, timed with CUDA events on
+the launching stream; the reported time is the maximum over ranks.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Prints one JSON line on rank 0.  ``--impl reference`` times the CPU oracle
+(plain fp64 C, single thread) on a bounded sample of the same workload.
+``--sweep`` prints one line per workload shape instead (for the notes).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+from lut_dequant_gemv_b200 import accounting as acc  # noqa: E402
+
+DEFAULT_WORKLOAD = "llama7b-up-3bit"
+METRIC = "3-bit dense+sparse GEMV achieved HBM GB/s (LLaMA-7B up_proj 11008x4096, batch 1)"
+FALLBACK_HBM_GBS = 6650.0
+
+WORKLOAD_DESC = {
+    "llama7b-q-4bit": "LLaMA-7B q_proj 4096x4096, 4-bit, 0.45% CSR outliers, batch 1",
+    "llama7b-up-3bit": "LLaMA-7B MLP up_proj 11008x4096, 3-bit, 0.45% CSR outliers, batch 1",
+}
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=50000)
+    p.add_argument("--warmup", type=int, default=5000)
+    p.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    p.add_argument("--shape-index", type=int, default=0)
+    p.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    p.add_argument("--sweep", action="store_true", help="one JSON line per workload shape")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--seed", type=int, default=0)
+    return p.parse_args()
+
+
+# ----------------------------------------------------------------- helpers
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "lut_dequant_gemv_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str, shape_key: str):
+    """DRAM bytes per launch from the committed ncu summary, valid only while
+    the kernel sources are unchanged since the capture."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    want = kernel_source_hash()
+    with open(path) as f:
+        for line in f:
+            line = line.split("#", 1)[0].strip()
+            if not line:
+                continue
+            kv = dict(tok.split("=", 1) for tok in line.split())
+            if kv.get("shape") == shape_key and kv.get("source_hash") == want:
+                return int(kv["bytes_per_launch"])
+    return None
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.ok = False
+        self.samples, self.reasons = [], 0
+        self.period = period_s
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(self._physical_index(device_index))
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # NVML missing: report that instead of clocks
+            self.err = str(e)
+        self._stop = threading.Event()
+
+    @staticmethod
+    def _physical_index(i):
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        if vis:
+            try:
+                return int(vis.split(",")[i])
+            except Exception:
+                return i
+        return i
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": f"NVML unavailable: {self.err}"}
+        names = [n for b, n in self.REASONS.items() if self.reasons & b]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+
+
+def shape_for(args) -> synth.Shape:
+    shapes = synth.workloads()[args.workload]
+    return shapes[args.shape_index]
+
+
+def config_for(args, shape, instances, inst_bytes):
+    return {
+        "workload": f"{args.workload}: " + WORKLOAD_DESC.get(
+            args.workload, f"{shape.n_out}x{shape.k_in}, {shape.bits}-bit, {shape.density:.2%} CSR, batch {shape.batch}"),
+        "n_out": shape.n_out, "k_in": shape.k_in, "bits": shape.bits, "density": shape.density,
+        "batch": shape.batch, "outliers": shape.dist,
+        "l2": f"inputs larger than L2: {instances} rotating layer instances, {instances * inst_bytes / 1e6:.0f} MB",
+        "parallelism": "replicas (independent layers per GPU)",
+    }
+
+
+# ------------------------------------------------------------- CPU oracle
+
+def cpu_oracle_rate(shape, seconds: float, rows_per_call: int, instance: int = 0):
+    """Time the oracle on rows of one layer instance; returns (GB/s, rows done, s)."""
+    import oracle
+
+    orc = oracle.default()
+    L = synth.layer_for(shape, instance=instance)
+    x = synth.x_for(shape, instance=instance)
+    per_row_bytes = acc.gemv_bytes(shape.n_out, shape.k_in, shape.bits, L.nnz, shape.batch) / shape.n_out
+    done, t0 = 0, time.perf_counter()
+    start = 0
+    while True:
+        rows = (np.arange(start, start + rows_per_call) % shape.n_out).astype(np.int32)
+        orc.gemv_layer(L, x, rows=rows)
+        done += rows_per_call
+        start += rows_per_call
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    return done * per_row_bytes / el / 1e9, done, el
+
+
+def run_reference(args):
+    world, rank, local = dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+
+    shape = shape_for(args)
+    orc = oracle.default()
+    L = synth.layer_for(shape)
+    x = synth.x_for(shape)
+    # size each step so that W + K steps take about 90 s of CPU time
+    t0 = time.perf_counter()
+    orc.gemv_layer(L, x, rows=np.arange(64, dtype=np.int32))
+    per_row = (time.perf_counter() - t0) / 64
+    rows_per_step = max(1, min(shape.n_out, int(90.0 / max(1, args.steps + args.warmup) / per_row)))
+    per_row_bytes = acc.gemv_bytes(shape.n_out, shape.k_in, shape.bits, L.nnz, shape.batch) / shape.n_out
+
+    def step(i):
+        rows = ((np.arange(rows_per_step) + i * rows_per_step) % shape.n_out).astype(np.int32)
+        orc.gemv_layer(L, x, rows=rows)
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(args.warmup + i)
+    el = time.perf_counter() - t0
+    gbs = args.steps * rows_per_step * per_row_bytes / el / 1e9
+    sample = f"{rows_per_step} of {shape.n_out} rows per step (fp64 C oracle, one thread)"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_for(args, shape, 1, L.nbytes()),
+        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------ GPU arm
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from lut_dequant_gemv_b200 import binding as B
+
+    world, rank, local = dist_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    B.lib()
+
+    shape = shape_for(args)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    L0 = synth.layer_for(shape, seed=args.seed, instance=rank * 1000)
+    inst_bytes = L0.nbytes()
+    instances = max(2, math.ceil(4 * l2 / inst_bytes))
+    layers, xs, ys = [], [], []
+    for i in range(instances):
+        L = L0 if i == 0 else synth.layer_for(shape, seed=args.seed, instance=rank * 1000 + i)
+        layers.append(B.create_layer_from_numpy(L.n_out, L.k_in, L.bits, L.codes, L.lut, L.rowptr, L.col, L.val,
+                                                device=dev))
+        xs.append(torch.from_numpy(synth.x_for(shape, seed=args.seed, instance=rank * 1000 + i).view(np.int16)).to(dev))
+        ys.append(torch.empty((shape.batch, shape.n_out), dtype=torch.int16, device=dev))
+    nnz = L0.nnz
+    bytes_per_step = acc.gemv_bytes(shape.n_out, shape.k_in, shape.bits, nnz, shape.batch)
+
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.synchronize(dev)
+    with torch.cuda.stream(stream):
+        for i in range(instances):
+            B.sqz_gemv(layers[i], xs[i], ys[i], stream=stream)
+    stream.synchronize()
+
+    def capture(n, offset):
+        g = torch.cuda.CUDAGraph()
+        if n == 0:
+            return None
+        with torch.cuda.graph(g, stream=stream):
+            for j in range(n):
+                i = (offset + j) % instances
+                B.sqz_gemv(layers[i], xs[i], ys[i], stream=stream)
+        return g
+
+    per_graph = instances * max(1, 512 // instances)
+
+    def run_steps(k, graphs):
+        full, tail = divmod(k, per_graph)
+        for _ in range(full):
+            graphs[0].replay()
+        if tail:
+            graphs[1][tail].replay()
+
+    main_graph = capture(per_graph, 0)
+    tails = {}
+    for k in {args.warmup % per_graph, args.steps % per_graph} - {0}:
+        tails[k] = capture(k, 0)
+    graphs = (main_graph, tails)
+
+    with torch.cuda.stream(stream):
+        run_steps(args.warmup, graphs)
+    stream.synchronize()
+
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        with torch.cuda.stream(stream):
+            ev0.record(stream)
+            run_steps(args.steps, graphs)
+            ev1.record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_per_step = ms / args.steps
+    value = world * bytes_per_step * args.steps / (ms / 1e3) / 1e9
+    per_launch_gbs = bytes_per_step / (ms_per_step / 1e3) / 1e9
+
+    # ---- end to end through the host entry point (pinned buffers)
+    xh = [torch.from_numpy(synth.x_for(shape, seed=args.seed, instance=rank * 1000 + i).view(np.int16).copy())
+          .pin_memory() for i in range(instances)]
+    yh = torch.empty((shape.batch, shape.n_out), dtype=torch.int16).pin_memory()
+    e2e_steps = min(args.steps, 20000)
+    with torch.cuda.stream(stream):
+        for j in range(min(args.warmup, 200)):
+            B.sqz_gemv_host(layers[j % instances], xh[j % instances], yh, stream=stream)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for j in range(e2e_steps):
+            B.sqz_gemv_host(layers[j % instances], xh[j % instances], yh, stream=stream)
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * bytes_per_step * e2e_steps / (e2e_ms / 1e3) / 1e9
+
+    # ---- fp16 dense yardstick (same shape, uncompressed weights)
+    yard = None
+    try:
+        yard = fp16_yardstick(B, torch, shape, dev, stream, l2)
+    except Exception as e:  # reported, never fatal for the headline
+        yard = {"error": str(e)}
+
+    peak, peak_kind = measured_peaks()
+    traffic = recorded_traffic(args.workload, shape.key)
+    line = {
+        "metric": METRIC if args.workload == DEFAULT_WORKLOAD else f"dense+sparse GEMV achieved HBM GB/s ({args.workload})",
+        "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_per_step, "us_per_call": ms_per_step * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f16 storage, f32 accumulate", "data": "synthetic",
+        "config": config_for(args, shape, instances, inst_bytes),
+        "roofline": {"bound": "hbm", "achieved": per_launch_gbs, "peak": peak, "unit": "GB/s",
+                     "frac": per_launch_gbs / peak, "traffic": traffic,
+                     "peak_kind": f"{peak_kind} copy bandwidth", "algorithmic_bytes_per_launch": bytes_per_step,
+                     "frac_of_nominal_8000": per_launch_gbs / 8000.0},
+        "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": 2 * shape.batch * shape.k_in,
+                "d2h_bytes_per_step": 2 * shape.batch * shape.n_out, "us_per_call": e2e_ms / e2e_steps * 1e3,
+                "steps": e2e_steps, "api": "sqz_gemv_host"},
+        "gpu_launches": args.steps,
+        "clocks": clk.summary(),
+        "yardstick_fp16_dense": yard,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        gbs, rows, secs = cpu_oracle_rate(shape, 10.0, 256)
+        line["cpu_baseline"] = {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                                "sample": f"{rows} rows of one {shape.n_out}x{shape.k_in} layer in {secs:.1f} s "
+                                          f"(fp64 C oracle, one thread)"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    for lay in layers:
+        lay.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def fp16_yardstick(B, torch, shape, dev, stream, l2):
+    """fp16 dense GEMV over the same shape (2*N*K weight bytes), same protocol."""
+    wbytes = 2 * shape.n_out * shape.k_in
+    n = max(2, math.ceil(4 * l2 / wbytes))
+    g = torch.Generator(device=dev).manual_seed(1)
+    ws = [(torch.randn(shape.n_out, shape.k_in, device=dev, generator=g) * 0.02).half() for _ in range(n)]
+    x = torch.randn(shape.batch, shape.k_in, device=dev, generator=g).half()
+    y = torch.empty(shape.batch, shape.n_out, device=dev, dtype=torch.half)
+    torch.cuda.synchronize(dev)
+    reps = n * max(1, 256 // n)
+    with torch.cuda.stream(stream):
+        for i in range(n):
+            B.sqz_fp16_gemv(ws[i], x, y, stream=stream)
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=stream):
+            for j in range(reps):
+                B.sqz_fp16_gemv(ws[j % n], x, y, stream=stream)
+        gr.replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(5):
+            gr.replay()
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    us = e0.elapsed_time(e1) * 1e3 / (5 * reps)
+    nbytes = acc.fp16_dense_bytes(shape.n_out, shape.k_in, shape.batch)
+    del ws
+    return {"us_per_call": us, "GB/s": nbytes / (us * 1e-6) / 1e9, "bytes": nbytes}
+
+
+def run_sweep(args):
+    """One JSON line per workload shape (single GPU, short)."""
+    import subprocess
+
+    for name, shapes in synth.workloads().items():
+        for i in range(len(shapes)):
+            cmd = [sys.executable, __file__, "--workload", name, "--shape-index", str(i), "--steps",
+                   str(args.steps), "--warmup", str(args.warmup), "--no-cpu-baseline"]
+            subprocess.run(cmd, check=True)
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    if args.sweep:
+        return run_sweep(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

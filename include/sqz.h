@@ -1,0 +1,174 @@
+/*
+ * sqz.h -- C ABI of the Dense-and-Sparse LUT-dequant GEMV library (libsqz.so)
+ * for NVIDIA B200 (sm_100a).
+ *
+ * Operation ("SqueezeLLM: Dense-and-Sparse Quantization", summary page,
+ * §3.4 "The Dense-and-Sparse Decomposition" and "Kernel Implementation"):
+ *
+ *     y = (Q + S) x
+ *
+ *   Q  dense part: every weight w(i,k) is a b-bit index (b = 3 or 4) into a
+ *      lookup table of 2^b fp16 centroids owned by output row i
+ *      (channel-wise LUTs, §3.2 "Sensitivity-Based K-Means Quantizer");
+ *      w(i,k) = lut[i][code(i,k)].
+ *   S  sparse outliers in CSR form: fp16 values, int32 column indices,
+ *      int32 row pointer (§3.4 "The Sparse Matrix Storage Format").
+ *   x  fp16 activations, batch 1..16; y fp16 outputs.
+ *
+ * Canonical storage (what sqz_create_layer reads):
+ *   codes  uint32 [n_out][k_in*bits/32], one LSB-first bitstream per row:
+ *          code(i,k) is the bits-wide field that starts at stream bit k*bits,
+ *          stream bit p being bit (p mod 32) of word (p div 32) of row i.
+ *          Exactly `bits` bits per index, no padding (§3.4 "The 3/4-bit
+ *          storage format": eight 3-bit indices in 3 bytes).  For 3-bit codes
+ *          this is the same as groups of 32 codes in 3 words; codes 10 and
+ *          21 of every group straddle two words.
+ *   lut    uint16 (fp16 bit patterns) [n_out][2^bits]
+ *   rowptr int32 [n_out+1], col int32 [nnz], val uint16 (fp16 bits) [nnz].
+ *          Columns within a row may be unsorted; duplicates are summed;
+ *          empty rows are allowed.  Q and S are added: a position present
+ *          in S still has a code in Q.
+ *
+ * Arithmetic: products of fp16 operands are exact in fp32; accumulation is
+ * in fp32; y(i,b) is rounded once to fp16 (round to nearest even).  The
+ * result agrees with the exact value within 1e-3 * sum_k |w x| + 1e-6 and is
+ * bitwise reproducible from run to run (no floating-point atomics).
+ *
+ * Layouts: x is [batch][ldx] and y is [batch][ldy], row-major (the
+ * torch `x @ W.T` convention).  y is overwritten, never accumulated into.
+ *
+ * Errors: every entry point returns an sqz_status; nothing throws, aborts or
+ * traps.  sqz_last_error() gives a message for the last non-OK status of the
+ * calling thread.
+ */
+#ifndef SQZ_H_
+#define SQZ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Exported entry points keep default visibility even when the library is
+ * built with -fvisibility=hidden. */
+#if defined(__GNUC__)
+#define SQZ_API __attribute__((visibility("default")))
+#else
+#define SQZ_API
+#endif
+
+typedef struct sqz_layer* sqz_layer_t;
+
+typedef enum {
+    SQZ_OK = 0,
+    SQZ_ERR_INVALID_ARG = 1, /* null pointer, bad size, malformed CSR          */
+    SQZ_ERR_UNSUPPORTED = 2, /* valid request this build does not implement    */
+    SQZ_ERR_CUDA = 3,        /* a CUDA runtime call or kernel launch failed    */
+    SQZ_ERR_OOM = 4,         /* device allocation failed                       */
+    SQZ_ERR_TIMEOUT = 5      /* a bounded device wait gave up                  */
+} sqz_status;
+
+/* Largest batch (columns of x) one call accepts. */
+#define SQZ_MAX_BATCH 16
+
+/* Description of one layer in canonical storage.  All pointers are DEVICE
+ * pointers on the current CUDA device, owned by the caller. */
+typedef struct {
+    int32_t n_out;          /* N: output rows, >= 0                                   */
+    int32_t k_in;           /* K: input columns, >= 0; K % 32 == 0 for 3-bit,
+                               K % 8 == 0 for 4-bit (whole 32-bit words per row)      */
+    int32_t bits;           /* 3 or 4                                                 */
+    const uint32_t* codes;  /* [n_out][k_in*bits/32]; may be NULL when N*K == 0        */
+    const uint16_t* lut;    /* [n_out][1<<bits] fp16 bits; may be NULL when N == 0     */
+    int64_t nnz;            /* outliers, 0 <= nnz <= INT32_MAX                        */
+    const int32_t* rowptr;  /* [n_out+1]; may be NULL when nnz == 0                   */
+    const int32_t* col;     /* [nnz];     may be NULL when nnz == 0                   */
+    const uint16_t* val;    /* [nnz] fp16 bits; may be NULL when nnz == 0             */
+} sqz_layer_desc;
+
+/*
+ * Build a layer handle from canonical storage: the per-layer output of the
+ * offline compression pipeline (codes, LUTs and outlier matrix; §3.2
+ * "Big-Picture Architecture"), which the inference kernels consume.
+ *
+ * Copies every array into device memory the handle owns, rearranged into
+ * the kernels' layout; the caller may free its arrays once this returns.
+ * Work is ordered on `stream` (a cudaStream_t; NULL = legacy default
+ * stream) and the call synchronises that stream once to read the CSR
+ * validation result.
+ *
+ * Errors: SQZ_ERR_INVALID_ARG for a NULL desc/out, bits not in {3,4}, K not
+ * a whole number of words per row, negative sizes, a required NULL array,
+ * or a CSR that fails the device-side check (rowptr[0] != 0, rowptr
+ * decreasing, rowptr[N] != nnz, a column outside [0, K)); SQZ_ERR_OOM;
+ * SQZ_ERR_CUDA.  On error *out is set to NULL and nothing is leaked.
+ */
+SQZ_API sqz_status sqz_create_layer(const sqz_layer_desc* desc, void* stream, sqz_layer_t* out);
+
+/*
+ * y = (Q + S) x for `batch` columns, asynchronously on `stream`.
+ *
+ * x: device, fp16 bits, [batch][ldx] (ldx >= K); y: device, fp16 bits,
+ * [batch][ldy] (ldy >= N).  x and y are borrowed until the stream reaches
+ * the end of this call; they must not overlap.  One fused kernel launch:
+ * the dense LUT part and the CSR part of a row are summed on chip and y is
+ * written once (§3.4 "Kernel fusion").
+ *
+ * Errors: SQZ_ERR_INVALID_ARG (NULL layer/x/y with non-empty sizes, batch
+ * outside [1, SQZ_MAX_BATCH], ldx < K, ldy < N); SQZ_ERR_CUDA if the launch
+ * fails.  No synchronisation.
+ */
+SQZ_API sqz_status sqz_gemv(sqz_layer_t layer, const uint16_t* x, int32_t batch, int64_t ldx, uint16_t* y,
+                    int64_t ldy, void* stream);
+
+/*
+ * The same product for callers whose activations live in HOST memory:
+ * copies x (host, [batch][ldx]) to the handle's device staging buffer,
+ * runs sqz_gemv, copies y back to host memory ([batch][ldy]) and
+ * synchronises `stream` before returning.  Pinned host buffers give
+ * asynchronous copies; pageable ones work but copy synchronously.
+ * Errors as sqz_gemv.
+ */
+SQZ_API sqz_status sqz_gemv_host(sqz_layer_t layer, const uint16_t* x_host, int32_t batch, int64_t ldx,
+                         uint16_t* y_host, int64_t ldy, void* stream);
+
+/*
+ * Write the dequantized dense weights w(i,k) = lut[i][code(i,k)] as fp16 bit
+ * patterns to w_out (device, [n_out][k_in]), decoded from the handle's
+ * internal layout with the same decoder the GEMV kernel uses.  For
+ * checking only (the GEMV never materialises these weights).  Async on
+ * `stream`.  Errors: SQZ_ERR_INVALID_ARG, SQZ_ERR_CUDA.
+ */
+SQZ_API sqz_status sqz_debug_dequant(sqz_layer_t layer, uint16_t* w_out, void* stream);
+
+/* Sizes of a handle (any output pointer may be NULL). */
+SQZ_API sqz_status sqz_layer_info(sqz_layer_t layer, int32_t* n_out, int32_t* k_in, int32_t* bits, int64_t* nnz,
+                          int64_t* device_bytes);
+
+/* Release a handle and its device memory.  NULL is accepted.  The caller
+ * must make sure no work that uses the handle is still in flight. */
+SQZ_API sqz_status sqz_destroy(sqz_layer_t layer);
+
+/*
+ * fp16 dense matrix-vector product y = W x with W fp16 [n_out][ldw] (ldw >=
+ * k_in), x [batch][ldx], y [batch][ldy]: the uncompressed fp16 baseline that
+ * the quantized kernels' speedups are reported against (§5 "Inference
+ * Latency and Memory Benchmarking", Table G.12), used here as a bandwidth
+ * yardstick.  Same arithmetic contract and errors as sqz_gemv.
+ */
+SQZ_API sqz_status sqz_fp16_gemv(const uint16_t* w, int32_t n_out, int32_t k_in, int64_t ldw, const uint16_t* x,
+                         int32_t batch, int64_t ldx, uint16_t* y, int64_t ldy, void* stream);
+
+/* Message for the calling thread's last non-OK status ("" if none). */
+SQZ_API const char* sqz_last_error(void);
+
+/* Library version: major*10000 + minor*100 + patch. */
+SQZ_API int32_t sqz_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SQZ_H_ */

@@ -1,0 +1,341 @@
+// sqz_api.cu -- host side of the C ABI declared in include/sqz.h.
+//
+// Argument checks happen on the host before any CUDA call; device-content
+// checks (CSR well-formedness) run in a validation kernel whose result the
+// create call reads back.  Nothing here aborts, throws across the ABI or
+// traps on the device.
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <string>
+
+#include "../../include/sqz.h"
+#include "kernels_basic.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+sqz_status fail(sqz_status s, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return s;
+}
+
+sqz_status cuda_fail(cudaError_t e, const char* what) {
+    return fail(e == cudaErrorMemoryAllocation ? SQZ_ERR_OOM : SQZ_ERR_CUDA, "%s: %s (%s)", what,
+                cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+#define SQZ_CUDA_TRY(expr, what)                 \
+    do {                                         \
+        cudaError_t e_ = (expr);                 \
+        if (e_ != cudaSuccess) {                 \
+            (void)cudaGetLastError();            \
+            return cuda_fail(e_, what);          \
+        }                                        \
+    } while (0)
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+int sm_count_of_current_device() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+    return n;
+}
+
+}  // namespace
+
+struct sqz_layer {
+    int32_t n_out = 0, k_in = 0, bits = 0;
+    int64_t nnz = 0;
+    int64_t wpr = 0;  // 32-bit words per row of codes
+    int device = 0;
+    int sm_count = 148;
+    uint32_t* codes = nullptr;
+    uint16_t* lut = nullptr;
+    int32_t* rowptr = nullptr;
+    int32_t* col = nullptr;
+    uint16_t* val = nullptr;
+    uint16_t* x_stage = nullptr;  // [SQZ_MAX_BATCH][k_in] for sqz_gemv_host
+    uint16_t* y_stage = nullptr;  // [SQZ_MAX_BATCH][n_out]
+    int64_t device_bytes = 0;
+};
+
+namespace {
+
+void free_layer(sqz_layer* L) {
+    if (!L) return;
+    cudaFree(L->codes);
+    cudaFree(L->lut);
+    cudaFree(L->rowptr);
+    cudaFree(L->col);
+    cudaFree(L->val);
+    cudaFree(L->x_stage);
+    cudaFree(L->y_stage);
+    delete L;
+}
+
+template <class T>
+sqz_status alloc(T** p, size_t count, sqz_layer* L, const char* what) {
+    *p = nullptr;
+    if (count == 0) return SQZ_OK;
+    cudaError_t e = cudaMalloc(reinterpret_cast<void**>(p), count * sizeof(T));
+    if (e != cudaSuccess) {
+        (void)cudaGetLastError();
+        *p = nullptr;
+        return cuda_fail(e, what);
+    }
+    L->device_bytes += (int64_t)(count * sizeof(T));
+    return SQZ_OK;
+}
+
+sqz_status check_desc(const sqz_layer_desc* d) {
+    if (d->bits != 3 && d->bits != 4) return fail(SQZ_ERR_INVALID_ARG, "bits must be 3 or 4 (got %d)", d->bits);
+    if (d->n_out < 0 || d->k_in < 0) return fail(SQZ_ERR_INVALID_ARG, "negative size (n_out=%d, k_in=%d)", d->n_out, d->k_in);
+    const int kmult = d->bits == 3 ? 32 : 8;
+    if (d->k_in % kmult != 0)
+        return fail(SQZ_ERR_INVALID_ARG, "k_in=%d must be a multiple of %d for %d-bit codes (whole words per row)",
+                    d->k_in, kmult, d->bits);
+    if (d->nnz < 0 || d->nnz > INT32_MAX) return fail(SQZ_ERR_INVALID_ARG, "nnz=%lld out of range", (long long)d->nnz);
+    if ((int64_t)d->n_out * d->k_in > 0 && !d->codes) return fail(SQZ_ERR_INVALID_ARG, "codes is NULL");
+    if (d->n_out > 0 && !d->lut) return fail(SQZ_ERR_INVALID_ARG, "lut is NULL");
+    if (d->nnz > 0 && (!d->rowptr || !d->col || !d->val))
+        return fail(SQZ_ERR_INVALID_ARG, "nnz=%lld but rowptr/col/val is NULL", (long long)d->nnz);
+    if (d->nnz > 0 && d->k_in == 0) return fail(SQZ_ERR_INVALID_ARG, "nnz > 0 with k_in == 0");
+    return SQZ_OK;
+}
+
+sqz_status check_gemv_args(const sqz_layer* L, const void* x, int32_t batch, int64_t ldx, const void* y, int64_t ldy) {
+    if (!L) return fail(SQZ_ERR_INVALID_ARG, "layer is NULL");
+    if (batch < 1 || batch > SQZ_MAX_BATCH)
+        return fail(SQZ_ERR_INVALID_ARG, "batch=%d outside [1, %d]", batch, SQZ_MAX_BATCH);
+    if (ldx < L->k_in) return fail(SQZ_ERR_INVALID_ARG, "ldx=%lld < k_in=%d", (long long)ldx, L->k_in);
+    if (ldy < L->n_out) return fail(SQZ_ERR_INVALID_ARG, "ldy=%lld < n_out=%d", (long long)ldy, L->n_out);
+    if (L->k_in > 0 && !x) return fail(SQZ_ERR_INVALID_ARG, "x is NULL");
+    if (L->n_out > 0 && !y) return fail(SQZ_ERR_INVALID_ARG, "y is NULL");
+    return SQZ_OK;
+}
+
+template <int BITS, int B>
+void launch_rowwarp(const sqz_layer* L, const uint16_t* x, int64_t ldx, uint16_t* y, int64_t ldy, cudaStream_t s) {
+    const int64_t blocks = (L->n_out + 7) / 8;
+    const unsigned grid = (unsigned)(blocks < 65535 * 8 ? blocks : 65535 * 8);
+    sqz::gemv_rowwarp_kernel<BITS, B><<<grid, 256, 0, s>>>(L->codes, L->lut, L->rowptr, L->col, L->val, L->nnz, x,
+                                                         ldx, y, ldy, L->n_out, L->k_in);
+}
+
+template <int BITS>
+void dispatch_batch(const sqz_layer* L, const uint16_t* x, int32_t batch, int64_t ldx, uint16_t* y, int64_t ldy,
+                    cudaStream_t s) {
+    switch (batch) {
+#define SQZ_CASE(B) \
+    case B: launch_rowwarp<BITS, B>(L, x, ldx, y, ldy, s); break;
+        SQZ_CASE(1) SQZ_CASE(2) SQZ_CASE(3) SQZ_CASE(4) SQZ_CASE(5) SQZ_CASE(6) SQZ_CASE(7) SQZ_CASE(8)
+        SQZ_CASE(9) SQZ_CASE(10) SQZ_CASE(11) SQZ_CASE(12) SQZ_CASE(13) SQZ_CASE(14) SQZ_CASE(15) SQZ_CASE(16)
+#undef SQZ_CASE
+        default: break;
+    }
+}
+
+sqz_status gemv_impl(const sqz_layer* L, const uint16_t* x, int32_t batch, int64_t ldx, uint16_t* y, int64_t ldy,
+                     cudaStream_t s) {
+    if (L->n_out == 0) return SQZ_OK;
+    if (L->bits == 3)
+        dispatch_batch<3>(L, x, batch, ldx, y, ldy, s);
+    else
+        dispatch_batch<4>(L, x, batch, ldx, y, ldy, s);
+    SQZ_CUDA_TRY(cudaGetLastError(), "gemv launch");
+    return SQZ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+sqz_status sqz_create_layer(const sqz_layer_desc* desc, void* stream, sqz_layer_t* out) {
+    if (out) *out = nullptr;
+    if (!desc || !out) return fail(SQZ_ERR_INVALID_ARG, "desc and out must be non-NULL");
+    sqz_status st = check_desc(desc);
+    if (st != SQZ_OK) return st;
+    cudaStream_t s = as_stream(stream);
+
+    sqz_layer* L = new (std::nothrow) sqz_layer();
+    if (!L) return fail(SQZ_ERR_OOM, "host allocation of the layer handle failed");
+    L->n_out = desc->n_out;
+    L->k_in = desc->k_in;
+    L->bits = desc->bits;
+    L->nnz = desc->nnz;
+    L->wpr = (int64_t)desc->k_in * desc->bits / 32;
+    L->sm_count = sm_count_of_current_device();
+    cudaGetDevice(&L->device);
+
+    const size_t n = (size_t)desc->n_out, lut_n = n << desc->bits, code_n = n * (size_t)L->wpr;
+    const size_t nnz = (size_t)desc->nnz;
+#define SQZ_STEP(expr)                 \
+    do {                               \
+        sqz_status s_ = (expr);        \
+        if (s_ != SQZ_OK) {            \
+            free_layer(L);             \
+            return s_;                 \
+        }                              \
+    } while (0)
+#define SQZ_CUDA_STEP(expr, what)               \
+    do {                                        \
+        cudaError_t e_ = (expr);                \
+        if (e_ != cudaSuccess) {                \
+            (void)cudaGetLastError();           \
+            free_layer(L);                      \
+            return cuda_fail(e_, what);         \
+        }                                       \
+    } while (0)
+
+    SQZ_STEP(alloc(&L->codes, code_n, L, "codes allocation"));
+    SQZ_STEP(alloc(&L->lut, lut_n, L, "lut allocation"));
+    if (nnz > 0) {
+        SQZ_STEP(alloc(&L->rowptr, n + 1, L, "rowptr allocation"));
+        SQZ_STEP(alloc(&L->col, nnz, L, "col allocation"));
+        SQZ_STEP(alloc(&L->val, nnz, L, "val allocation"));
+    }
+    SQZ_STEP(alloc(&L->x_stage, (size_t)SQZ_MAX_BATCH * desc->k_in, L, "x staging allocation"));
+    SQZ_STEP(alloc(&L->y_stage, (size_t)SQZ_MAX_BATCH * n, L, "y staging allocation"));
+
+    if (code_n)
+        SQZ_CUDA_STEP(cudaMemcpyAsync(L->codes, desc->codes, code_n * 4, cudaMemcpyDeviceToDevice, s), "codes copy");
+    if (lut_n)
+        SQZ_CUDA_STEP(cudaMemcpyAsync(L->lut, desc->lut, lut_n * 2, cudaMemcpyDeviceToDevice, s), "lut copy");
+    if (nnz > 0) {
+        SQZ_CUDA_STEP(cudaMemcpyAsync(L->rowptr, desc->rowptr, (n + 1) * 4, cudaMemcpyDeviceToDevice, s), "rowptr copy");
+        SQZ_CUDA_STEP(cudaMemcpyAsync(L->col, desc->col, nnz * 4, cudaMemcpyDeviceToDevice, s), "col copy");
+        SQZ_CUDA_STEP(cudaMemcpyAsync(L->val, desc->val, nnz * 2, cudaMemcpyDeviceToDevice, s), "val copy");
+
+        int* d_flag = nullptr;
+        SQZ_CUDA_STEP(cudaMalloc(&d_flag, sizeof(int)), "validation flag allocation");
+        int h_flag = 0;
+        cudaError_t e = cudaMemsetAsync(d_flag, 0, sizeof(int), s);
+        if (e == cudaSuccess) {
+            const int64_t work = (nnz > n + 1 ? (int64_t)nnz : (int64_t)n + 1);
+            int64_t blocks = (work + 255) / 256;
+            if (blocks > (int64_t)L->sm_count * 8) blocks = (int64_t)L->sm_count * 8;
+            sqz::validate_csr_kernel<<<(unsigned)blocks, 256, 0, s>>>(L->rowptr, L->col, L->n_out, L->k_in, L->nnz,
+                                                                        d_flag);
+            e = cudaGetLastError();
+        }
+        if (e == cudaSuccess) e = cudaMemcpyAsync(&h_flag, d_flag, sizeof(int), cudaMemcpyDeviceToHost, s);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+        cudaFree(d_flag);
+        if (e != cudaSuccess) {
+            (void)cudaGetLastError();
+            free_layer(L);
+            return cuda_fail(e, "CSR validation");
+        }
+        if (h_flag) {
+            free_layer(L);
+            return fail(SQZ_ERR_INVALID_ARG, "malformed CSR:%s%s%s%s", (h_flag & 1) ? " rowptr[0]!=0" : "",
+                        (h_flag & 2) ? " rowptr[N]!=nnz" : "", (h_flag & 4) ? " rowptr decreasing" : "",
+                        (h_flag & 8) ? " column outside [0,K)" : "");
+        }
+    }
+#undef SQZ_STEP
+#undef SQZ_CUDA_STEP
+    *out = L;
+    return SQZ_OK;
+}
+
+sqz_status sqz_gemv(sqz_layer_t layer, const uint16_t* x, int32_t batch, int64_t ldx, uint16_t* y, int64_t ldy,
+                    void* stream) {
+    sqz_status st = check_gemv_args(layer, x, batch, ldx, y, ldy);
+    if (st != SQZ_OK) return st;
+    return gemv_impl(layer, x, batch, ldx, y, ldy, as_stream(stream));
+}
+
+sqz_status sqz_gemv_host(sqz_layer_t layer, const uint16_t* x_host, int32_t batch, int64_t ldx, uint16_t* y_host,
+                         int64_t ldy, void* stream) {
+    sqz_status st = check_gemv_args(layer, x_host, batch, ldx, y_host, ldy);
+    if (st != SQZ_OK) return st;
+    cudaStream_t s = as_stream(stream);
+    const sqz_layer* L = layer;
+    if (L->k_in > 0)
+        SQZ_CUDA_TRY(cudaMemcpy2DAsync(L->x_stage, (size_t)L->k_in * 2, x_host, (size_t)ldx * 2, (size_t)L->k_in * 2,
+                                       (size_t)batch, cudaMemcpyHostToDevice, s),
+                     "x host-to-device copy");
+    st = gemv_impl(L, L->x_stage, batch, L->k_in, L->y_stage, L->n_out, s);
+    if (st != SQZ_OK) return st;
+    if (L->n_out > 0)
+        SQZ_CUDA_TRY(cudaMemcpy2DAsync(y_host, (size_t)ldy * 2, L->y_stage, (size_t)L->n_out * 2, (size_t)L->n_out * 2,
+                                       (size_t)batch, cudaMemcpyDeviceToHost, s),
+                     "y device-to-host copy");
+    SQZ_CUDA_TRY(cudaStreamSynchronize(s), "stream synchronize");
+    return SQZ_OK;
+}
+
+sqz_status sqz_debug_dequant(sqz_layer_t layer, uint16_t* w_out, void* stream) {
+    if (!layer) return fail(SQZ_ERR_INVALID_ARG, "layer is NULL");
+    const sqz_layer* L = layer;
+    if ((int64_t)L->n_out * L->k_in == 0) return SQZ_OK;
+    if (!w_out) return fail(SQZ_ERR_INVALID_ARG, "w_out is NULL");
+    cudaStream_t s = as_stream(stream);
+    const int grid = L->sm_count * 4;
+    if (L->bits == 3)
+        sqz::dequant_canonical_kernel<3><<<grid, 256, 0, s>>>(L->codes, L->lut, L->n_out, L->k_in, w_out);
+    else
+        sqz::dequant_canonical_kernel<4><<<grid, 256, 0, s>>>(L->codes, L->lut, L->n_out, L->k_in, w_out);
+    SQZ_CUDA_TRY(cudaGetLastError(), "dequant launch");
+    return SQZ_OK;
+}
+
+sqz_status sqz_layer_info(sqz_layer_t layer, int32_t* n_out, int32_t* k_in, int32_t* bits, int64_t* nnz,
+                          int64_t* device_bytes) {
+    if (!layer) return fail(SQZ_ERR_INVALID_ARG, "layer is NULL");
+    if (n_out) *n_out = layer->n_out;
+    if (k_in) *k_in = layer->k_in;
+    if (bits) *bits = layer->bits;
+    if (nnz) *nnz = layer->nnz;
+    if (device_bytes) *device_bytes = layer->device_bytes;
+    return SQZ_OK;
+}
+
+sqz_status sqz_destroy(sqz_layer_t layer) {
+    free_layer(layer);
+    return SQZ_OK;
+}
+
+sqz_status sqz_fp16_gemv(const uint16_t* w, int32_t n_out, int32_t k_in, int64_t ldw, const uint16_t* x,
+                         int32_t batch, int64_t ldx, uint16_t* y, int64_t ldy, void* stream) {
+    if (n_out < 0 || k_in < 0) return fail(SQZ_ERR_INVALID_ARG, "negative size");
+    if (batch < 1 || batch > SQZ_MAX_BATCH)
+        return fail(SQZ_ERR_INVALID_ARG, "batch=%d outside [1, %d]", batch, SQZ_MAX_BATCH);
+    if (ldw < k_in || ldx < k_in || ldy < n_out) return fail(SQZ_ERR_INVALID_ARG, "leading dimension too small");
+    if ((int64_t)n_out * k_in > 0 && (!w || !x)) return fail(SQZ_ERR_INVALID_ARG, "w or x is NULL");
+    if (n_out > 0 && !y) return fail(SQZ_ERR_INVALID_ARG, "y is NULL");
+    if (n_out == 0) return SQZ_OK;
+    cudaStream_t s = as_stream(stream);
+    const int vec_ok = ((reinterpret_cast<uintptr_t>(w) | reinterpret_cast<uintptr_t>(x)) % 16 == 0) &&
+                       ldw % 8 == 0 && ldx % 8 == 0 && k_in % 8 == 0;
+    const int64_t blocks = (n_out + 7) / 8;
+    const unsigned grid = (unsigned)(blocks < 65535 * 8 ? blocks : 65535 * 8);
+    switch (batch) {
+#define SQZ_CASE(B) \
+    case B: sqz::fp16_gemv_kernel<B><<<grid, 256, 0, s>>>(w, ldw, x, ldx, y, ldy, n_out, k_in, vec_ok); break;
+        SQZ_CASE(1) SQZ_CASE(2) SQZ_CASE(3) SQZ_CASE(4) SQZ_CASE(5) SQZ_CASE(6) SQZ_CASE(7) SQZ_CASE(8)
+        SQZ_CASE(9) SQZ_CASE(10) SQZ_CASE(11) SQZ_CASE(12) SQZ_CASE(13) SQZ_CASE(14) SQZ_CASE(15) SQZ_CASE(16)
+#undef SQZ_CASE
+        default: break;
+    }
+    SQZ_CUDA_TRY(cudaGetLastError(), "fp16 gemv launch");
+    return SQZ_OK;
+}
+
+const char* sqz_last_error(void) { return g_last_error.c_str(); }
+
+int32_t sqz_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,251 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Tolerance (from the arithmetic contract in include/sqz.h): for every output
+    |y_gpu - y| <= 1e-3 * sum_k |w x| + 1e-6
+with y the oracle's fp64 value and the bound computed by the oracle.
+Dequantized weights must match the oracle bit for bit.
+"""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from pins import f16_val, random_csr
+
+pytestmark = pytest.mark.gpu
+
+REL, ABS = 1e-3, 1e-6
+
+
+@pytest.fixture(scope="module")
+def B():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from lut_dequant_gemv_b200 import binding, build
+
+    build.build()
+    binding.lib()
+    return binding
+
+
+def upload(B, L):
+    return B.create_layer_from_numpy(L.n_out, L.k_in, L.bits, L.codes, L.lut, L.rowptr, L.col, L.val)
+
+
+def gpu_gemv(B, layer, x_np, ldx=None, ldy=None, n_out=None):
+    batch, k_in = x_np.shape
+    ldx = ldx or k_in
+    n_out = layer.n_out if n_out is None else n_out
+    ldy = ldy or n_out
+    xd = torch.zeros((batch, ldx), dtype=torch.int16, device="cuda")
+    xd[:, :k_in] = torch.from_numpy(x_np.view(np.int16)).cuda()
+    yd = torch.full((batch, ldy), 0x7E00, dtype=torch.int16, device="cuda")  # NaN sentinel
+    B.sqz_gemv(layer, xd, yd)
+    torch.cuda.synchronize()
+    return yd.cpu().numpy().view(np.uint16)
+
+
+def assert_close(y16, y_ref, bound, where=""):
+    yg = f16_val(y16)
+    err = np.abs(yg - y_ref)
+    lim = REL * bound + ABS
+    bad = np.argwhere(~(err <= lim))
+    assert bad.size == 0, (f"{where}: {len(bad)} outputs out of tolerance, first {bad[:5].tolist()}, "
+                           f"gpu={yg[tuple(bad[0])]}, ref={y_ref[tuple(bad[0])]}, bound={bound[tuple(bad[0])]}")
+
+
+def make_small(seed, n_out, k_in, bits, nnz, dup=False, unsorted=False):
+    rng = np.random.default_rng(seed)
+    wpr = k_in * bits // 32
+    codes = rng.integers(0, 1 << 32, size=(n_out, wpr), dtype=np.uint64).astype(np.uint32)
+    lut = np.sort(rng.normal(0, 0.02, size=(n_out, 1 << bits)), axis=1).astype(np.float16).view(np.uint16)
+    rowptr, col, val = random_csr(rng, n_out, k_in, nnz, dup=dup, unsorted=unsorted)
+    return synth.Layer(n_out, k_in, bits, codes, lut, rowptr, col, val)
+
+
+SMALL = [
+    # (n_out, k_in, bits, nnz, batch, dup, unsorted)
+    (1, 32, 3, 0, 1, False, False),
+    (1, 8, 4, 1, 1, False, False),
+    (7, 96, 3, 9, 3, True, True),
+    (33, 24, 4, 40, 2, False, False),
+    (65, 1024, 3, 300, 1, False, True),
+    (129, 1000, 4, 500, 5, True, False),
+    (300, 4128, 3, 2000, 16, False, False),
+    (257, 4104, 4, 1500, 7, False, False),
+    (64, 2048, 3, 0, 16, False, False),
+]
+
+
+@pytest.mark.parametrize("n_out,k_in,bits,nnz,batch,dup,unsorted", SMALL)
+def test_small_shapes(B, orc, n_out, k_in, bits, nnz, batch, dup, unsorted):
+    L = make_small(1000 + n_out + k_in, n_out, k_in, bits, nnz, dup, unsorted)
+    x = (np.random.default_rng(7).standard_normal((batch, k_in))).astype(np.float16).view(np.uint16)
+    layer = upload(B, L)
+    y = gpu_gemv(B, layer, x)
+    y_ref, bound = orc.gemv_layer(L, x)
+    assert_close(y, y_ref, bound, f"{n_out}x{k_in} b{bits}")
+
+
+def test_skewed_row(B, orc):
+    """One very dense row (every column an outlier) among empty rows."""
+    n_out, k_in, bits = 40, 512, 3
+    L = make_small(5, n_out, k_in, bits, 0)
+    counts = np.zeros(n_out, dtype=np.int64)
+    counts[17] = k_in
+    counts[3] = 5
+    rowptr = np.zeros(n_out + 1, dtype=np.int32)
+    np.cumsum(counts, out=rowptr[1:])
+    col = np.concatenate([np.arange(5) * 7, np.arange(k_in)[::-1]]).astype(np.int32)
+    val = np.random.default_rng(3).uniform(-0.5, 0.5, size=len(col)).astype(np.float16).view(np.uint16)
+    L = synth.Layer(n_out, k_in, bits, L.codes, L.lut, rowptr, col, val)
+    x = synth.make_x(2, k_in, seed=1)
+    y = gpu_gemv(B, upload(B, L), x)
+    y_ref, bound = orc.gemv_layer(L, x)
+    assert_close(y, y_ref, bound)
+
+
+def test_strided_x_and_y(B, orc):
+    """ldx > K and ldy > N: padding of y is left untouched."""
+    L = make_small(9, 50, 256, 4, 30)
+    x = synth.make_x(3, 256, seed=2)
+    layer = upload(B, L)
+    y = gpu_gemv(B, layer, x, ldx=256 + 24, ldy=50 + 13)
+    y_ref, bound = orc.gemv_layer(L, x)
+    assert_close(y[:, :50], y_ref, bound)
+    assert np.all(y[:, 50:] == 0x7E00)
+
+
+def test_degenerate_sizes(B, orc):
+    # N = 0: nothing written, no error
+    L0 = synth.Layer(0, 64, 3, np.zeros((0, 6), np.uint32), np.zeros((0, 8), np.uint16),
+                     np.zeros(1, np.int32), np.zeros(0, np.int32), np.zeros(0, np.uint16))
+    layer = upload(B, L0)
+    xd = torch.zeros((1, 64), dtype=torch.int16, device="cuda")
+    yd = torch.zeros((1, 1), dtype=torch.int16, device="cuda")
+    B.lib().sqz_gemv(layer, xd.data_ptr(), 1, 64, yd.data_ptr(), 1, None)
+    # K = 0: y = 0
+    Lk = synth.Layer(5, 0, 4, np.zeros((5, 0), np.uint32), np.ones((5, 16), np.uint16) * 0x3C00,
+                     np.zeros(6, np.int32), np.zeros(0, np.int32), np.zeros(0, np.uint16))
+    layer = upload(B, Lk)
+    yd = torch.full((1, 5), 0x7E00, dtype=torch.int16, device="cuda")
+    B.lib().sqz_gemv(layer, None, 1, 0, yd.data_ptr(), 5, None)
+    torch.cuda.synchronize()
+    assert np.all(yd.cpu().numpy() == 0)
+
+
+def test_dequant_bit_exact(B, orc):
+    for L in (make_small(11, 37, 4096, 3, 10), make_small(12, 19, 1032, 4, 0),
+              synth.layer_for(synth.workloads()["llama7b-q-4bit"][0])):
+        layer = upload(B, L)
+        w = torch.empty((L.n_out, L.k_in), dtype=torch.int16, device="cuda")
+        B.sqz_debug_dequant(layer, w)
+        torch.cuda.synchronize()
+        ref = orc.dequant(L.codes, L.lut, L.n_out, L.k_in, L.bits)
+        assert np.array_equal(w.cpu().numpy().view(np.uint16), ref)
+
+
+def _rows_for(shape, limit=60_000_000):
+    if shape.n_out * shape.k_in * shape.batch <= limit:
+        return None
+    rng = np.random.default_rng(shape.n_out + shape.k_in)
+    r = rng.choice(shape.n_out, size=384, replace=False)
+    return np.unique(np.concatenate([r, [0, 1, shape.n_out - 2, shape.n_out - 1]])).astype(np.int32)
+
+
+ALL_SHAPES = [(name, s) for name, shapes in synth.workloads().items() for s in shapes]
+
+
+@pytest.mark.parametrize("name,shape", ALL_SHAPES, ids=[f"{n}:{s.key}:B{s.batch}" for n, s in ALL_SHAPES])
+def test_workload_parity(B, orc, name, shape):
+    """Every workload shape at full size, in the launch configuration the
+    benchmark times; rows sampled where the oracle would take too long."""
+    L = synth.layer_for(shape)
+    x = synth.x_for(shape)
+    y = gpu_gemv(B, upload(B, L), x)
+    rows = _rows_for(shape)
+    y_ref, bound = orc.gemv_layer(L, x, rows=rows)
+    yg = y if rows is None else y[:, rows]
+    assert_close(yg, y_ref, bound, shape.key)
+
+
+def test_deterministic_and_batch_independent(B):
+    shape = synth.workloads()["llama7b-up-3bit"][0]
+    L = synth.layer_for(shape)
+    layer = upload(B, L)
+    x = synth.make_x(16, shape.k_in, seed=5, key="det")
+    y16 = gpu_gemv(B, layer, x)
+    assert np.array_equal(y16, gpu_gemv(B, layer, x))
+    for b in (0, 7, 15):
+        y1 = gpu_gemv(B, layer, x[b:b + 1])
+        assert np.array_equal(y1[0], y16[b])
+
+
+def test_host_entry_point_matches_device(B):
+    shape = synth.workloads()["llama7b-q-4bit"][0]
+    L = synth.layer_for(shape)
+    layer = upload(B, L)
+    x = synth.make_x(4, shape.k_in, seed=8)
+    yd = gpu_gemv(B, layer, x)
+    xh = torch.from_numpy(x.view(np.int16).copy()).pin_memory()
+    yh = torch.zeros((4, shape.n_out), dtype=torch.int16).pin_memory()
+    B.sqz_gemv_host(layer, xh, yh)
+    assert np.array_equal(yh.numpy().view(np.uint16), yd)
+
+
+def test_non_default_stream(B, orc):
+    L = make_small(21, 500, 2048, 3, 400)
+    x = synth.make_x(2, 2048, seed=9)
+    layer = upload(B, L)
+    s = torch.cuda.Stream()
+    xd = torch.from_numpy(x.view(np.int16)).cuda()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(s):
+        yd = torch.empty((2, 500), dtype=torch.int16, device="cuda")
+        B.sqz_gemv(layer, xd, yd, stream=s)
+    s.synchronize()
+    y_ref, bound = orc.gemv_layer(L, x)
+    assert_close(yd.cpu().numpy().view(np.uint16), y_ref, bound)
+
+
+@pytest.mark.parametrize("case", ["rowptr0", "decreasing", "end", "col_high", "col_neg"])
+def test_malformed_csr_rejected_on_device(B, case):
+    L = make_small(31, 10, 64, 3, 12)
+    rowptr, col = L.rowptr.copy(), L.col.copy()
+    if case == "rowptr0":
+        rowptr[0] = 1
+    elif case == "decreasing":
+        rowptr[5] = rowptr[6] + 1
+    elif case == "end":
+        rowptr[-1] -= 1
+    elif case == "col_high":
+        col[3] = 64
+    else:
+        col[0] = -1
+    with pytest.raises(B.SqzError) as ei:
+        B.create_layer_from_numpy(10, 64, 3, L.codes, L.lut, rowptr, col, L.val)
+    assert ei.value.status == B.SQZ_ERR_INVALID_ARG
+
+
+def test_invalid_gemv_args(B):
+    L = make_small(41, 8, 64, 4, 3)
+    layer = upload(B, L)
+    x = torch.zeros((17, 64), dtype=torch.int16, device="cuda")
+    y = torch.zeros((17, 8), dtype=torch.int16, device="cuda")
+    with pytest.raises(B.SqzError):
+        B.sqz_gemv(layer, x, y)  # batch 17
+    with pytest.raises(B.SqzError):
+        B.sqz_gemv(layer, x[:2, :63], y[:2])  # ldx < K
+
+
+def test_fp16_yardstick(B, orc):
+    L = make_small(51, 333, 1032, 4, 0)
+    w = orc.dequant(L.codes, L.lut, L.n_out, L.k_in, 4)
+    x = synth.make_x(3, 1032, seed=3)
+    ref = f16_val(x) @ f16_val(w).T
+    bound = np.abs(f16_val(x)) @ np.abs(f16_val(w)).T
+    wd = torch.from_numpy(w.view(np.int16)).cuda()
+    xd = torch.from_numpy(x.view(np.int16)).cuda()
+    yd = torch.empty((3, 333), dtype=torch.int16, device="cuda")
+    B.sqz_fp16_gemv(wd, xd, yd)
+    torch.cuda.synchronize()
+    assert_close(yd.cpu().numpy().view(np.uint16), ref, bound)
