@@ -181,9 +181,20 @@ def sqz_create_layer(n_out: int, k_in: int, bits: int, codes: torch.Tensor, lut:
     return Layer(out.value, n_out, k_in, bits, nnz)
 
 
+def _check_shapes(layer: Layer, x: torch.Tensor, y: torch.Tensor, batch: int) -> None:
+    rows_x = x.shape[0] if x.dim() == 2 else 1
+    rows_y = y.shape[0] if y.dim() == 2 else 1
+    if x.shape[-1] < layer.k_in or y.shape[-1] < layer.n_out:
+        raise ValueError(f"x needs >= {layer.k_in} columns and y >= {layer.n_out} (got {tuple(x.shape)}, "
+                         f"{tuple(y.shape)})")
+    if batch > rows_x or batch > rows_y:
+        raise ValueError(f"batch {batch} exceeds the rows of x {tuple(x.shape)} or y {tuple(y.shape)}")
+
+
 def sqz_gemv(layer: Layer, x: torch.Tensor, y: torch.Tensor, batch: Optional[int] = None, stream=None) -> None:
     """y[b, :N] = (Q + S) x[b, :K] for b < batch (device tensors, fp16)."""
     batch = (x.shape[0] if x.dim() == 2 else 1) if batch is None else batch
+    _check_shapes(layer, x, y, batch)
     _check(lib().sqz_gemv(layer, _dptr_any(x, "x"), batch, _lead(x, "x"), _dptr_any(y, "y"), _lead(y, "y"),
                           _stream(stream)), "sqz_gemv")
 
@@ -199,6 +210,7 @@ def _dptr_any(t: torch.Tensor, name: str) -> Optional[int]:
 def sqz_gemv_host(layer: Layer, x: torch.Tensor, y: torch.Tensor, batch: Optional[int] = None, stream=None) -> None:
     """Host-memory variant: x and y are CPU tensors (pinned for async copies)."""
     batch = (x.shape[0] if x.dim() == 2 else 1) if batch is None else batch
+    _check_shapes(layer, x, y, batch)
     _check(lib().sqz_gemv_host(layer, _hptr(x, "x"), batch, _lead(x, "x"), _hptr(y, "y"), _lead(y, "y"),
                                _stream(stream)), "sqz_gemv_host")
 

@@ -233,8 +233,12 @@ def test_invalid_gemv_args(B):
     y = torch.zeros((17, 8), dtype=torch.int16, device="cuda")
     with pytest.raises(B.SqzError):
         B.sqz_gemv(layer, x, y)  # batch 17
-    with pytest.raises(B.SqzError):
-        B.sqz_gemv(layer, x[:2, :63], y[:2])  # ldx < K
+    st = B.lib().sqz_gemv(layer, x.data_ptr(), 2, 63, y.data_ptr(), 8, None)  # ldx < K
+    assert st == B.SQZ_ERR_INVALID_ARG
+    st = B.lib().sqz_gemv(layer, x.data_ptr(), 2, 64, y.data_ptr(), 7, None)  # ldy < N
+    assert st == B.SQZ_ERR_INVALID_ARG
+    with pytest.raises(ValueError):
+        B.sqz_gemv(layer, x[:2, :63], y[:2])  # the binding checks tensor widths
 
 
 def test_fp16_yardstick(B, orc):
