@@ -31,7 +31,7 @@ STATUS_NAMES = {0: "SQZ_OK", 1: "SQZ_ERR_INVALID_ARG", 2: "SQZ_ERR_UNSUPPORTED",
 
 # Every entry point include/sqz.h declares.
 EXPORTED = ("sqz_create_layer", "sqz_gemv", "sqz_gemv_host", "sqz_debug_dequant", "sqz_layer_info",
-            "sqz_destroy", "sqz_fp16_gemv", "sqz_last_error", "sqz_version")
+            "sqz_destroy", "sqz_fp16_gemv", "sqz_last_error", "sqz_version", "sqz_check_csr_static")
 
 
 class SqzError(RuntimeError):
@@ -76,6 +76,8 @@ def lib() -> ctypes.CDLL:
         for name in ("sqz_create_layer", "sqz_gemv", "sqz_gemv_host", "sqz_debug_dequant", "sqz_layer_info",
                      "sqz_destroy", "sqz_fp16_gemv"):
             getattr(L, name).restype = ctypes.c_int
+        L.sqz_check_csr_static.argtypes = [P, P, i32, i32, i64, P, ctypes.POINTER(i32)]
+        L.sqz_check_csr_static.restype = ctypes.c_int
         L.sqz_last_error.argtypes = []
         L.sqz_last_error.restype = ctypes.c_char_p
         L.sqz_version.argtypes = []
@@ -264,3 +266,14 @@ def create_layer_from_numpy(n_out: int, k_in: int, bits: int, codes, lut, rowptr
     layer = sqz_create_layer(n_out, k_in, bits, t_codes, t_lut, t_rp, t_col, t_val, stream=stream)
     torch.cuda.current_stream(dev).synchronize()
     return layer
+
+
+def sqz_check_csr_static(rowptr: Optional[torch.Tensor], col: Optional[torch.Tensor], n_out: int, k_in: int,
+                         stream=None) -> int:
+    """CSR check without device allocation; returns the flag word (0 = well formed)."""
+    nnz = 0 if col is None else int(col.numel())
+    flags = ctypes.c_int32(-1)
+    _check(lib().sqz_check_csr_static(_dptr(rowptr, "rowptr", (torch.int32,)), _dptr(col, "col", (torch.int32,)),
+                                      n_out, k_in, nnz, _stream(stream), ctypes.byref(flags)),
+           "sqz_check_csr_static")
+    return int(flags.value)

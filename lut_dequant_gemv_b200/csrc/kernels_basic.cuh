@@ -17,8 +17,9 @@ namespace sqz {
 
 // ---------------------------------------------------------------- CSR check
 // Sets bits of *flag: 1 rowptr[0] != 0, 2 rowptr[N] != nnz, 4 rowptr
-// decreasing, 8 column outside [0, K).
-__global__ void validate_csr_kernel(const int32_t* __restrict__ rowptr, const int32_t* __restrict__ col,
+// decreasing, 8 column outside [0, K).  Internal linkage: every
+// translation unit that launches it gets its own copy.
+static __global__ void validate_csr_kernel(const int32_t* __restrict__ rowptr, const int32_t* __restrict__ col,
                                     int32_t n_out, int32_t k_in, int64_t nnz, int* __restrict__ flag) {
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     const int64_t t0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;

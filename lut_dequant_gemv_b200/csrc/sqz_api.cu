@@ -336,6 +336,14 @@ sqz_status sqz_fp16_gemv(const uint16_t* w, int32_t n_out, int32_t k_in, int64_t
 
 const char* sqz_last_error(void) { return g_last_error.c_str(); }
 
+}  // extern "C"
+
+// Lets other translation units of the library report a message through
+// sqz_last_error(); not exported.
+void sqz_internal_set_last_error(const char* msg) { g_last_error = msg ? msg : ""; }
+
+extern "C" {
+
 int32_t sqz_version(void) { return 100; }
 
 }  // extern "C"
