@@ -143,6 +143,29 @@ SQZ_API sqz_status sqz_gemv_host(sqz_layer_t layer, const uint16_t* x_host, int3
  */
 SQZ_API sqz_status sqz_debug_dequant(sqz_layer_t layer, uint16_t* w_out, void* stream);
 
+/* Multiply-accumulate unit of the fused kernel (sqz_layer_set_mac). */
+#define SQZ_MAC_TENSOR_CORES 0 /* mma.sync m16n8k16, fp32 accumulate (default)       */
+#define SQZ_MAC_CUDA_CORES 1   /* fma.rn.f32.f16 on the CUDA cores, batch 1 only    */
+
+/*
+ * Choose the unit that performs the multiply-accumulates of the dense part.
+ * Both give results within the same bound; the CUDA-core variant exists to
+ * compare the two on the same decode and data path (it applies to batch-1
+ * calls; other batches keep the tensor cores).  Not thread-safe against
+ * concurrent sqz_gemv calls on the same handle.
+ * Errors: SQZ_ERR_INVALID_ARG.
+ */
+SQZ_API sqz_status sqz_layer_set_mac(sqz_layer_t layer, int32_t mac);
+
+/*
+ * Read and clear the handle's device status word, ordered on `stream`
+ * (synchronises it).  0 means every call so far completed normally; bit 0
+ * (1) means a bounded wait for a copy into shared memory gave up, in which
+ * case the outputs of the affected call are not valid.
+ * Errors: SQZ_ERR_INVALID_ARG, SQZ_ERR_CUDA.
+ */
+SQZ_API sqz_status sqz_layer_status(sqz_layer_t layer, void* stream, int32_t* status);
+
 /* Sizes of a handle (any output pointer may be NULL). */
 SQZ_API sqz_status sqz_layer_info(sqz_layer_t layer, int32_t* n_out, int32_t* k_in, int32_t* bits, int64_t* nnz,
                           int64_t* device_bytes);

@@ -25,13 +25,16 @@ SQZ_ERR_CUDA = 3
 SQZ_ERR_OOM = 4
 SQZ_ERR_TIMEOUT = 5
 SQZ_MAX_BATCH = 16
+SQZ_MAC_TENSOR_CORES = 0
+SQZ_MAC_CUDA_CORES = 1
 
 STATUS_NAMES = {0: "SQZ_OK", 1: "SQZ_ERR_INVALID_ARG", 2: "SQZ_ERR_UNSUPPORTED", 3: "SQZ_ERR_CUDA",
                 4: "SQZ_ERR_OOM", 5: "SQZ_ERR_TIMEOUT"}
 
 # Every entry point include/sqz.h declares.
 EXPORTED = ("sqz_create_layer", "sqz_gemv", "sqz_gemv_host", "sqz_debug_dequant", "sqz_layer_info",
-            "sqz_destroy", "sqz_fp16_gemv", "sqz_last_error", "sqz_version", "sqz_check_csr_static")
+            "sqz_destroy", "sqz_fp16_gemv", "sqz_last_error", "sqz_version", "sqz_check_csr_static",
+            "sqz_layer_set_mac", "sqz_layer_status")
 
 
 class SqzError(RuntimeError):
@@ -76,6 +79,10 @@ def lib() -> ctypes.CDLL:
         for name in ("sqz_create_layer", "sqz_gemv", "sqz_gemv_host", "sqz_debug_dequant", "sqz_layer_info",
                      "sqz_destroy", "sqz_fp16_gemv"):
             getattr(L, name).restype = ctypes.c_int
+        L.sqz_layer_set_mac.argtypes = [P, i32]
+        L.sqz_layer_set_mac.restype = ctypes.c_int
+        L.sqz_layer_status.argtypes = [P, P, ctypes.POINTER(i32)]
+        L.sqz_layer_status.restype = ctypes.c_int
         L.sqz_check_csr_static.argtypes = [P, P, i32, i32, i64, P, ctypes.POINTER(i32)]
         L.sqz_check_csr_static.restype = ctypes.c_int
         L.sqz_last_error.argtypes = []
@@ -277,3 +284,13 @@ def sqz_check_csr_static(rowptr: Optional[torch.Tensor], col: Optional[torch.Ten
                                       n_out, k_in, nnz, _stream(stream), ctypes.byref(flags)),
            "sqz_check_csr_static")
     return int(flags.value)
+
+
+def sqz_layer_set_mac(layer: Layer, mac: int) -> None:
+    _check(lib().sqz_layer_set_mac(layer, int(mac)), "sqz_layer_set_mac")
+
+
+def sqz_layer_status(layer: Layer, stream=None) -> int:
+    st = ctypes.c_int32(-1)
+    _check(lib().sqz_layer_status(layer, _stream(stream), ctypes.byref(st)), "sqz_layer_status")
+    return int(st.value)

@@ -11,9 +11,11 @@
 #include <cstring>
 #include <new>
 #include <string>
+#include <vector>
 
 #include "../../include/sqz.h"
 #include "kernels_basic.cuh"
+#include "kernels_tc.cuh"
 
 namespace {
 
@@ -52,21 +54,50 @@ int sm_count_of_current_device() {
     return n;
 }
 
+int max_smem_optin() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 232448;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess || n <= 0)
+        return 232448;
+    return n;
+}
+
+constexpr int kDefaultStages = 6;
+
 }  // namespace
 
 struct sqz_layer {
     int32_t n_out = 0, k_in = 0, bits = 0;
     int64_t nnz = 0;
-    int64_t wpr = 0;  // 32-bit words per row of codes
+    int64_t wpr = 0;  // 32-bit words per row of canonical codes
     int device = 0;
     int sm_count = 148;
+    int smem_optin = 232448;
+    int mac = SQZ_MAC_TENSOR_CORES;
+    // The fused kernel works on whole k16-steps: K % 16 == 0 (4-bit layers
+    // with K % 16 == 8 use the row-per-warp kernel).
+    bool fused_ok = false;
+    // canonical copies (row-per-warp kernel for requests the fused kernel
+    // cannot stage in shared memory)
     uint32_t* codes = nullptr;
     uint16_t* lut = nullptr;
+    // CSR copies, padded by 8 elements so that 16-byte aligned bulk copies
+    // of any slice stay inside the allocation
     int32_t* rowptr = nullptr;
     int32_t* col = nullptr;
     uint16_t* val = nullptr;
-    uint16_t* x_stage = nullptr;  // [SQZ_MAX_BATCH][k_in] for sqz_gemv_host
-    uint16_t* y_stage = nullptr;  // [SQZ_MAX_BATCH][n_out]
+    // kernel-native layout for the fused kernel
+    int ntiles = 0, nsteps = 0, nsg = 0;
+    int64_t units = 0;
+    int grid = 0;
+    uint8_t* codes_native = nullptr;  // [ntiles][nsg][sg_bytes]
+    uint8_t* lut_native = nullptr;    // [ntiles*16][2 << bits] byte planes
+    float* part = nullptr;            // [grid][2][16][16]
+    int* tile_cnt = nullptr;          // [ntiles], zero between calls
+    int* status = nullptr;            // [1]
+    std::vector<int> csr_rp;          // [grid+1]
+    uint16_t* x_stage = nullptr;      // [SQZ_MAX_BATCH][k_in] for sqz_gemv_host
+    uint16_t* y_stage = nullptr;      // [SQZ_MAX_BATCH][n_out]
     int64_t device_bytes = 0;
 };
 
@@ -79,6 +110,11 @@ void free_layer(sqz_layer* L) {
     cudaFree(L->rowptr);
     cudaFree(L->col);
     cudaFree(L->val);
+    cudaFree(L->codes_native);
+    cudaFree(L->lut_native);
+    cudaFree(L->part);
+    cudaFree(L->tile_cnt);
+    cudaFree(L->status);
     cudaFree(L->x_stage);
     cudaFree(L->y_stage);
     delete L;
@@ -100,7 +136,8 @@ sqz_status alloc(T** p, size_t count, sqz_layer* L, const char* what) {
 
 sqz_status check_desc(const sqz_layer_desc* d) {
     if (d->bits != 3 && d->bits != 4) return fail(SQZ_ERR_INVALID_ARG, "bits must be 3 or 4 (got %d)", d->bits);
-    if (d->n_out < 0 || d->k_in < 0) return fail(SQZ_ERR_INVALID_ARG, "negative size (n_out=%d, k_in=%d)", d->n_out, d->k_in);
+    if (d->n_out < 0 || d->k_in < 0)
+        return fail(SQZ_ERR_INVALID_ARG, "negative size (n_out=%d, k_in=%d)", d->n_out, d->k_in);
     const int kmult = d->bits == 3 ? 32 : 8;
     if (d->k_in % kmult != 0)
         return fail(SQZ_ERR_INVALID_ARG, "k_in=%d must be a multiple of %d for %d-bit codes (whole words per row)",
@@ -111,6 +148,7 @@ sqz_status check_desc(const sqz_layer_desc* d) {
     if (d->nnz > 0 && (!d->rowptr || !d->col || !d->val))
         return fail(SQZ_ERR_INVALID_ARG, "nnz=%lld but rowptr/col/val is NULL", (long long)d->nnz);
     if (d->nnz > 0 && d->k_in == 0) return fail(SQZ_ERR_INVALID_ARG, "nnz > 0 with k_in == 0");
+    if (d->n_out >= INT32_MAX - 16) return fail(SQZ_ERR_INVALID_ARG, "n_out too large");
     return SQZ_OK;
 }
 
@@ -125,6 +163,7 @@ sqz_status check_gemv_args(const sqz_layer* L, const void* x, int32_t batch, int
     return SQZ_OK;
 }
 
+// ------------------------------------------------------------ row per warp
 template <int BITS, int B>
 void launch_rowwarp(const sqz_layer* L, const uint16_t* x, int64_t ldx, uint16_t* y, int64_t ldy, cudaStream_t s) {
     const int64_t blocks = (L->n_out + 7) / 8;
@@ -134,8 +173,8 @@ void launch_rowwarp(const sqz_layer* L, const uint16_t* x, int64_t ldx, uint16_t
 }
 
 template <int BITS>
-void dispatch_batch(const sqz_layer* L, const uint16_t* x, int32_t batch, int64_t ldx, uint16_t* y, int64_t ldy,
-                    cudaStream_t s) {
+void dispatch_rowwarp(const sqz_layer* L, const uint16_t* x, int32_t batch, int64_t ldx, uint16_t* y, int64_t ldy,
+                      cudaStream_t s) {
     switch (batch) {
 #define SQZ_CASE(B) \
     case B: launch_rowwarp<BITS, B>(L, x, ldx, y, ldy, s); break;
@@ -146,14 +185,148 @@ void dispatch_batch(const sqz_layer* L, const uint16_t* x, int32_t batch, int64_
     }
 }
 
+// ------------------------------------------------------------ fused kernel
+template <int BITS, int NT, bool TC>
+sqz_status set_smem_attr(int bytes) {
+    SQZ_CUDA_TRY(cudaFuncSetAttribute(sqz::tc::gemv_fused_kernel<BITS, NT, TC>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, bytes),
+                 "cudaFuncSetAttribute");
+    return SQZ_OK;
+}
+
+sqz_status prepare_fused_kernels(int optin) {
+    sqz_status st;
+    if ((st = set_smem_attr<3, 1, true>(optin)) != SQZ_OK) return st;
+    if ((st = set_smem_attr<3, 2, true>(optin)) != SQZ_OK) return st;
+    if ((st = set_smem_attr<4, 1, true>(optin)) != SQZ_OK) return st;
+    if ((st = set_smem_attr<4, 2, true>(optin)) != SQZ_OK) return st;
+    if ((st = set_smem_attr<3, 1, false>(optin)) != SQZ_OK) return st;
+    if ((st = set_smem_attr<4, 1, false>(optin)) != SQZ_OK) return st;
+    return SQZ_OK;
+}
+
+// Plan for a call, or false when the fused kernel cannot stage x.
+bool fused_plan(const sqz_layer* L, int batch, sqz::tc::Plan* out) {
+    const int nt = batch > 8 ? 2 : 1;
+    for (int stages = kDefaultStages; stages >= 2; --stages) {
+        sqz::tc::Plan P = sqz::tc::make_plan(L->bits, L->n_out, L->k_in, batch, nt, L->sm_count, stages);
+        if (P.total <= L->smem_optin) {
+            *out = P;
+            return P.grid == L->grid;
+        }
+    }
+    return false;
+}
+
+template <int BITS, int NT, bool TC>
+void launch_fused(const sqz::tc::Params& prm, cudaStream_t s) {
+    sqz::tc::gemv_fused_kernel<BITS, NT, TC>
+        <<<prm.plan.grid, sqz::tc::kThreads, prm.plan.total, s>>>(prm);
+}
+
 sqz_status gemv_impl(const sqz_layer* L, const uint16_t* x, int32_t batch, int64_t ldx, uint16_t* y, int64_t ldy,
                      cudaStream_t s) {
     if (L->n_out == 0) return SQZ_OK;
-    if (L->bits == 3)
-        dispatch_batch<3>(L, x, batch, ldx, y, ldy, s);
-    else
-        dispatch_batch<4>(L, x, batch, ldx, y, ldy, s);
+    sqz::tc::Plan P;
+    if (L->fused_ok && fused_plan(L, batch, &P)) {
+        sqz::tc::Params prm{};
+        prm.codes = L->codes_native;
+        prm.lutp = L->lut_native;
+        prm.rowptr = L->rowptr;
+        prm.col = L->col;
+        prm.val = L->val;
+        prm.nnz = L->nnz;
+        prm.x = x;
+        prm.ldx = ldx;
+        prm.y = y;
+        prm.ldy = ldy;
+        prm.part = L->part;
+        prm.tile_cnt = L->tile_cnt;
+        prm.status = L->status;
+        prm.n_out = L->n_out;
+        prm.k_in = L->k_in;
+        prm.nsteps = L->nsteps;
+        prm.nsg = L->nsg;
+        prm.ntiles = L->ntiles;
+        prm.batch = batch;
+        prm.x_bulk = (reinterpret_cast<uintptr_t>(x) % 16 == 0) && (ldx % 8 == 0) && (L->k_in % 8 == 0);
+        prm.plan = P;
+        for (int c = 0; c <= L->grid; ++c) prm.csr_rp[c] = L->csr_rp[c];
+        const bool cuda_cores = L->mac == SQZ_MAC_CUDA_CORES && batch == 1;
+        if (L->bits == 3) {
+            if (cuda_cores) launch_fused<3, 1, false>(prm, s);
+            else if (batch > 8) launch_fused<3, 2, true>(prm, s);
+            else launch_fused<3, 1, true>(prm, s);
+        } else {
+            if (cuda_cores) launch_fused<4, 1, false>(prm, s);
+            else if (batch > 8) launch_fused<4, 2, true>(prm, s);
+            else launch_fused<4, 1, true>(prm, s);
+        }
+    } else if (L->bits == 3) {
+        dispatch_rowwarp<3>(L, x, batch, ldx, y, ldy, s);
+    } else {
+        dispatch_rowwarp<4>(L, x, batch, ldx, y, ldy, s);
+    }
     SQZ_CUDA_TRY(cudaGetLastError(), "gemv launch");
+    return SQZ_OK;
+}
+
+// Kernel-native copies of codes and LUT, scratch of the fused kernel, and
+// the per-CTA CSR bounds.  `h_rowptr` is the host copy of rowptr (or empty).
+sqz_status build_native(sqz_layer* L, const std::vector<int32_t>& h_rowptr, cudaStream_t s) {
+    using namespace sqz::tc;
+    L->ntiles = (L->n_out + kTileRows - 1) / kTileRows;
+    L->nsteps = L->k_in / 16;
+    L->nsg = (L->nsteps + kSgSteps - 1) / kSgSteps;
+    L->units = (int64_t)L->ntiles * L->nsg;
+    const Plan P = make_plan(L->bits, L->n_out, L->k_in, 1, 1, L->sm_count, kDefaultStages);
+    L->grid = P.grid;
+    if (L->grid > kMaxGrid) return fail(SQZ_ERR_UNSUPPORTED, "more than %d SMs", kMaxGrid);
+    const int sg_bytes = L->bits == 3 ? 1536 : 2048;
+    const int lut_row = 2 << L->bits;
+    sqz_status st;
+    if ((st = alloc(&L->codes_native, (size_t)L->units * sg_bytes, L, "native codes")) != SQZ_OK) return st;
+    if ((st = alloc(&L->lut_native, (size_t)L->ntiles * kTileRows * lut_row, L, "native lut")) != SQZ_OK) return st;
+    if ((st = alloc(&L->part, (size_t)L->grid * 2 * kTileRows * 16, L, "partials")) != SQZ_OK) return st;
+    if ((st = alloc(&L->tile_cnt, (size_t)(L->ntiles > 0 ? L->ntiles : 1), L, "tile counters")) != SQZ_OK) return st;
+    if ((st = alloc(&L->status, 1, L, "status")) != SQZ_OK) return st;
+    if (L->tile_cnt) SQZ_CUDA_TRY(cudaMemsetAsync(L->tile_cnt, 0, sizeof(int) * (L->ntiles > 0 ? L->ntiles : 1), s), "memset");
+    SQZ_CUDA_TRY(cudaMemsetAsync(L->status, 0, sizeof(int), s), "memset");
+    if (L->units > 0) {
+        const int64_t words = L->units * (sg_bytes / 4);
+        int64_t blocks = (words + 255) / 256;
+        if (blocks > (int64_t)L->sm_count * 16) blocks = (int64_t)L->sm_count * 16;
+        if (L->bits == 3)
+            sqz::tc::repack_codes_kernel<3><<<(unsigned)blocks, 256, 0, s>>>(L->codes, L->n_out, L->k_in, L->nsg,
+                                                                             words,
+                                                                             reinterpret_cast<uint32_t*>(L->codes_native));
+        else
+            sqz::tc::repack_codes_kernel<4><<<(unsigned)blocks, 256, 0, s>>>(L->codes, L->n_out, L->k_in, L->nsg,
+                                                                             words,
+                                                                             reinterpret_cast<uint32_t*>(L->codes_native));
+        SQZ_CUDA_TRY(cudaGetLastError(), "repack codes");
+    }
+    if (L->ntiles > 0) {
+        const int rows = L->ntiles * kTileRows;
+        const int blocks = (rows + 255) / 256;
+        if (L->bits == 3)
+            sqz::tc::repack_lut_kernel<3><<<blocks, 256, 0, s>>>(L->lut, L->n_out, rows, L->lut_native);
+        else
+            sqz::tc::repack_lut_kernel<4><<<blocks, 256, 0, s>>>(L->lut, L->n_out, rows, L->lut_native);
+        SQZ_CUDA_TRY(cudaGetLastError(), "repack lut");
+    }
+    // CSR entries owned by each CTA: rows of the tiles whose first unit is in
+    // the CTA's unit range.
+    L->csr_rp.assign(L->grid + 1, 0);
+    for (int c = 0; c <= L->grid; ++c) {
+        int ra = L->n_out;
+        if (c < L->grid && L->units > 0) {
+            const int64_t u0 = L->units * c / L->grid;
+            const int64_t ta = (u0 + L->nsg - 1) / L->nsg;
+            ra = (int)(ta * kTileRows < L->n_out ? ta * kTileRows : L->n_out);
+        }
+        L->csr_rp[c] = h_rowptr.empty() ? 0 : h_rowptr[ra];
+    }
     return SQZ_OK;
 }
 
@@ -176,6 +349,7 @@ sqz_status sqz_create_layer(const sqz_layer_desc* desc, void* stream, sqz_layer_
     L->nnz = desc->nnz;
     L->wpr = (int64_t)desc->k_in * desc->bits / 32;
     L->sm_count = sm_count_of_current_device();
+    L->smem_optin = max_smem_optin();
     cudaGetDevice(&L->device);
 
     const size_t n = (size_t)desc->n_out, lut_n = n << desc->bits, code_n = n * (size_t)L->wpr;
@@ -198,12 +372,14 @@ sqz_status sqz_create_layer(const sqz_layer_desc* desc, void* stream, sqz_layer_
         }                                       \
     } while (0)
 
+    SQZ_STEP(prepare_fused_kernels(L->smem_optin));
     SQZ_STEP(alloc(&L->codes, code_n, L, "codes allocation"));
     SQZ_STEP(alloc(&L->lut, lut_n, L, "lut allocation"));
+    std::vector<int32_t> h_rowptr;
     if (nnz > 0) {
-        SQZ_STEP(alloc(&L->rowptr, n + 1, L, "rowptr allocation"));
-        SQZ_STEP(alloc(&L->col, nnz, L, "col allocation"));
-        SQZ_STEP(alloc(&L->val, nnz, L, "val allocation"));
+        SQZ_STEP(alloc(&L->rowptr, n + 1 + 8, L, "rowptr allocation"));
+        SQZ_STEP(alloc(&L->col, nnz + 8, L, "col allocation"));
+        SQZ_STEP(alloc(&L->val, nnz + 8, L, "val allocation"));
     }
     SQZ_STEP(alloc(&L->x_stage, (size_t)SQZ_MAX_BATCH * desc->k_in, L, "x staging allocation"));
     SQZ_STEP(alloc(&L->y_stage, (size_t)SQZ_MAX_BATCH * n, L, "y staging allocation"));
@@ -213,6 +389,9 @@ sqz_status sqz_create_layer(const sqz_layer_desc* desc, void* stream, sqz_layer_
     if (lut_n)
         SQZ_CUDA_STEP(cudaMemcpyAsync(L->lut, desc->lut, lut_n * 2, cudaMemcpyDeviceToDevice, s), "lut copy");
     if (nnz > 0) {
+        SQZ_CUDA_STEP(cudaMemsetAsync(L->rowptr, 0, (n + 1 + 8) * 4, s), "rowptr clear");
+        SQZ_CUDA_STEP(cudaMemsetAsync(L->col, 0, (nnz + 8) * 4, s), "col clear");
+        SQZ_CUDA_STEP(cudaMemsetAsync(L->val, 0, (nnz + 8) * 2, s), "val clear");
         SQZ_CUDA_STEP(cudaMemcpyAsync(L->rowptr, desc->rowptr, (n + 1) * 4, cudaMemcpyDeviceToDevice, s), "rowptr copy");
         SQZ_CUDA_STEP(cudaMemcpyAsync(L->col, desc->col, nnz * 4, cudaMemcpyDeviceToDevice, s), "col copy");
         SQZ_CUDA_STEP(cudaMemcpyAsync(L->val, desc->val, nnz * 2, cudaMemcpyDeviceToDevice, s), "val copy");
@@ -243,7 +422,12 @@ sqz_status sqz_create_layer(const sqz_layer_desc* desc, void* stream, sqz_layer_
                         (h_flag & 2) ? " rowptr[N]!=nnz" : "", (h_flag & 4) ? " rowptr decreasing" : "",
                         (h_flag & 8) ? " column outside [0,K)" : "");
         }
+        h_rowptr.resize(n + 1);
+        SQZ_CUDA_STEP(cudaMemcpy(h_rowptr.data(), L->rowptr, (n + 1) * 4, cudaMemcpyDeviceToHost), "rowptr readback");
     }
+    L->fused_ok = L->n_out > 0 && L->k_in > 0 && L->k_in % 16 == 0;
+    if (L->fused_ok) SQZ_STEP(build_native(L, h_rowptr, s));
+    SQZ_CUDA_STEP(cudaStreamSynchronize(s), "layer creation");
 #undef SQZ_STEP
 #undef SQZ_CUDA_STEP
     *out = L;
@@ -284,10 +468,17 @@ sqz_status sqz_debug_dequant(sqz_layer_t layer, uint16_t* w_out, void* stream) {
     if (!w_out) return fail(SQZ_ERR_INVALID_ARG, "w_out is NULL");
     cudaStream_t s = as_stream(stream);
     const int grid = L->sm_count * 4;
-    if (L->bits == 3)
-        sqz::dequant_canonical_kernel<3><<<grid, 256, 0, s>>>(L->codes, L->lut, L->n_out, L->k_in, w_out);
+    if (!L->fused_ok) {
+        if (L->bits == 3)
+            sqz::dequant_canonical_kernel<3><<<grid, 256, 0, s>>>(L->codes, L->lut, L->n_out, L->k_in, w_out);
+        else
+            sqz::dequant_canonical_kernel<4><<<grid, 256, 0, s>>>(L->codes, L->lut, L->n_out, L->k_in, w_out);
+    } else if (L->bits == 3)
+        sqz::tc::dequant_native_kernel<3><<<grid, 256, 0, s>>>(L->codes_native, L->lut_native, L->n_out, L->k_in,
+                                                               L->nsg, L->units, w_out);
     else
-        sqz::dequant_canonical_kernel<4><<<grid, 256, 0, s>>>(L->codes, L->lut, L->n_out, L->k_in, w_out);
+        sqz::tc::dequant_native_kernel<4><<<grid, 256, 0, s>>>(L->codes_native, L->lut_native, L->n_out, L->k_in,
+                                                               L->nsg, L->units, w_out);
     SQZ_CUDA_TRY(cudaGetLastError(), "dequant launch");
     return SQZ_OK;
 }
@@ -300,6 +491,27 @@ sqz_status sqz_layer_info(sqz_layer_t layer, int32_t* n_out, int32_t* k_in, int3
     if (bits) *bits = layer->bits;
     if (nnz) *nnz = layer->nnz;
     if (device_bytes) *device_bytes = layer->device_bytes;
+    return SQZ_OK;
+}
+
+sqz_status sqz_layer_set_mac(sqz_layer_t layer, int32_t mac) {
+    if (!layer) return fail(SQZ_ERR_INVALID_ARG, "layer is NULL");
+    if (mac != SQZ_MAC_TENSOR_CORES && mac != SQZ_MAC_CUDA_CORES)
+        return fail(SQZ_ERR_INVALID_ARG, "unknown MAC unit %d", mac);
+    layer->mac = mac;
+    return SQZ_OK;
+}
+
+sqz_status sqz_layer_status(sqz_layer_t layer, void* stream, int32_t* status) {
+    if (!layer || !status) return fail(SQZ_ERR_INVALID_ARG, "layer and status must be non-NULL");
+    *status = 0;
+    if (!layer->status) return SQZ_OK;
+    cudaStream_t s = as_stream(stream);
+    int h = 0;
+    SQZ_CUDA_TRY(cudaMemcpyAsync(&h, layer->status, sizeof(int), cudaMemcpyDeviceToHost, s), "status read");
+    SQZ_CUDA_TRY(cudaMemsetAsync(layer->status, 0, sizeof(int), s), "status clear");
+    SQZ_CUDA_TRY(cudaStreamSynchronize(s), "stream synchronize");
+    *status = h;
     return SQZ_OK;
 }
 
@@ -344,6 +556,6 @@ void sqz_internal_set_last_error(const char* msg) { g_last_error = msg ? msg : "
 
 extern "C" {
 
-int32_t sqz_version(void) { return 100; }
+int32_t sqz_version(void) { return 200; }
 
 }  // extern "C"

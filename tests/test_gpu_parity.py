@@ -253,3 +253,32 @@ def test_fp16_yardstick(B, orc):
     B.sqz_fp16_gemv(wd, xd, yd)
     torch.cuda.synchronize()
     assert_close(yd.cpu().numpy().view(np.uint16), ref, bound)
+
+
+@pytest.mark.parametrize("wl", ["llama7b-q-4bit", "llama7b-up-3bit"])
+def test_cuda_core_mac_matches_oracle(B, orc, wl):
+    """The CUDA-core multiply-accumulate variant (batch 1) meets the same
+    bound as the tensor-core one."""
+    shape = synth.workloads()[wl][0]
+    L = synth.layer_for(shape)
+    x = synth.x_for(shape)
+    layer = upload(B, L)
+    y_tc = gpu_gemv(B, layer, x)
+    B.sqz_layer_set_mac(layer, B.SQZ_MAC_CUDA_CORES)
+    y_cc = gpu_gemv(B, layer, x)
+    y_ref, bound = orc.gemv_layer(L, x)
+    assert_close(y_cc, y_ref, bound, "cuda cores")
+    assert_close(y_tc, y_ref, bound, "tensor cores")
+    assert B.sqz_layer_status(layer) == 0
+
+
+def test_status_word_clear_after_runs(B):
+    shape = synth.workloads()["llama65b-3bit-t3"][2]
+    L = synth.layer_for(shape)
+    layer = upload(B, L)
+    x = synth.x_for(shape)
+    for _ in range(3):
+        gpu_gemv(B, layer, x)
+    assert B.sqz_layer_status(layer) == 0
+    with pytest.raises(B.SqzError):
+        B.sqz_layer_set_mac(layer, 7)
