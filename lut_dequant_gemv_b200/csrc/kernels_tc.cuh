@@ -47,8 +47,9 @@
 namespace sqz {
 namespace tc {
 
-constexpr int kWarps = 8;
+constexpr int kWarps = 16;
 constexpr int kThreads = kWarps * 32;
+constexpr int kCsrThreads = 256;  // threads that share the sparse part
 constexpr int kTileRows = 16;
 constexpr int kSgSteps = 16;   // k16-steps per super-group
 constexpr int kSgCols = 256;   // columns per super-group
@@ -123,13 +124,13 @@ __host__ __device__ inline Plan make_plan(int bits, int n_out, int k_in, int bat
     P.off_val = off;
     off += (kCsrCap + 16) * 2;  // a slice starts up to 7 entries early and is rounded up to 8
     P.off_head = off;
-    off += kThreads * P.bmax * 4;
+    off += kCsrThreads * P.bmax * 4;
     P.off_tail = off;
-    off += kThreads * P.bmax * 4;
+    off += kCsrThreads * P.bmax * 4;
     P.off_headrow = off;
-    off += kThreads * 4;
+    off += kCsrThreads * 4;
     P.off_tailrow = off;
-    off += kThreads * 4;
+    off += kCsrThreads * 4;
     P.off_rowsum = off;
     off += round_up(csr_rows * P.bmax * 4, 128);
     P.off_ctile = off;
@@ -408,11 +409,11 @@ __global__ void dequant_native_kernel(const uint8_t* __restrict__ codes, const u
 }
 
 // ------------------------------------------------------------ main kernel
-__device__ __forceinline__ int64_t cta_begin(int64_t units, int grid, int c) { return units * c / grid; }
+__device__ __forceinline__ int cta_begin(int units, int grid, int c) { return (int)((int64_t)units * c / grid); }
 
 // CTA whose unit range contains u.
-__device__ __forceinline__ int cta_of(int64_t units, int grid, int64_t u) {
-    int c = (int)((u * grid) / units);
+__device__ __forceinline__ int cta_of(int units, int grid, int u) {
+    int c = (int)(((int64_t)u * grid) / units);
     while (c + 1 < grid && cta_begin(units, grid, c + 1) <= u) ++c;
     while (c > 0 && cta_begin(units, grid, c) > u) --c;
     return c;
@@ -422,18 +423,19 @@ template <int BITS, int NT, bool TC>
 __global__ void __launch_bounds__(kThreads, 1) gemv_fused_kernel(const __grid_constant__ Params p) {
     using F = Fmt<BITS>;
     using TAB = typename std::conditional<BITS == 3, Tab3, Tab4>::type;
-    constexpr int BM = 8 * NT;  // batch columns held per accumulator set
+    constexpr int BM = 8 * NT;             // batch columns per accumulator set
+    constexpr int TE = kTileRows * BM;      // elements of one tile's result
     extern __shared__ __align__(128) uint8_t smem[];
     const Plan& P = p.plan;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t4 = lane & 3;
     const int G = gridDim.x, c = blockIdx.x;
     const int nsg = p.nsg;
-    const int64_t U = P.units;
-    const int64_t u0 = cta_begin(U, G, c), u1 = cta_begin(U, G, c + 1);
-    const int64_t cn = u1 - u0;
-    const int64_t wu0 = u0 + cn * warp / kWarps, wu1 = u0 + cn * (warp + 1) / kWarps;
-    const int t_first = (int)(u0 / nsg), t_last = (int)((u1 - 1) / nsg);
+    const int U = (int)P.units;
+    const int u0 = cta_begin(U, G, c), u1 = cta_begin(U, G, c + 1);
+    const int cn = u1 - u0;
+    const int wu0 = u0 + cn * warp / kWarps, wu1 = u0 + cn * (warp + 1) / kWarps;
+    const int t_first = u0 / nsg, t_last = (u1 - 1) / nsg;
     const int ctiles = t_last - t_first + 1;
     const int stages = P.stages;
 
@@ -461,7 +463,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_fused_kernel(const __grid_co
 
     // ---- sparse rows owned by this CTA: those of the tiles whose first unit
     // lies in [u0, u1); their CSR entries are [csr_rp[c], csr_rp[c+1]).
-    const int ta = (int)((u0 + nsg - 1) / nsg), tb = t_last;
+    const int ta = (u0 + nsg - 1) / nsg, tb = t_last;
     const int ra = min(p.n_out, ta * kTileRows);
     const int nrows = ta <= tb ? min(p.n_out, (tb + 1) * kTileRows) - ra : 0;
     const int p0 = p.csr_rp[c], p1 = p.csr_rp[c + 1];
@@ -490,16 +492,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_fused_kernel(const __grid_co
         if (val_bytes) bulk_g2s(smem + P.off_val, p.val + (p0 - val_off), val_bytes, xbar);
     }
     // ---- per-warp ring prologue
-    const int64_t nwu = wu1 - wu0;
-    int issued = 0;
-    if (lane == 0) {
-        const int pre = (int)(nwu < stages ? nwu : stages);
-        for (int s = 0; s < pre; ++s) {
+    const int nwu = wu1 - wu0;
+    int issued = nwu < stages ? nwu : stages;
+    if (lane == 0)
+        for (int s = 0; s < issued; ++s) {
             mbar_expect_tx(&wbar[s], F::kSgBytes);
-            bulk_g2s(ring + s * F::kSgBytes, p.codes + (wu0 + s) * F::kSgBytes, F::kSgBytes, &wbar[s]);
+            bulk_g2s(ring + s * F::kSgBytes, p.codes + (int64_t)(wu0 + s) * F::kSgBytes, F::kSgBytes, &wbar[s]);
         }
-    }
-    issued = (int)(nwu < stages ? nwu : stages);
     if (!p.x_bulk) {
         for (int i = tid; i < p.batch * p.k_in; i += kThreads) {
             const int b = i / p.k_in, k = i - b * p.k_in;
@@ -508,10 +507,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_fused_kernel(const __grid_co
     }
     if (has_csr) {
         for (int i = tid; i < nrows * BM; i += kThreads) s_rowsum[i] = 0.f;
-        s_headrow[tid] = -1;
-        s_tailrow[tid] = -1;
+        if (tid < kCsrThreads) {
+            s_headrow[tid] = -1;
+            s_tailrow[tid] = -1;
+        }
     }
-    __syncthreads();  // x copied when not bulk; CSR bookkeeping initialised
     const bool ok = __syncthreads_and(mbar_wait(xbar, 0) ? 1 : 0) != 0;
     if (!ok && tid == 0) atomicOr(p.status, kStatusWaitTimeout);
 
@@ -519,9 +519,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_fused_kernel(const __grid_co
     const int B = p.batch;
     const int* s_rp = reinterpret_cast<const int*>(smem + P.off_rp) + rp_off;
     const int* csr_col = csr_smem ? reinterpret_cast<const int*>(smem + P.off_col) + col_off - p0 : p.col;
-    const uint16_t* csr_val = csr_smem ? reinterpret_cast<const uint16_t*>(smem + P.off_val) + val_off - p0 : p.val;
-    const int e_per = has_csr ? max(1, (nz + kThreads - 1) / kThreads) : 1;
-    if (has_csr && ok) {
+    const uint16_t* csr_val =
+        csr_smem ? reinterpret_cast<const uint16_t*>(smem + P.off_val) + val_off - p0 : p.val;
+    const int e_per = has_csr ? max(1, (nz + kCsrThreads - 1) / kCsrThreads) : 1;
+    if (has_csr && ok && tid < kCsrThreads) {
         const int a = p0 + tid * e_per;
         const int b_end = min(p1, a + e_per);
         if (a < b_end) {
@@ -583,13 +584,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_fused_kernel(const __grid_co
     const int xrow = (g < B) ? g : 0;  // batch column of this lane's B fragment (n = g)
     const int xrow2 = (NT == 2 && g + 8 < B) ? g + 8 : 0;
     const bool xon = g < B, xon2 = (NT == 2) && (g + 8 < B);
-    int64_t u = wu0;
-    int it = 0;  // ring use counter
+    const int wfirst = nwu > 0 ? wu0 / nsg : -1;
+    int tile = wfirst, sg = nwu > 0 ? wu0 - wfirst * nsg : 0;
+    int s = 0, consumed = 0;
+    uint32_t par = 0;
     bool alive = ok;
-    int fail_it = -1;
-    while (u < wu1) {
-        const int tile = (int)(u / nsg);
-        const int64_t run_end = min(wu1, (int64_t)(tile + 1) * nsg);
+    int fail_at = -1;
+    for (int u = wu0; u < wu1;) {
+        const int run = min(wu1 - u, nsg - sg);  // units of `tile` in this warp's range
         const uint8_t* lt = luts + (tile - t_first) * kTileRows * F::kLutBytes;
         TAB tg, tg8;
         if constexpr (BITS == 3) {
@@ -606,14 +608,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_fused_kernel(const __grid_co
             for (int i = 0; i < 4; ++i) d0[n][i] = d1[n][i] = 0.f;
         float f0 = 0.f, f1 = 0.f;  // CUDA-core accumulators (rows g, g+8)
 
-        for (; u < run_end; ++u, ++it) {
-            const int s = it % stages;
-            const uint32_t par = (uint32_t)(it / stages) & 1u;
+        for (int r = 0; r < run; ++r, ++sg, ++consumed) {
             if (alive) {
                 const bool got = __all_sync(0xffffffffu, mbar_wait(&wbar[s], par));
                 if (!got) {
                     alive = false;
-                    fail_it = it;
+                    fail_at = consumed;
                     if (lane == 0) atomicOr(p.status, kStatusWaitTimeout);
                 }
             }
@@ -625,16 +625,19 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_fused_kernel(const __grid_co
                 w[4 * m] = v.x, w[4 * m + 1] = v.y, w[4 * m + 2] = v.z, w[4 * m + 3] = v.w;
             }
             __syncwarp();
-            if (alive && it + stages < nwu) {
+            if (alive && issued < nwu) {
                 if (lane == 0) {
                     fence_proxy_async();
                     mbar_expect_tx(&wbar[s], F::kSgBytes);
-                    bulk_g2s(ring + s * F::kSgBytes, p.codes + (wu0 + it + stages) * F::kSgBytes, F::kSgBytes,
+                    bulk_g2s(ring + s * F::kSgBytes, p.codes + (int64_t)(wu0 + issued) * F::kSgBytes, F::kSgBytes,
                              &wbar[s]);
                 }
-                issued = it + stages + 1;
+                ++issued;
             }
-            const int sg = (int)(u % nsg);
+            if (++s == stages) {
+                s = 0;
+                par ^= 1u;
+            }
             const int step0 = sg * kSgSteps;
             const int nvalid = min(kSgSteps, p.nsteps - step0);
             const uint16_t* xb0 = xs + xrow * P.x_stride + step0 * 16 + 4 * t4;
@@ -667,43 +670,43 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_fused_kernel(const __grid_co
             }
         }
         // ---- this warp's contribution to `tile`
-        float r[NT][4];
+        float rr[NT][4];
         if constexpr (TC) {
 #pragma unroll
             for (int n = 0; n < NT; ++n)
 #pragma unroll
-                for (int i = 0; i < 4; ++i) r[n][i] = d0[n][i] + d1[n][i];
+                for (int i = 0; i < 4; ++i) rr[n][i] = d0[n][i] + d1[n][i];
         } else {
             f0 += __shfl_xor_sync(0xffffffffu, f0, 1);
             f0 += __shfl_xor_sync(0xffffffffu, f0, 2);
             f1 += __shfl_xor_sync(0xffffffffu, f1, 1);
             f1 += __shfl_xor_sync(0xffffffffu, f1, 2);
-            r[0][0] = t4 == 0 ? f0 : 0.f;
-            r[0][1] = 0.f;
-            r[0][2] = t4 == 0 ? f1 : 0.f;
-            r[0][3] = 0.f;
+            rr[0][0] = t4 == 0 ? f0 : 0.f;
+            rr[0][1] = 0.f;
+            rr[0][2] = t4 == 0 ? f1 : 0.f;
+            rr[0][3] = 0.f;
         }
-        const int64_t ta_u = max(u0, (int64_t)tile * nsg), tb_u = min(u1, (int64_t)(tile + 1) * nsg);
-        const int64_t wa_u = max(wu0, (int64_t)tile * nsg), wb_u = min(wu1, (int64_t)(tile + 1) * nsg);
-        float* dst;
-        if (wa_u == ta_u && wb_u == tb_u)
-            dst = s_ctile + (tile - t_first) * kTileRows * BM;  // only this warp touches the tile
-        else
-            dst = s_slots + (warp * 2 + (tile == (int)(wu0 / nsg) ? 0 : 1)) * kTileRows * BM;
+        // exclusive: this warp holds all of the CTA's units of the tile
+        const bool excl = u == max(u0, tile * nsg) && u + run == min(u1, (tile + 1) * nsg);
+        float* dst = excl ? s_ctile + (tile - t_first) * TE
+                          : s_slots + (warp * 2 + (tile == wfirst ? 0 : 1)) * TE;
 #pragma unroll
         for (int n = 0; n < NT; ++n) {
             const int col = 8 * n + 2 * t4;
-            dst[g * BM + col] = r[n][0];
-            dst[g * BM + col + 1] = r[n][1];
-            dst[(g + 8) * BM + col] = r[n][2];
-            dst[(g + 8) * BM + col + 1] = r[n][3];
+            dst[g * BM + col] = rr[n][0];
+            dst[g * BM + col + 1] = rr[n][1];
+            dst[(g + 8) * BM + col] = rr[n][2];
+            dst[(g + 8) * BM + col + 1] = rr[n][3];
         }
+        u += run;
+        ++tile;
+        sg = 0;
     }
     // A wait that gave up leaves copies in flight into this warp's ring (and
     // possibly the CTA-wide ones): wait for them, again with a bound, before
     // the shared memory can be retired.
-    if (!alive && fail_it >= 0)
-        for (int j = fail_it; j < issued; ++j) (void)mbar_wait(&wbar[j % stages], (uint32_t)(j / stages) & 1u);
+    if (!alive && fail_at >= 0)
+        for (int j = fail_at; j < issued; ++j) (void)mbar_wait(&wbar[j % stages], (uint32_t)(j / stages) & 1u);
     if (!ok) (void)mbar_wait(xbar, 0);
     __syncthreads();
 
@@ -712,7 +715,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_fused_kernel(const __grid_co
         for (int i = tid; i < nrows; i += kThreads) {
             const int rs = s_rp[i], re = s_rp[i + 1];
             if (re > rs) {
-                const int tau_a = (rs - p0) / e_per, tau_b = min(kThreads - 1, (re - 1 - p0) / e_per);
+                const int tau_a = (rs - p0) / e_per, tau_b = min(kCsrThreads - 1, (re - 1 - p0) / e_per);
                 for (int tau = tau_a; tau <= tau_b; ++tau) {
                     if (s_headrow[tau] == i)
 #pragma unroll
@@ -723,81 +726,71 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_fused_kernel(const __grid_co
                 }
             }
         }
+        __syncthreads();
     }
 
-    // ---- combine warps per tile (warp order), add the sparse rows
-    for (int e = tid; e < ctiles * kTileRows * BM; e += kThreads) {
-        const int tl = e / (kTileRows * BM), rr = (e / BM) % kTileRows, col = e % BM;
-        const int tile = t_first + tl;
-        const int64_t ta_u = max(u0, (int64_t)tile * nsg), tb_u = min(u1, (int64_t)(tile + 1) * nsg);
-        float sum = 0.f;
-        bool single = false;
-        for (int wv = 0; wv < kWarps; ++wv) {
-            const int64_t a = u0 + cn * wv / kWarps, b = u0 + cn * (wv + 1) / kWarps;
-            const int64_t lo = max(a, ta_u), hi = min(b, tb_u);
-            if (lo >= hi) continue;
-            if (lo == ta_u && hi == tb_u) {
-                single = true;
-                break;
+    // ---- per tile: sum the warps' parts (warp order), add the sparse rows,
+    // then write y (tile complete in this CTA) or publish the partial
+    for (int tl = 0; tl < ctiles; ++tl) {
+        const int tile_i = t_first + tl;
+        const int ta_u = max(u0, tile_i * nsg), tb_u = min(u1, (tile_i + 1) * nsg);
+        const bool whole = ta_u == tile_i * nsg && tb_u == (tile_i + 1) * nsg;
+        for (int e = tid; e < TE; e += kThreads) {
+            const int row_l = e / BM, col = e - row_l * BM;
+            float sum = 0.f;
+            bool direct = false;
+            for (int wv = 0; wv < kWarps; ++wv) {
+                const int a = u0 + cn * wv / kWarps, b = u0 + cn * (wv + 1) / kWarps;
+                const int lo = max(a, ta_u), hi = min(b, tb_u);
+                if (lo >= hi) continue;
+                if (lo == ta_u && hi == tb_u) {
+                    direct = true;
+                    break;
+                }
+                const int wf = a / nsg;
+                sum += s_slots[(wv * 2 + (tile_i == wf ? 0 : 1)) * TE + e];
             }
-            const int slot = (tile == (int)(a / nsg)) ? 0 : 1;
-            sum += s_slots[((wv * 2 + slot) * kTileRows + rr) * BM + col];
-        }
-        if (!single) s_ctile[e] = sum;
-    }
-    __syncthreads();
-    if (has_csr) {
-        for (int e = tid; e < ctiles * kTileRows * BM; e += kThreads) {
-            const int tl = e / (kTileRows * BM), rr = (e / BM) % kTileRows, col = e % BM;
-            const int row = (t_first + tl) * kTileRows + rr;
-            if (row >= ra && row < ra + nrows) s_ctile[e] += s_rowsum[(row - ra) * BM + col];
-        }
-        __syncthreads();
-    }
-
-    // ---- write finished tiles; publish partial tiles
-    for (int e = tid; e < ctiles * kTileRows * BM; e += kThreads) {
-        const int tl = e / (kTileRows * BM), rr = (e / BM) % kTileRows, col = e % BM;
-        const int tile = t_first + tl;
-        const int row = tile * kTileRows + rr;
-        const bool whole = u0 <= (int64_t)tile * nsg && (int64_t)(tile + 1) * nsg <= u1;
-        if (whole) {
-            if (row < p.n_out && col < B) p.y[col * p.ldy + row] = f2h_rn(s_ctile[e]);
-        } else {
-            const int slot = (tile == t_first) ? 0 : 1;
-            p.part[(((int64_t)c * 2 + slot) * kTileRows + rr) * 16 + col] = s_ctile[e];
+            if (direct) sum = s_ctile[tl * TE + e];
+            const int row = tile_i * kTileRows + row_l;
+            if (has_csr && row >= ra && row < ra + nrows) sum += s_rowsum[(row - ra) * BM + col];
+            if (whole) {
+                if (row < p.n_out && col < B) p.y[col * p.ldy + row] = f2h_rn(sum);
+            } else {
+                const int slot = (tile_i == t_first) ? 0 : 1;
+                p.part[(((int64_t)c * 2 + slot) * kTileRows + row_l) * 16 + col] = sum;
+            }
         }
     }
-    // boundary tiles: first and last tile when they are shared with other CTAs
+    // ---- tiles shared with other CTAs: the last CTA to arrive adds the parts
     for (int side = 0; side < 2; ++side) {
-        const int tile = side == 0 ? t_first : t_last;
+        const int tile_i = side == 0 ? t_first : t_last;
         if (side == 1 && t_last == t_first) break;
-        const bool whole = u0 <= (int64_t)tile * nsg && (int64_t)(tile + 1) * nsg <= u1;
+        const bool whole = u0 <= tile_i * nsg && (tile_i + 1) * nsg <= u1;
         if (whole) continue;
-        __threadfence();
-        __syncthreads();
+        __syncthreads();  // this CTA's partial is written
         if (tid == 0) {
-            const int cf = cta_of(U, G, (int64_t)tile * nsg);
-            const int cl = cta_of(U, G, (int64_t)(tile + 1) * nsg - 1);
-            const int old = atomicAdd(&p.tile_cnt[tile], 1);
-            *s_flag = (old == cl - cf) ? 1 : 0;
+            const int cf = cta_of(U, G, tile_i * nsg), cl = cta_of(U, G, (tile_i + 1) * nsg - 1);
+            __threadfence();  // release the CTA's partial before counting
+            const int old = atomicAdd(&p.tile_cnt[tile_i], 1);
+            const int last = old == cl - cf;
+            if (last) __threadfence();  // acquire the other CTAs' partials
+            *s_flag = last ? (cf | (cl << 16)) + 1 : 0;
         }
         __syncthreads();
-        if (*s_flag) {
-            __threadfence();
-            const int cf = cta_of(U, G, (int64_t)tile * nsg);
-            const int cl = cta_of(U, G, (int64_t)(tile + 1) * nsg - 1);
-            for (int e = tid; e < kTileRows * BM; e += kThreads) {
-                const int rr = e / BM, col = e % BM;
-                const int row = tile * kTileRows + rr;
+        const int fl = *s_flag;
+        if (fl) {
+            const int cf = (fl - 1) & 0xffff, cl = (fl - 1) >> 16;
+            for (int e = tid; e < TE; e += kThreads) {
+                const int row_l = e / BM, col = e - row_l * BM;
+                const int row = tile_i * kTileRows + row_l;
                 float sum = 0.f;
                 for (int cc = cf; cc <= cl; ++cc) {
-                    const int slot = (tile == (int)(cta_begin(U, G, cc) / nsg)) ? 0 : 1;
-                    sum += __ldcg(p.part + (((int64_t)cc * 2 + slot) * kTileRows + rr) * 16 + col);
+                    const int slot = (tile_i == cta_begin(U, G, cc) / nsg) ? 0 : 1;
+                    sum += __ldcg(p.part + (((int64_t)cc * 2 + slot) * kTileRows + row_l) * 16 + col);
                 }
                 if (row < p.n_out && col < B) p.y[col * p.ldy + row] = f2h_rn(sum);
             }
-            if (tid == 0) p.tile_cnt[tile] = 0;
+            if (tid == 0) p.tile_cnt[tile_i] = 0;
         }
     }
 }

@@ -62,7 +62,7 @@ int max_smem_optin() {
     return n;
 }
 
-constexpr int kDefaultStages = 6;
+constexpr int kDefaultStages = 4;
 
 }  // namespace
 
