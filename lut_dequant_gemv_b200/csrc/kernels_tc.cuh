@@ -7,18 +7,21 @@
 // Work decomposition
 //   * Rows are grouped in tiles of 16 (the M of an m16n8k16 MMA); columns in
 //     super-groups of 256 (16 k16-steps).  A unit = (tile, super-group).
-//   * Units are numbered tile-major and split into equal contiguous ranges:
-//     one range per CTA (one CTA per SM), then one sub-range per warp.
-//     Every SM and every warp streams the same number of code bytes.
-//   * A tile whose units fall in several warps or CTAs is combined
-//     deterministically: warps through shared memory, CTAs through a small
-//     global partial buffer where the last CTA to arrive (atomic counter,
-//     reset by that CTA) adds the parts in CTA order.  No thread ever waits
-//     for another CTA.
+//   * Each CTA owns a contiguous run of whole tiles (runs differ by at most
+//     one tile; grid = min(tiles, 2 CTAs per SM)) and its warps split the
+//     CTA's units into equal contiguous ranges.  A tile is therefore
+//     finished inside one CTA: the warps' partial sums are added in warp
+//     order in shared memory -- deterministic, no global atomics.
+//     Consecutive calls overlap through programmatic dependent launch, so
+//     SMs that finish early start the next call's loads.
 //
-// Streaming: each warp owns a ring of shared-memory stages filled by
-// cp.async.bulk (TMA, 1-D) copies that complete on per-stage mbarriers; all
-// waits are bounded and record a status bit instead of hanging.
+// Streaming: the codes are read with coalesced 128-bit loads straight into
+// registers.  Each warp issues the loads of its first units before waiting
+// for the previous kernel in the stream (programmatic dependent launch:
+// the weights never depend on it), then keeps a fixed number of units in
+// flight while it decodes.  The LUT planes and the CTA's CSR slices are
+// bulk-copied (TMA, 1-D) into shared memory, x after the wait; the waits
+// on those copies are bounded and record a status bit instead of hanging.
 //
 // Decode (kernel-native code layout, built by repack_codes_kernel): for each
 // k16-step a lane holds 4 codes of row g and 4 of row g+8 (g = lane/4) at
@@ -47,15 +50,16 @@
 namespace sqz {
 namespace tc {
 
-constexpr int kWarps = 16;
+constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
-constexpr int kCsrThreads = 256;  // threads that share the sparse part
+constexpr int kCtasPerSm = 2;
+constexpr int kCsrThreads = kThreads;  // threads that share the sparse part
 constexpr int kTileRows = 16;
 constexpr int kSgSteps = 16;   // k16-steps per super-group
 constexpr int kSgCols = 256;   // columns per super-group
-constexpr uint32_t kWaitLimit = 1u << 22;
-constexpr int kMaxGrid = 256;  // CTAs (one per SM)
-constexpr int kCsrCap = 4096;  // CSR entries per CTA staged in shared memory
+constexpr uint32_t kSuspendNs = 1000000u;  // 1 ms per poll
+constexpr uint32_t kWaitLimit = 2000u;
+constexpr int kCsrCap = 2048;  // CSR entries per CTA staged in shared memory
 
 constexpr int kStatusWaitTimeout = 1;
 
@@ -66,12 +70,14 @@ struct Fmt<3> {
     static constexpr int kVecs = 3;        // uint4 per lane per super-group
     static constexpr int kSgBytes = 1536;  // 16 rows x 256 cols x 3 bits
     static constexpr int kLutBytes = 16;   // per row: 8 low bytes, 8 high bytes
+    static constexpr int kDepth = 4;       // units a warp keeps in flight (registers)
 };
 template <>
 struct Fmt<4> {
     static constexpr int kVecs = 4;
     static constexpr int kSgBytes = 2048;
     static constexpr int kLutBytes = 32;   // 16 low bytes, 16 high bytes
+    static constexpr int kDepth = 3;
 };
 
 // ------------------------------------------------------------ shared plan
@@ -80,38 +86,36 @@ struct Fmt<4> {
 struct Plan {
     int64_t units;      // ntiles * nsg
     int grid;           // CTAs
-    int stages;         // ring stages per warp
     int ctiles_max;     // max tiles touched by one CTA
     int x_stride;       // shared-memory row stride of x, in halves
-    int bmax;           // 8 * NT
+    int cm;             // batch columns carried by the sparse part and the combine (1 or 8*NT)
     // byte offsets
-    int off_ring, off_x, off_lut, off_rp, off_col, off_val, off_head, off_tail, off_headrow, off_tailrow, off_rowsum, off_ctile,
-        off_slots, off_flag, total;
+    int off_x, off_lut, off_rp, off_col, off_val, off_head, off_tail, off_headrow, off_tailrow, off_rowsum, off_ctile,
+        off_slots, off_wrange, off_tinfo, total;
 };
 
 __host__ __device__ inline int round_up(int v, int m) { return (v + m - 1) / m * m; }
 
-__host__ __device__ inline Plan make_plan(int bits, int n_out, int k_in, int batch, int nt, int sms, int stages) {
+// First tile of CTA c when `ntiles` tiles are split over `grid` CTAs.
+__host__ __device__ inline int tile_begin(int ntiles, int grid, int c) { return (int)((int64_t)ntiles * c / grid); }
+
+// `ctas`: CTAs the device keeps resident (kCtasPerSm per SM).
+__host__ __device__ inline Plan make_plan(int bits, int n_out, int k_in, int batch, int nt, bool single, int ctas) {
     Plan P{};
     const int ntiles = (n_out + kTileRows - 1) / kTileRows;
     const int nsteps = k_in / 16;
     const int nsg = (nsteps + kSgSteps - 1) / kSgSteps;
-    const int sg_bytes = bits == 3 ? 1536 : 2048;
     const int lut_bytes = bits == 3 ? 16 : 32;
     P.units = (int64_t)ntiles * nsg;
-    P.grid = (int)(P.units < sms ? P.units : sms);
+    P.grid = ntiles < ctas ? ntiles : ctas;
     if (P.grid < 1) P.grid = 1;
-    P.stages = stages;
-    const int64_t upc = (P.units + P.grid - 1) / P.grid;
-    P.ctiles_max = nsg > 0 ? (int)((upc + nsg - 1) / nsg) + 1 : 1;
-    P.bmax = 8 * nt;
+    P.ctiles_max = (ntiles + P.grid - 1) / P.grid;
+    P.cm = single ? 1 : 8 * nt;
     // x rows: stride = 32 (mod 128) bytes keeps the batch rows of one
     // fragment load in different banks.
     int xs_bytes = round_up(k_in * 2, 128) + 32;
     P.x_stride = xs_bytes / 2;
-    int off = 512;  // mbarriers: kWarps*stages + 1 (at most 65 * 8 B)
-    P.off_ring = off;
-    off += kWarps * stages * sg_bytes;
+    int off = 128;  // three mbarriers, CSR bounds
     P.off_x = off;
     off += round_up(batch * xs_bytes, 128);
     P.off_lut = off;
@@ -124,21 +128,23 @@ __host__ __device__ inline Plan make_plan(int bits, int n_out, int k_in, int bat
     P.off_val = off;
     off += (kCsrCap + 16) * 2;  // a slice starts up to 7 entries early and is rounded up to 8
     P.off_head = off;
-    off += kCsrThreads * P.bmax * 4;
+    off += kCsrThreads * P.cm * 4;
     P.off_tail = off;
-    off += kCsrThreads * P.bmax * 4;
+    off += kCsrThreads * P.cm * 4;
     P.off_headrow = off;
     off += kCsrThreads * 4;
     P.off_tailrow = off;
     off += kCsrThreads * 4;
     P.off_rowsum = off;
-    off += round_up(csr_rows * P.bmax * 4, 128);
+    off += round_up(csr_rows * P.cm * 4, 128);
     P.off_ctile = off;
-    off += P.ctiles_max * kTileRows * P.bmax * 4;
+    off += P.ctiles_max * kTileRows * P.cm * 4;
     P.off_slots = off;
-    off += kWarps * 2 * kTileRows * P.bmax * 4;
-    P.off_flag = off;
-    off += 128;
+    off += kWarps * 2 * kTileRows * P.cm * 4;
+    P.off_wrange = off;
+    off += kWarps * 3 * 4;
+    P.off_tinfo = off;
+    off += round_up(P.ctiles_max * 4, 16);
     P.total = off;
     return P;
 }
@@ -154,16 +160,10 @@ struct Params {
     int64_t ldx;
     uint16_t* y;
     int64_t ldy;
-    float* part;             // [grid][2][16][16] cross-CTA partial sums
-    int* tile_cnt;           // [ntiles] arrival counters, zero between calls
     int* status;             // error bits (bounded waits that gave up)
     int n_out, k_in, nsteps, nsg, ntiles, batch;
     int x_bulk;              // 1: every x row is 16-byte aligned -> bulk copies
     Plan plan;
-    // rowptr at the first row owned by each CTA (the rows of the tiles whose
-    // first unit is in the CTA), and at n_out for c = grid: the CTA's CSR
-    // entries are [csr_rp[c], csr_rp[c+1]).  Computed once per layer.
-    int csr_rp[kMaxGrid + 1];
 };
 
 // ------------------------------------------------------------- PTX helpers
@@ -176,16 +176,20 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                  : "memory");
 }
+// One bounded poll: the thread is suspended until the phase completes or
+// kSuspendNs nanoseconds pass, whichever comes first (no busy spinning that
+// would take issue slots from the warps doing the arithmetic).
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendNs)
         : "memory");
     return ok != 0;
 }
-// Bounded wait: false if the phase did not complete within kWaitLimit polls.
+// Bounded wait: false if the phase did not complete within kWaitLimit polls
+// (at most kWaitLimit * kSuspendNs, about two seconds).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
     for (uint32_t i = 0; i < kWaitLimit; ++i)
         if (mbar_try_wait(bar, parity)) return true;
@@ -200,6 +204,11 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
 }
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ __forceinline__ void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
+// Programmatic dependent launch: let the next kernel of the stream start
+// (its CTAs may begin on SMs this grid leaves), and wait until the previous
+// kernel of the stream has finished and its writes are visible.
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait_previous() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t s) {
     uint32_t d;
@@ -253,29 +262,35 @@ __device__ __forceinline__ uint32_t sel3_extra(uint32_t w0, uint32_t w1, uint32_
     return ((w0 >> 3) & 0x11111111u) | ((w1 >> 2) & 0x22222222u) | ((w2 >> 1) & 0x44444444u);
 }
 
-// Decode one k16-step of a lane: a0/a2 = row g pairs, a1/a3 = row g+8 pairs.
-template <int BITS, class TAB>
-__device__ __forceinline__ void decode_step(const TAB& tg, const TAB& tg8, uint32_t word, uint32_t& a0, uint32_t& a1,
-                                            uint32_t& a2, uint32_t& a3) {
-    if constexpr (BITS == 3) {
-        dec3(tg, word & 0x7777u, a0, a2);
-        dec3(tg8, (word >> 16) & 0x7777u, a1, a3);
-    } else {
-        dec4(tg, word & 0x7777u, 0x3210u | ((word >> 1) & 0x4444u), a0, a2);
-        dec4(tg8, (word >> 16) & 0x7777u, 0x3210u | ((word >> 17) & 0x4444u), a1, a3);
-    }
+// Decode one k16-step of a lane from its selector word(s): a0/a2 = row g
+// pairs, a1/a3 = row g+8 pairs.  3-bit: `m` holds the codes of row g in its
+// low 16 bits and of row g+8 in its high 16 bits, bit 3 of every nibble
+// clear.  4-bit: the step word `w`; bit 3 of a nibble selects the upper
+// half of the table.
+__device__ __forceinline__ void decode3(const Tab3& tg, const Tab3& tg8, uint32_t m, uint32_t& a0, uint32_t& a1,
+                                        uint32_t& a2, uint32_t& a3) {
+    dec3(tg, m, a0, a2);
+    dec3(tg8, m >> 16, a1, a3);
+}
+__device__ __forceinline__ void decode4(const Tab4& tg, const Tab4& tg8, uint32_t w, uint32_t& a0, uint32_t& a1,
+                                        uint32_t& a2, uint32_t& a3) {
+    const uint32_t m = w & 0x77777777u;
+    const uint32_t pk = ((w >> 1) & 0x44444444u) | 0x32103210u;
+    dec4(tg, m, pk, a0, a2);
+    dec4(tg8, m >> 16, pk >> 16, a1, a3);
 }
 
-// Step word j (0..15) of a super-group for a lane, from its uint4 vectors.
-// 3-bit: word 4q+j' (j' < 3) is stored; word 4q+3 is rebuilt from the three.
-template <int BITS>
-__device__ __forceinline__ uint32_t step_word(const uint32_t* w, int step) {
-    if constexpr (BITS == 4) {
-        return w[step];
+// Step `st` (0..15) of a lane's super-group words.  3-bit: word 4q+j (j < 3)
+// is stored as such; step 4q+3 is rebuilt from bit 3 of the three words.
+template <int BITS, class TAB>
+__device__ __forceinline__ void decode_step(const TAB& tg, const TAB& tg8, const uint32_t* w, int st, uint32_t& a0,
+                                            uint32_t& a1, uint32_t& a2, uint32_t& a3) {
+    if constexpr (BITS == 3) {
+        const int q = st >> 2, j = st & 3;
+        const uint32_t m = j < 3 ? (w[3 * q + j] & 0x77777777u) : sel3_extra(w[3 * q], w[3 * q + 1], w[3 * q + 2]);
+        decode3(tg, tg8, m, a0, a1, a2, a3);
     } else {
-        const int q = step >> 2, j = step & 3;
-        if (j < 3) return w[3 * q + j];
-        return sel3_extra(w[3 * q], w[3 * q + 1], w[3 * q + 2]);
+        decode4(tg, tg8, w[st], a0, a1, a2, a3);
     }
 }
 
@@ -394,7 +409,7 @@ __global__ void dequant_native_kernel(const uint8_t* __restrict__ codes, const u
             const int gstep = sg * kSgSteps + st;
             if (gstep >= nsteps) break;
             uint32_t a0, a1, a2, a3;
-            decode_step<BITS>(tg, tg8, step_word<BITS>(w, st), a0, a1, a2, a3);
+            decode_step<BITS>(tg, tg8, w, st, a0, a1, a2, a3);
             const int k = gstep * 16 + 4 * t4;
             if (rg < n_out) {
                 uint32_t* o = reinterpret_cast<uint32_t*>(w_out + (int64_t)rg * k_in + k);
@@ -409,40 +424,50 @@ __global__ void dequant_native_kernel(const uint8_t* __restrict__ codes, const u
 }
 
 // ------------------------------------------------------------ main kernel
-__device__ __forceinline__ int cta_begin(int units, int grid, int c) { return (int)((int64_t)units * c / grid); }
-
-// CTA whose unit range contains u.
-__device__ __forceinline__ int cta_of(int units, int grid, int u) {
-    int c = (int)(((int64_t)u * grid) / units);
-    while (c + 1 < grid && cta_begin(units, grid, c + 1) <= u) ++c;
-    while (c > 0 && cta_begin(units, grid, c) > u) --c;
-    return c;
-}
-
-template <int BITS, int NT, bool TC>
-__global__ void __launch_bounds__(kThreads, 1) gemv_fused_kernel(const __grid_constant__ Params p) {
+// SB: batch 1 (one column carried through the sparse part and the combine).
+template <int BITS, int NT, bool TC, bool SB>
+__global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_fused_kernel(const __grid_constant__ Params p) {
     using F = Fmt<BITS>;
     using TAB = typename std::conditional<BITS == 3, Tab3, Tab4>::type;
-    constexpr int BM = 8 * NT;             // batch columns per accumulator set
-    constexpr int TE = kTileRows * BM;      // elements of one tile's result
+    constexpr int BM = 8 * NT;              // batch columns of the MMA accumulators
+    constexpr int CM = SB ? 1 : BM;         // batch columns carried after the dense loop
+    constexpr int TE = kTileRows * CM;      // elements of one tile's result
+    constexpr int D = F::kDepth;            // units in flight per warp
+    static_assert(!SB || NT == 1, "single-batch variant uses one n-tile");
     extern __shared__ __align__(128) uint8_t smem[];
     const Plan& P = p.plan;
+
+    // The next kernel in the stream may start as soon as SMs free up.
+    pdl_launch_dependents();
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t4 = lane & 3;
     const int G = gridDim.x, c = blockIdx.x;
     const int nsg = p.nsg;
-    const int U = (int)P.units;
-    const int u0 = cta_begin(U, G, c), u1 = cta_begin(U, G, c + 1);
+    const int t_first = tile_begin(p.ntiles, G, c), t_end = tile_begin(p.ntiles, G, c + 1);
+    const int ctiles = t_end - t_first;
+    const int u0 = t_first * nsg, u1 = t_end * nsg;  // whole tiles
     const int cn = u1 - u0;
     const int wu0 = u0 + cn * warp / kWarps, wu1 = u0 + cn * (warp + 1) / kWarps;
-    const int t_first = u0 / nsg, t_last = (u1 - 1) / nsg;
-    const int ctiles = t_last - t_first + 1;
-    const int stages = P.stages;
+    const int nwu = wu1 - wu0;
+    const int wfirst = nwu > 0 ? wu0 / nsg : -1;
 
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
-    uint64_t* wbar = bars + warp * stages;
-    uint64_t* xbar = bars + kWarps * stages;
-    uint8_t* ring = smem + P.off_ring + warp * stages * F::kSgBytes;
+    // ---- code prefetch: the first D units of this warp, straight into
+    // registers (coalesced: each 128-bit load of the warp reads 512
+    // consecutive bytes); weights never depend on the previous kernel
+    uint4 R[D][F::kVecs];
+#pragma unroll
+    for (int j = 0; j < D; ++j) {
+        if (j < nwu) {
+            const uint8_t* src = p.codes + (int64_t)(wu0 + j) * F::kSgBytes + lane * 16;
+#pragma unroll
+            for (int m = 0; m < F::kVecs; ++m) R[j][m] = ldg_stream_u128(src + m * 512);
+        }
+    }
+
+    uint64_t* lbar = reinterpret_cast<uint64_t*>(smem);      // LUT planes
+    uint64_t* cbar = reinterpret_cast<uint64_t*>(smem) + 1;  // CSR slices
+    uint64_t* xbar = reinterpret_cast<uint64_t*>(smem) + 2;  // x
+    int* s_bounds = reinterpret_cast<int*>(smem + 32);       // CSR entries [p0, p1) of the CTA's rows
     uint16_t* xs = reinterpret_cast<uint16_t*>(smem + P.off_x);
     uint8_t* luts = smem + P.off_lut;
     float* s_head = reinterpret_cast<float*>(smem + P.off_head);
@@ -452,77 +477,256 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_fused_kernel(const __grid_co
     float* s_rowsum = reinterpret_cast<float*>(smem + P.off_rowsum);
     float* s_ctile = reinterpret_cast<float*>(smem + P.off_ctile);
     float* s_slots = reinterpret_cast<float*>(smem + P.off_slots);
-    int* s_flag = reinterpret_cast<int*>(smem + P.off_flag);
+    int* s_wrange = reinterpret_cast<int*>(smem + P.off_wrange);  // [warp] = {first unit, end unit, first tile}
+    int* s_tinfo = reinterpret_cast<int*>(smem + P.off_tinfo);    // [tile] = {mask of warps holding parts}
 
-    // ---- barriers
-    if (lane == 0)
-        for (int s = 0; s < stages; ++s) mbar_init(&wbar[s], 1);
-    if (tid == 0) mbar_init(xbar, 1);
+    // ---- rows of the CTA's tiles and their outliers
+    const int ra = min(p.n_out, t_first * kTileRows);
+    const int nrows = min(p.n_out, t_end * kTileRows) - ra;
+    const bool has_csr = p.nnz > 0 && nrows > 0;
+    const int rp_off = ra & 3;
+
+    // ---- barriers, warp ranges, per-tile contributor masks
+    if (lane == 0) {
+        s_wrange[warp * 3] = wu0;
+        s_wrange[warp * 3 + 1] = wu1;
+        s_wrange[warp * 3 + 2] = wfirst;
+    }
+    if (tid == 0) {
+        mbar_init(lbar, 1);
+        mbar_init(cbar, 1);
+        mbar_init(xbar, 1);
+    }
+    for (int tl = tid; tl < ctiles; tl += kThreads) {
+        const int ta_u = (t_first + tl) * nsg, tb_u = ta_u + nsg;
+        // warps holding a part of the tile (a warp range may be empty when
+        // the CTA has fewer units than warps)
+        int mask = 0;
+        for (int wv = 0; wv < kWarps; ++wv) {
+            const int a = u0 + cn * wv / kWarps, b = u0 + cn * (wv + 1) / kWarps;
+            if (max(a, ta_u) < min(b, tb_u)) mask |= 1 << wv;
+        }
+        s_tinfo[tl] = mask;
+    }
+    if (has_csr) {
+        for (int i = tid; i < nrows * CM; i += kThreads) s_rowsum[i] = 0.f;
+        s_headrow[tid] = -1;
+        s_tailrow[tid] = -1;
+    }
     fence_mbar_init();
     __syncthreads();
 
-    // ---- sparse rows owned by this CTA: those of the tiles whose first unit
-    // lies in [u0, u1); their CSR entries are [csr_rp[c], csr_rp[c+1]).
-    const int ta = (u0 + nsg - 1) / nsg, tb = t_last;
-    const int ra = min(p.n_out, ta * kTileRows);
-    const int nrows = ta <= tb ? min(p.n_out, (tb + 1) * kTileRows) - ra : 0;
-    const int p0 = p.csr_rp[c], p1 = p.csr_rp[c + 1];
-    const int nz = p1 - p0;
-    const bool has_csr = p.nnz > 0 && nrows > 0;
-    const bool csr_smem = has_csr && nz <= kCsrCap;
-    // staged slices start at 16-byte aligned source addresses; these are the
-    // element offsets of the first wanted entry inside the staged buffers
-    const int rp_off = ra & 3, col_off = p0 & 3, val_off = p0 & 7;
-
-    // ---- CTA-wide copies: LUT planes of the CTA's tiles, x (when every row
-    // is 16-byte aligned) and the CTA's CSR slices
-    const uint32_t lut_bytes = (uint32_t)ctiles * kTileRows * F::kLutBytes;
+    // ---- weights that do not depend on the previous kernel: the LUT planes
+    // of the CTA's tiles, then (after reading the CTA's rowptr bounds) its
+    // CSR slices, which are only needed after the dense part
     if (tid == 0) {
-        uint32_t tx = lut_bytes + (p.x_bulk ? (uint32_t)p.batch * p.k_in * 2 : 0u);
+        const uint32_t lut_bytes = (uint32_t)ctiles * kTileRows * F::kLutBytes;
+        mbar_expect_tx(lbar, lut_bytes);
+        bulk_g2s(luts, p.lutp + (int64_t)t_first * kTileRows * F::kLutBytes, lut_bytes, lbar);
+        const int q0 = has_csr ? p.rowptr[ra] : 0, q1 = has_csr ? p.rowptr[ra + nrows] : 0;
+        s_bounds[0] = q0;
+        s_bounds[1] = q1;
+        const int nzz = q1 - q0;
+        const bool in_smem = has_csr && nzz <= kCsrCap;
         const uint32_t rp_bytes = has_csr ? (uint32_t)round_up(nrows + 1 + rp_off, 4) * 4 : 0u;
-        const uint32_t col_bytes = csr_smem ? (uint32_t)round_up(nz + col_off, 4) * 4 : 0u;
-        const uint32_t val_bytes = csr_smem ? (uint32_t)round_up(nz + val_off, 8) * 2 : 0u;
-        tx += rp_bytes + col_bytes + val_bytes;
-        mbar_expect_tx(xbar, tx);
-        bulk_g2s(luts, p.lutp + (int64_t)t_first * kTileRows * F::kLutBytes, lut_bytes, xbar);
-        if (p.x_bulk)
-            for (int b = 0; b < p.batch; ++b) bulk_g2s(xs + b * P.x_stride, p.x + b * p.ldx, p.k_in * 2, xbar);
-        if (rp_bytes) bulk_g2s(smem + P.off_rp, p.rowptr + (ra - rp_off), rp_bytes, xbar);
-        if (col_bytes) bulk_g2s(smem + P.off_col, p.col + (p0 - col_off), col_bytes, xbar);
-        if (val_bytes) bulk_g2s(smem + P.off_val, p.val + (p0 - val_off), val_bytes, xbar);
+        const uint32_t col_bytes = in_smem ? (uint32_t)round_up(nzz + (q0 & 3), 4) * 4 : 0u;
+        const uint32_t val_bytes = in_smem ? (uint32_t)round_up(nzz + (q0 & 7), 8) * 2 : 0u;
+        mbar_expect_tx(cbar, rp_bytes + col_bytes + val_bytes);
+        if (rp_bytes) bulk_g2s(smem + P.off_rp, p.rowptr + (ra - rp_off), rp_bytes, cbar);
+        if (col_bytes) bulk_g2s(smem + P.off_col, p.col + (q0 - (q0 & 3)), col_bytes, cbar);
+        if (val_bytes) bulk_g2s(smem + P.off_val, p.val + (q0 - (q0 & 7)), val_bytes, cbar);
     }
-    // ---- per-warp ring prologue
-    const int nwu = wu1 - wu0;
-    int issued = nwu < stages ? nwu : stages;
-    if (lane == 0)
-        for (int s = 0; s < issued; ++s) {
-            mbar_expect_tx(&wbar[s], F::kSgBytes);
-            bulk_g2s(ring + s * F::kSgBytes, p.codes + (int64_t)(wu0 + s) * F::kSgBytes, F::kSgBytes, &wbar[s]);
+
+    // ---- x and y may be written or read by the previous kernel of the
+    // stream: wait for it to finish
+    pdl_wait_previous();
+    if (tid == 0) {
+        if (p.x_bulk) {
+            mbar_expect_tx(xbar, (uint32_t)p.batch * p.k_in * 2);
+            for (int b = 0; b < p.batch; ++b) bulk_g2s(xs + b * P.x_stride, p.x + b * p.ldx, p.k_in * 2, xbar);
+        } else {
+            mbar_expect_tx(xbar, 0);
         }
+    }
     if (!p.x_bulk) {
         for (int i = tid; i < p.batch * p.k_in; i += kThreads) {
             const int b = i / p.k_in, k = i - b * p.k_in;
             xs[b * P.x_stride + k] = p.x[b * p.ldx + k];
         }
     }
-    if (has_csr) {
-        for (int i = tid; i < nrows * BM; i += kThreads) s_rowsum[i] = 0.f;
-        if (tid < kCsrThreads) {
-            s_headrow[tid] = -1;
-            s_tailrow[tid] = -1;
-        }
-    }
-    const bool ok = __syncthreads_and(mbar_wait(xbar, 0) ? 1 : 0) != 0;
+    const bool got_l = mbar_wait(lbar, 0), got_x = mbar_wait(xbar, 0);
+    const bool ok = __syncthreads_and(got_l && got_x ? 1 : 0) != 0;
     if (!ok && tid == 0) atomicOr(p.status, kStatusWaitTimeout);
 
-    // ---- sparse part: a fixed share of nonzeros per thread (balanced)
+    // ---- dense part
     const int B = p.batch;
+    const int xrow = (g < B) ? g : 0;  // batch column of this lane's B fragment (n = g)
+    const int xrow2 = (NT == 2 && g + 8 < B) ? g + 8 : 0;
+    TAB tg, tg8;
+    float d0[NT][4], d1[NT][4];
+    float f0 = 0.f, f1 = 0.f;  // CUDA-core accumulators (rows g, g+8)
+    int tile = -1;
+
+    // Hand this warp's part of `tile` to the CTA (shared memory).
+    auto flush_tile = [&]() {
+        float rr[NT][4];
+        if constexpr (TC) {
+#pragma unroll
+            for (int n = 0; n < NT; ++n)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) rr[n][q] = d0[n][q] + d1[n][q];
+        } else {
+            f0 += __shfl_xor_sync(0xffffffffu, f0, 1);
+            f0 += __shfl_xor_sync(0xffffffffu, f0, 2);
+            f1 += __shfl_xor_sync(0xffffffffu, f1, 1);
+            f1 += __shfl_xor_sync(0xffffffffu, f1, 2);
+            rr[0][0] = f0;
+            rr[0][1] = 0.f;
+            rr[0][2] = f1;
+            rr[0][3] = 0.f;
+        }
+        const int tl = tile - t_first;
+        const int mask = s_tinfo[tl];
+        const bool excl = (mask & (mask - 1)) == 0;  // this warp is the tile's only contributor
+        float* dst = excl ? s_ctile + tl * TE : s_slots + (warp * 2 + (tile == wfirst ? 0 : 1)) * TE;
+        if constexpr (SB) {
+            if (t4 == 0) {
+                dst[g] = rr[0][0];
+                dst[g + 8] = rr[0][2];
+            }
+        } else {
+#pragma unroll
+            for (int n = 0; n < NT; ++n) {
+                const int col = 8 * n + 2 * t4;
+                dst[g * CM + col] = rr[n][0];
+                dst[g * CM + col + 1] = rr[n][1];
+                dst[(g + 8) * CM + col] = rr[n][2];
+                dst[(g + 8) * CM + col + 1] = rr[n][3];
+            }
+        }
+    };
+
+    // Decode and multiply-accumulate one unit (16 rows x 256 columns).
+    auto process = [&](const uint4 (&v)[F::kVecs], int unit) {
+        const int ut = unit / nsg;
+        if (ut != tile) {
+            if (tile >= 0) flush_tile();
+            tile = ut;
+            const uint8_t* lt = luts + (tile - t_first) * kTileRows * F::kLutBytes;
+            if constexpr (BITS == 3) {
+                tg = load_tab3(lt + g * F::kLutBytes);
+                tg8 = load_tab3(lt + (g + 8) * F::kLutBytes);
+            } else {
+                tg = load_tab4(lt + g * F::kLutBytes);
+                tg8 = load_tab4(lt + (g + 8) * F::kLutBytes);
+            }
+#pragma unroll
+            for (int n = 0; n < NT; ++n)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) d0[n][q] = d1[n][q] = 0.f;
+            f0 = f1 = 0.f;
+        }
+        uint32_t w[4 * F::kVecs];
+#pragma unroll
+        for (int m = 0; m < F::kVecs; ++m) w[4 * m] = v[m].x, w[4 * m + 1] = v[m].y, w[4 * m + 2] = v[m].z, w[4 * m + 3] = v[m].w;
+        const int step0 = (unit - tile * nsg) * kSgSteps;
+        const int nvalid = min(kSgSteps, p.nsteps - step0);
+        // x fragment source: batch rows >= B read row 0 (those MMA columns
+        // are never written out), so every lane loads unconditionally
+        const uint16_t* xb0 = xs + xrow * P.x_stride + step0 * 16 + 4 * t4;
+        const uint16_t* xb1 = xs + xrow2 * P.x_stride + step0 * 16 + 4 * t4;
+        auto mac = [&](int st, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3) {
+            if constexpr (TC) {
+                const uint2 xv = *reinterpret_cast<const uint2*>(xb0 + st * 16);
+                if (st & 1)
+                    mma16816(d1[0], a0, a1, a2, a3, xv.x, xv.y);
+                else
+                    mma16816(d0[0], a0, a1, a2, a3, xv.x, xv.y);
+                if constexpr (NT == 2) {
+                    const uint2 xw = *reinterpret_cast<const uint2*>(xb1 + st * 16);
+                    if (st & 1)
+                        mma16816(d1[1], a0, a1, a2, a3, xw.x, xw.y);
+                    else
+                        mma16816(d0[1], a0, a1, a2, a3, xw.x, xw.y);
+                }
+            } else {
+                const uint2 xv = *reinterpret_cast<const uint2*>(xb0 + st * 16);
+                fma2_mixed(f0, a0, xv.x);
+                fma2_mixed(f0, a2, xv.y);
+                fma2_mixed(f1, a1, xv.x);
+                fma2_mixed(f1, a3, xv.y);
+            }
+        };
+        if (nvalid == kSgSteps) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                if constexpr (BITS == 3) {
+                    const uint32_t w0 = w[3 * q], w1 = w[3 * q + 1], w2 = w[3 * q + 2];
+                    uint32_t a0, a1, a2, a3;
+                    decode3(tg, tg8, w0 & 0x77777777u, a0, a1, a2, a3);
+                    mac(4 * q, a0, a1, a2, a3);
+                    decode3(tg, tg8, w1 & 0x77777777u, a0, a1, a2, a3);
+                    mac(4 * q + 1, a0, a1, a2, a3);
+                    decode3(tg, tg8, w2 & 0x77777777u, a0, a1, a2, a3);
+                    mac(4 * q + 2, a0, a1, a2, a3);
+                    decode3(tg, tg8, sel3_extra(w0, w1, w2), a0, a1, a2, a3);
+                    mac(4 * q + 3, a0, a1, a2, a3);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        uint32_t a0, a1, a2, a3;
+                        decode4(tg, tg8, w[4 * q + j], a0, a1, a2, a3);
+                        mac(4 * q + j, a0, a1, a2, a3);
+                    }
+                }
+            }
+        } else {
+            // ragged last super-group (K % 256 != 0): steps < nvalid only
+#pragma unroll
+            for (int st = 0; st < kSgSteps; ++st) {
+                if (st < nvalid) {
+                    uint32_t a0, a1, a2, a3;
+                    decode_step<BITS>(tg, tg8, w, st, a0, a1, a2, a3);
+                    mac(st, a0, a1, a2, a3);
+                }
+            }
+        }
+    };
+
+    // Software pipeline over the warp's units: slot j holds unit base+j; it
+    // is refilled with unit base+j+D as soon as its words are taken.
+    for (int base = 0; base < nwu; base += D) {
+#pragma unroll
+        for (int j = 0; j < D; ++j) {
+            const int i = base + j;
+            if (i < nwu) {
+                uint4 v[F::kVecs];
+#pragma unroll
+                for (int m = 0; m < F::kVecs; ++m) v[m] = R[j][m];
+                if (i + D < nwu) {
+                    const uint8_t* src = p.codes + (int64_t)(wu0 + i + D) * F::kSgBytes + lane * 16;
+#pragma unroll
+                    for (int m = 0; m < F::kVecs; ++m) R[j][m] = ldg_stream_u128(src + m * 512);
+                }
+                process(v, wu0 + i);
+            }
+        }
+    }
+    if (tile >= 0) flush_tile();
+
+    // ---- sparse part: a fixed share of nonzeros per thread (balanced);
+    // its slices were copied while the dense part ran
+    const bool got_c = mbar_wait(cbar, 0);
+    if (!got_c && lane == 0) atomicOr(p.status, kStatusWaitTimeout);
     const int* s_rp = reinterpret_cast<const int*>(smem + P.off_rp) + rp_off;
-    const int* csr_col = csr_smem ? reinterpret_cast<const int*>(smem + P.off_col) + col_off - p0 : p.col;
+    const int p0 = s_bounds[0], p1 = s_bounds[1];
+    const int nz = p1 - p0;
+    const bool csr_smem = has_csr && nz <= kCsrCap;
+    const int* csr_col = csr_smem ? reinterpret_cast<const int*>(smem + P.off_col) + (p0 & 3) - p0 : p.col;
     const uint16_t* csr_val =
-        csr_smem ? reinterpret_cast<const uint16_t*>(smem + P.off_val) + val_off - p0 : p.val;
+        csr_smem ? reinterpret_cast<const uint16_t*>(smem + P.off_val) + (p0 & 7) - p0 : p.val;
     const int e_per = has_csr ? max(1, (nz + kCsrThreads - 1) / kCsrThreads) : 1;
-    if (has_csr && ok && tid < kCsrThreads) {
+    if (has_csr && got_c) {
         const int a = p0 + tid * e_per;
         const int b_end = min(p1, a + e_per);
         if (a < b_end) {
@@ -533,23 +737,24 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_fused_kernel(const __grid_co
                 if (s_rp[mid] <= a) lo = mid; else hi = mid - 1;
             }
             int cur = lo;
+            int nxt = s_rp[cur + 1];
             bool first = true;
-            float acc[BM];
+            float acc[CM];
 #pragma unroll
-            for (int b = 0; b < BM; ++b) acc[b] = 0.f;
+            for (int b = 0; b < CM; ++b) acc[b] = 0.f;
             auto emit = [&](bool last) {
+                float* dstp;
                 if (first) {
                     s_headrow[tid] = cur;
-#pragma unroll
-                    for (int b = 0; b < BM; ++b) s_head[tid * BM + b] = acc[b];
+                    dstp = s_head + tid * CM;
                 } else if (last) {
                     s_tailrow[tid] = cur;
-#pragma unroll
-                    for (int b = 0; b < BM; ++b) s_tail[tid * BM + b] = acc[b];
+                    dstp = s_tail + tid * CM;
                 } else {
-#pragma unroll
-                    for (int b = 0; b < BM; ++b) s_rowsum[cur * BM + b] = acc[b];
+                    dstp = s_rowsum + cur * CM;
                 }
+#pragma unroll
+                for (int b = 0; b < CM; ++b) dstp[b] = acc[b];
             };
             for (int base = a; base < b_end; base += 8) {
                 int cc[8];
@@ -564,234 +769,57 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_fused_kernel(const __grid_co
                 for (int j = 0; j < 8; ++j) {
                     const int q = base + j;
                     if (q >= b_end) break;
-                    while (q >= s_rp[cur + 1]) {
+                    while (q >= nxt) {
                         emit(false);
                         first = false;
 #pragma unroll
-                        for (int b = 0; b < BM; ++b) acc[b] = 0.f;
+                        for (int b = 0; b < CM; ++b) acc[b] = 0.f;
                         ++cur;
+                        nxt = s_rp[cur + 1];
                     }
 #pragma unroll
-                    for (int b = 0; b < BM; ++b)
-                        if (b < B) acc[b] = fmaf(vv[j], h2f(xs[b * P.x_stride + cc[j]]), acc[b]);
+                    for (int b = 0; b < CM; ++b)
+                        if (SB || b < B) acc[b] = fmaf(vv[j], h2f(xs[b * P.x_stride + cc[j]]), acc[b]);
                 }
             }
             emit(true);
         }
     }
+    __syncthreads();  // every warp's dense parts and every sparse partial are in shared memory
 
-    // ---- dense part
-    const int xrow = (g < B) ? g : 0;  // batch column of this lane's B fragment (n = g)
-    const int xrow2 = (NT == 2 && g + 8 < B) ? g + 8 : 0;
-    const bool xon = g < B, xon2 = (NT == 2) && (g + 8 < B);
-    const int wfirst = nwu > 0 ? wu0 / nsg : -1;
-    int tile = wfirst, sg = nwu > 0 ? wu0 - wfirst * nsg : 0;
-    int s = 0, consumed = 0;
-    uint32_t par = 0;
-    bool alive = ok;
-    int fail_at = -1;
-    for (int u = wu0; u < wu1;) {
-        const int run = min(wu1 - u, nsg - sg);  // units of `tile` in this warp's range
-        const uint8_t* lt = luts + (tile - t_first) * kTileRows * F::kLutBytes;
-        TAB tg, tg8;
-        if constexpr (BITS == 3) {
-            tg = load_tab3(lt + g * F::kLutBytes);
-            tg8 = load_tab3(lt + (g + 8) * F::kLutBytes);
+    // ---- finish the CTA's tiles: sum the warps' parts in warp order, add
+    // the rows' nonzeros (interior sums plus the pieces of the threads whose
+    // shares cut a row, in thread order) and write y
+    for (int idx = tid; idx < ctiles * TE; idx += kThreads) {
+        const int tl = idx / TE, e = idx - tl * TE;
+        const int tile_i = t_first + tl;
+        const int row_l = e / CM, col = e - row_l * CM;
+        const int mask = s_tinfo[tl];
+        float sum;
+        if ((mask & (mask - 1)) == 0) {
+            sum = s_ctile[idx];
         } else {
-            tg = load_tab4(lt + g * F::kLutBytes);
-            tg8 = load_tab4(lt + (g + 8) * F::kLutBytes);
-        }
-        float d0[NT][4], d1[NT][4];
-#pragma unroll
-        for (int n = 0; n < NT; ++n)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) d0[n][i] = d1[n][i] = 0.f;
-        float f0 = 0.f, f1 = 0.f;  // CUDA-core accumulators (rows g, g+8)
-
-        for (int r = 0; r < run; ++r, ++sg, ++consumed) {
-            if (alive) {
-                const bool got = __all_sync(0xffffffffu, mbar_wait(&wbar[s], par));
-                if (!got) {
-                    alive = false;
-                    fail_at = consumed;
-                    if (lane == 0) atomicOr(p.status, kStatusWaitTimeout);
-                }
-            }
-            uint32_t w[4 * F::kVecs];
-            const uint8_t* sb = ring + s * F::kSgBytes + lane * 16;
-#pragma unroll
-            for (int m = 0; m < F::kVecs; ++m) {
-                const uint4 v = *reinterpret_cast<const uint4*>(sb + m * 512);
-                w[4 * m] = v.x, w[4 * m + 1] = v.y, w[4 * m + 2] = v.z, w[4 * m + 3] = v.w;
-            }
-            __syncwarp();
-            if (alive && issued < nwu) {
-                if (lane == 0) {
-                    fence_proxy_async();
-                    mbar_expect_tx(&wbar[s], F::kSgBytes);
-                    bulk_g2s(ring + s * F::kSgBytes, p.codes + (int64_t)(wu0 + issued) * F::kSgBytes, F::kSgBytes,
-                             &wbar[s]);
-                }
-                ++issued;
-            }
-            if (++s == stages) {
-                s = 0;
-                par ^= 1u;
-            }
-            const int step0 = sg * kSgSteps;
-            const int nvalid = min(kSgSteps, p.nsteps - step0);
-            const uint16_t* xb0 = xs + xrow * P.x_stride + step0 * 16 + 4 * t4;
-            const uint16_t* xb1 = xs + xrow2 * P.x_stride + step0 * 16 + 4 * t4;
-#pragma unroll
-            for (int st = 0; st < kSgSteps; ++st) {
-                if (st >= nvalid) break;  // ragged last super-group only
-                uint32_t a0, a1, a2, a3;
-                decode_step<BITS>(tg, tg8, step_word<BITS>(w, st), a0, a1, a2, a3);
-                if constexpr (TC) {
-                    const uint2 xv = xon ? *reinterpret_cast<const uint2*>(xb0 + st * 16) : make_uint2(0u, 0u);
-                    if (st & 1)
-                        mma16816(d1[0], a0, a1, a2, a3, xv.x, xv.y);
-                    else
-                        mma16816(d0[0], a0, a1, a2, a3, xv.x, xv.y);
-                    if constexpr (NT == 2) {
-                        const uint2 xw = xon2 ? *reinterpret_cast<const uint2*>(xb1 + st * 16) : make_uint2(0u, 0u);
-                        if (st & 1)
-                            mma16816(d1[1], a0, a1, a2, a3, xw.x, xw.y);
-                        else
-                            mma16816(d0[1], a0, a1, a2, a3, xw.x, xw.y);
-                    }
-                } else {
-                    const uint2 xv = *reinterpret_cast<const uint2*>(xs + step0 * 16 + 4 * t4 + st * 16);
-                    fma2_mixed(f0, a0, xv.x);
-                    fma2_mixed(f0, a2, xv.y);
-                    fma2_mixed(f1, a1, xv.x);
-                    fma2_mixed(f1, a3, xv.y);
-                }
+            sum = 0.f;
+            for (int mm = mask; mm; mm &= mm - 1) {
+                const int wv = __ffs(mm) - 1;
+                sum += s_slots[(wv * 2 + (tile_i == s_wrange[wv * 3 + 2] ? 0 : 1)) * TE + e];
             }
         }
-        // ---- this warp's contribution to `tile`
-        float rr[NT][4];
-        if constexpr (TC) {
-#pragma unroll
-            for (int n = 0; n < NT; ++n)
-#pragma unroll
-                for (int i = 0; i < 4; ++i) rr[n][i] = d0[n][i] + d1[n][i];
-        } else {
-            f0 += __shfl_xor_sync(0xffffffffu, f0, 1);
-            f0 += __shfl_xor_sync(0xffffffffu, f0, 2);
-            f1 += __shfl_xor_sync(0xffffffffu, f1, 1);
-            f1 += __shfl_xor_sync(0xffffffffu, f1, 2);
-            rr[0][0] = t4 == 0 ? f0 : 0.f;
-            rr[0][1] = 0.f;
-            rr[0][2] = t4 == 0 ? f1 : 0.f;
-            rr[0][3] = 0.f;
-        }
-        // exclusive: this warp holds all of the CTA's units of the tile
-        const bool excl = u == max(u0, tile * nsg) && u + run == min(u1, (tile + 1) * nsg);
-        float* dst = excl ? s_ctile + (tile - t_first) * TE
-                          : s_slots + (warp * 2 + (tile == wfirst ? 0 : 1)) * TE;
-#pragma unroll
-        for (int n = 0; n < NT; ++n) {
-            const int col = 8 * n + 2 * t4;
-            dst[g * BM + col] = rr[n][0];
-            dst[g * BM + col + 1] = rr[n][1];
-            dst[(g + 8) * BM + col] = rr[n][2];
-            dst[(g + 8) * BM + col + 1] = rr[n][3];
-        }
-        u += run;
-        ++tile;
-        sg = 0;
-    }
-    // A wait that gave up leaves copies in flight into this warp's ring (and
-    // possibly the CTA-wide ones): wait for them, again with a bound, before
-    // the shared memory can be retired.
-    if (!alive && fail_at >= 0)
-        for (int j = fail_at; j < issued; ++j) (void)mbar_wait(&wbar[j % stages], (uint32_t)(j / stages) & 1u);
-    if (!ok) (void)mbar_wait(xbar, 0);
-    __syncthreads();
-
-    // ---- sparse rows cut at thread boundaries: combine in thread order
-    if (has_csr) {
-        for (int i = tid; i < nrows; i += kThreads) {
+        const int row = tile_i * kTileRows + row_l;
+        if (has_csr && row < ra + nrows) {
+            const int i = row - ra;
             const int rs = s_rp[i], re = s_rp[i + 1];
+            float cs = s_rowsum[i * CM + col];
             if (re > rs) {
                 const int tau_a = (rs - p0) / e_per, tau_b = min(kCsrThreads - 1, (re - 1 - p0) / e_per);
                 for (int tau = tau_a; tau <= tau_b; ++tau) {
-                    if (s_headrow[tau] == i)
-#pragma unroll
-                        for (int b = 0; b < BM; ++b) s_rowsum[i * BM + b] += s_head[tau * BM + b];
-                    if (s_tailrow[tau] == i)
-#pragma unroll
-                        for (int b = 0; b < BM; ++b) s_rowsum[i * BM + b] += s_tail[tau * BM + b];
+                    if (s_headrow[tau] == i) cs += s_head[tau * CM + col];
+                    if (s_tailrow[tau] == i) cs += s_tail[tau * CM + col];
                 }
             }
+            sum += cs;
         }
-        __syncthreads();
-    }
-
-    // ---- per tile: sum the warps' parts (warp order), add the sparse rows,
-    // then write y (tile complete in this CTA) or publish the partial
-    for (int tl = 0; tl < ctiles; ++tl) {
-        const int tile_i = t_first + tl;
-        const int ta_u = max(u0, tile_i * nsg), tb_u = min(u1, (tile_i + 1) * nsg);
-        const bool whole = ta_u == tile_i * nsg && tb_u == (tile_i + 1) * nsg;
-        for (int e = tid; e < TE; e += kThreads) {
-            const int row_l = e / BM, col = e - row_l * BM;
-            float sum = 0.f;
-            bool direct = false;
-            for (int wv = 0; wv < kWarps; ++wv) {
-                const int a = u0 + cn * wv / kWarps, b = u0 + cn * (wv + 1) / kWarps;
-                const int lo = max(a, ta_u), hi = min(b, tb_u);
-                if (lo >= hi) continue;
-                if (lo == ta_u && hi == tb_u) {
-                    direct = true;
-                    break;
-                }
-                const int wf = a / nsg;
-                sum += s_slots[(wv * 2 + (tile_i == wf ? 0 : 1)) * TE + e];
-            }
-            if (direct) sum = s_ctile[tl * TE + e];
-            const int row = tile_i * kTileRows + row_l;
-            if (has_csr && row >= ra && row < ra + nrows) sum += s_rowsum[(row - ra) * BM + col];
-            if (whole) {
-                if (row < p.n_out && col < B) p.y[col * p.ldy + row] = f2h_rn(sum);
-            } else {
-                const int slot = (tile_i == t_first) ? 0 : 1;
-                p.part[(((int64_t)c * 2 + slot) * kTileRows + row_l) * 16 + col] = sum;
-            }
-        }
-    }
-    // ---- tiles shared with other CTAs: the last CTA to arrive adds the parts
-    for (int side = 0; side < 2; ++side) {
-        const int tile_i = side == 0 ? t_first : t_last;
-        if (side == 1 && t_last == t_first) break;
-        const bool whole = u0 <= tile_i * nsg && (tile_i + 1) * nsg <= u1;
-        if (whole) continue;
-        __syncthreads();  // this CTA's partial is written
-        if (tid == 0) {
-            const int cf = cta_of(U, G, tile_i * nsg), cl = cta_of(U, G, (tile_i + 1) * nsg - 1);
-            __threadfence();  // release the CTA's partial before counting
-            const int old = atomicAdd(&p.tile_cnt[tile_i], 1);
-            const int last = old == cl - cf;
-            if (last) __threadfence();  // acquire the other CTAs' partials
-            *s_flag = last ? (cf | (cl << 16)) + 1 : 0;
-        }
-        __syncthreads();
-        const int fl = *s_flag;
-        if (fl) {
-            const int cf = (fl - 1) & 0xffff, cl = (fl - 1) >> 16;
-            for (int e = tid; e < TE; e += kThreads) {
-                const int row_l = e / BM, col = e - row_l * BM;
-                const int row = tile_i * kTileRows + row_l;
-                float sum = 0.f;
-                for (int cc = cf; cc <= cl; ++cc) {
-                    const int slot = (tile_i == cta_begin(U, G, cc) / nsg) ? 0 : 1;
-                    sum += __ldcg(p.part + (((int64_t)cc * 2 + slot) * kTileRows + row_l) * 16 + col);
-                }
-                if (row < p.n_out && col < B) p.y[col * p.ldy + row] = f2h_rn(sum);
-            }
-            if (tid == 0) p.tile_cnt[tile_i] = 0;
-        }
+        if (row < p.n_out && col < B) p.y[col * p.ldy + row] = f2h_rn(sum);
     }
 }
 

@@ -62,7 +62,6 @@ int max_smem_optin() {
     return n;
 }
 
-constexpr int kDefaultStages = 4;
 
 }  // namespace
 
@@ -73,6 +72,7 @@ struct sqz_layer {
     int device = 0;
     int sm_count = 148;
     int smem_optin = 232448;
+    int smem_per_sm = 233472;
     int mac = SQZ_MAC_TENSOR_CORES;
     // The fused kernel works on whole k16-steps: K % 16 == 0 (4-bit layers
     // with K % 16 == 8 use the row-per-warp kernel).
@@ -89,13 +89,9 @@ struct sqz_layer {
     // kernel-native layout for the fused kernel
     int ntiles = 0, nsteps = 0, nsg = 0;
     int64_t units = 0;
-    int grid = 0;
     uint8_t* codes_native = nullptr;  // [ntiles][nsg][sg_bytes]
     uint8_t* lut_native = nullptr;    // [ntiles*16][2 << bits] byte planes
-    float* part = nullptr;            // [grid][2][16][16]
-    int* tile_cnt = nullptr;          // [ntiles], zero between calls
     int* status = nullptr;            // [1]
-    std::vector<int> csr_rp;          // [grid+1]
     uint16_t* x_stage = nullptr;      // [SQZ_MAX_BATCH][k_in] for sqz_gemv_host
     uint16_t* y_stage = nullptr;      // [SQZ_MAX_BATCH][n_out]
     int64_t device_bytes = 0;
@@ -112,8 +108,6 @@ void free_layer(sqz_layer* L) {
     cudaFree(L->val);
     cudaFree(L->codes_native);
     cudaFree(L->lut_native);
-    cudaFree(L->part);
-    cudaFree(L->tile_cnt);
     cudaFree(L->status);
     cudaFree(L->x_stage);
     cudaFree(L->y_stage);
@@ -186,9 +180,9 @@ void dispatch_rowwarp(const sqz_layer* L, const uint16_t* x, int32_t batch, int6
 }
 
 // ------------------------------------------------------------ fused kernel
-template <int BITS, int NT, bool TC>
+template <int BITS, int NT, bool TC, bool SB>
 sqz_status set_smem_attr(int bytes) {
-    SQZ_CUDA_TRY(cudaFuncSetAttribute(sqz::tc::gemv_fused_kernel<BITS, NT, TC>,
+    SQZ_CUDA_TRY(cudaFuncSetAttribute(sqz::tc::gemv_fused_kernel<BITS, NT, TC, SB>,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, bytes),
                  "cudaFuncSetAttribute");
     return SQZ_OK;
@@ -196,32 +190,43 @@ sqz_status set_smem_attr(int bytes) {
 
 sqz_status prepare_fused_kernels(int optin) {
     sqz_status st;
-    if ((st = set_smem_attr<3, 1, true>(optin)) != SQZ_OK) return st;
-    if ((st = set_smem_attr<3, 2, true>(optin)) != SQZ_OK) return st;
-    if ((st = set_smem_attr<4, 1, true>(optin)) != SQZ_OK) return st;
-    if ((st = set_smem_attr<4, 2, true>(optin)) != SQZ_OK) return st;
-    if ((st = set_smem_attr<3, 1, false>(optin)) != SQZ_OK) return st;
-    if ((st = set_smem_attr<4, 1, false>(optin)) != SQZ_OK) return st;
+    if ((st = set_smem_attr<3, 1, true, true>(optin)) != SQZ_OK) return st;
+    if ((st = set_smem_attr<3, 1, true, false>(optin)) != SQZ_OK) return st;
+    if ((st = set_smem_attr<3, 2, true, false>(optin)) != SQZ_OK) return st;
+    if ((st = set_smem_attr<4, 1, true, true>(optin)) != SQZ_OK) return st;
+    if ((st = set_smem_attr<4, 1, true, false>(optin)) != SQZ_OK) return st;
+    if ((st = set_smem_attr<4, 2, true, false>(optin)) != SQZ_OK) return st;
+    if ((st = set_smem_attr<3, 1, false, true>(optin)) != SQZ_OK) return st;
+    if ((st = set_smem_attr<4, 1, false, true>(optin)) != SQZ_OK) return st;
     return SQZ_OK;
 }
 
 // Plan for a call, or false when the fused kernel cannot stage x.
 bool fused_plan(const sqz_layer* L, int batch, sqz::tc::Plan* out) {
     const int nt = batch > 8 ? 2 : 1;
-    for (int stages = kDefaultStages; stages >= 2; --stages) {
-        sqz::tc::Plan P = sqz::tc::make_plan(L->bits, L->n_out, L->k_in, batch, nt, L->sm_count, stages);
-        if (P.total <= L->smem_optin) {
-            *out = P;
-            return P.grid == L->grid;
-        }
-    }
-    return false;
+    sqz::tc::Plan P =
+        sqz::tc::make_plan(L->bits, L->n_out, L->k_in, batch, nt, batch == 1, sqz::tc::kCtasPerSm * L->sm_count);
+    if (P.total > L->smem_optin) return false;
+    *out = P;
+    return true;
 }
 
-template <int BITS, int NT, bool TC>
-void launch_fused(const sqz::tc::Params& prm, cudaStream_t s) {
-    sqz::tc::gemv_fused_kernel<BITS, NT, TC>
-        <<<prm.plan.grid, sqz::tc::kThreads, prm.plan.total, s>>>(prm);
+// Launch with programmatic stream serialization: the kernel may start while
+// the previous kernel of the stream is still running; it prefetches only
+// weights before it waits for that kernel (griddepcontrol.wait).
+template <int BITS, int NT, bool TC, bool SB>
+cudaError_t launch_fused(const sqz::tc::Params& prm, cudaStream_t s) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)prm.plan.grid);
+    cfg.blockDim = dim3(sqz::tc::kThreads);
+    cfg.dynamicSmemBytes = (size_t)prm.plan.total;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, sqz::tc::gemv_fused_kernel<BITS, NT, TC, SB>, prm);
 }
 
 sqz_status gemv_impl(const sqz_layer* L, const uint16_t* x, int32_t batch, int64_t ldx, uint16_t* y, int64_t ldy,
@@ -240,8 +245,6 @@ sqz_status gemv_impl(const sqz_layer* L, const uint16_t* x, int32_t batch, int64
         prm.ldx = ldx;
         prm.y = y;
         prm.ldy = ldy;
-        prm.part = L->part;
-        prm.tile_cnt = L->tile_cnt;
         prm.status = L->status;
         prm.n_out = L->n_out;
         prm.k_in = L->k_in;
@@ -251,17 +254,20 @@ sqz_status gemv_impl(const sqz_layer* L, const uint16_t* x, int32_t batch, int64
         prm.batch = batch;
         prm.x_bulk = (reinterpret_cast<uintptr_t>(x) % 16 == 0) && (ldx % 8 == 0) && (L->k_in % 8 == 0);
         prm.plan = P;
-        for (int c = 0; c <= L->grid; ++c) prm.csr_rp[c] = L->csr_rp[c];
         const bool cuda_cores = L->mac == SQZ_MAC_CUDA_CORES && batch == 1;
+        cudaError_t e;
         if (L->bits == 3) {
-            if (cuda_cores) launch_fused<3, 1, false>(prm, s);
-            else if (batch > 8) launch_fused<3, 2, true>(prm, s);
-            else launch_fused<3, 1, true>(prm, s);
+            if (cuda_cores) e = launch_fused<3, 1, false, true>(prm, s);
+            else if (batch > 8) e = launch_fused<3, 2, true, false>(prm, s);
+            else if (batch > 1) e = launch_fused<3, 1, true, false>(prm, s);
+            else e = launch_fused<3, 1, true, true>(prm, s);
         } else {
-            if (cuda_cores) launch_fused<4, 1, false>(prm, s);
-            else if (batch > 8) launch_fused<4, 2, true>(prm, s);
-            else launch_fused<4, 1, true>(prm, s);
+            if (cuda_cores) e = launch_fused<4, 1, false, true>(prm, s);
+            else if (batch > 8) e = launch_fused<4, 2, true, false>(prm, s);
+            else if (batch > 1) e = launch_fused<4, 1, true, false>(prm, s);
+            else e = launch_fused<4, 1, true, true>(prm, s);
         }
+        SQZ_CUDA_TRY(e, "fused gemv launch");
     } else if (L->bits == 3) {
         dispatch_rowwarp<3>(L, x, batch, ldx, y, ldy, s);
     } else {
@@ -271,26 +277,19 @@ sqz_status gemv_impl(const sqz_layer* L, const uint16_t* x, int32_t batch, int64
     return SQZ_OK;
 }
 
-// Kernel-native copies of codes and LUT, scratch of the fused kernel, and
-// the per-CTA CSR bounds.  `h_rowptr` is the host copy of rowptr (or empty).
-sqz_status build_native(sqz_layer* L, const std::vector<int32_t>& h_rowptr, cudaStream_t s) {
+// Kernel-native copies of codes and LUT and the fused kernel's status word.
+sqz_status build_native(sqz_layer* L, cudaStream_t s) {
     using namespace sqz::tc;
     L->ntiles = (L->n_out + kTileRows - 1) / kTileRows;
     L->nsteps = L->k_in / 16;
     L->nsg = (L->nsteps + kSgSteps - 1) / kSgSteps;
     L->units = (int64_t)L->ntiles * L->nsg;
-    const Plan P = make_plan(L->bits, L->n_out, L->k_in, 1, 1, L->sm_count, kDefaultStages);
-    L->grid = P.grid;
-    if (L->grid > kMaxGrid) return fail(SQZ_ERR_UNSUPPORTED, "more than %d SMs", kMaxGrid);
     const int sg_bytes = L->bits == 3 ? 1536 : 2048;
     const int lut_row = 2 << L->bits;
     sqz_status st;
     if ((st = alloc(&L->codes_native, (size_t)L->units * sg_bytes, L, "native codes")) != SQZ_OK) return st;
     if ((st = alloc(&L->lut_native, (size_t)L->ntiles * kTileRows * lut_row, L, "native lut")) != SQZ_OK) return st;
-    if ((st = alloc(&L->part, (size_t)L->grid * 2 * kTileRows * 16, L, "partials")) != SQZ_OK) return st;
-    if ((st = alloc(&L->tile_cnt, (size_t)(L->ntiles > 0 ? L->ntiles : 1), L, "tile counters")) != SQZ_OK) return st;
     if ((st = alloc(&L->status, 1, L, "status")) != SQZ_OK) return st;
-    if (L->tile_cnt) SQZ_CUDA_TRY(cudaMemsetAsync(L->tile_cnt, 0, sizeof(int) * (L->ntiles > 0 ? L->ntiles : 1), s), "memset");
     SQZ_CUDA_TRY(cudaMemsetAsync(L->status, 0, sizeof(int), s), "memset");
     if (L->units > 0) {
         const int64_t words = L->units * (sg_bytes / 4);
@@ -315,18 +314,6 @@ sqz_status build_native(sqz_layer* L, const std::vector<int32_t>& h_rowptr, cuda
             sqz::tc::repack_lut_kernel<4><<<blocks, 256, 0, s>>>(L->lut, L->n_out, rows, L->lut_native);
         SQZ_CUDA_TRY(cudaGetLastError(), "repack lut");
     }
-    // CSR entries owned by each CTA: rows of the tiles whose first unit is in
-    // the CTA's unit range.
-    L->csr_rp.assign(L->grid + 1, 0);
-    for (int c = 0; c <= L->grid; ++c) {
-        int ra = L->n_out;
-        if (c < L->grid && L->units > 0) {
-            const int64_t u0 = L->units * c / L->grid;
-            const int64_t ta = (u0 + L->nsg - 1) / L->nsg;
-            ra = (int)(ta * kTileRows < L->n_out ? ta * kTileRows : L->n_out);
-        }
-        L->csr_rp[c] = h_rowptr.empty() ? 0 : h_rowptr[ra];
-    }
     return SQZ_OK;
 }
 
@@ -350,6 +337,12 @@ sqz_status sqz_create_layer(const sqz_layer_desc* desc, void* stream, sqz_layer_
     L->wpr = (int64_t)desc->k_in * desc->bits / 32;
     L->sm_count = sm_count_of_current_device();
     L->smem_optin = max_smem_optin();
+    {
+        int dev = 0, v = 0;
+        if (cudaGetDevice(&dev) == cudaSuccess &&
+            cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) == cudaSuccess && v > 0)
+            L->smem_per_sm = v;
+    }
     cudaGetDevice(&L->device);
 
     const size_t n = (size_t)desc->n_out, lut_n = n << desc->bits, code_n = n * (size_t)L->wpr;
@@ -375,7 +368,6 @@ sqz_status sqz_create_layer(const sqz_layer_desc* desc, void* stream, sqz_layer_
     SQZ_STEP(prepare_fused_kernels(L->smem_optin));
     SQZ_STEP(alloc(&L->codes, code_n, L, "codes allocation"));
     SQZ_STEP(alloc(&L->lut, lut_n, L, "lut allocation"));
-    std::vector<int32_t> h_rowptr;
     if (nnz > 0) {
         SQZ_STEP(alloc(&L->rowptr, n + 1 + 8, L, "rowptr allocation"));
         SQZ_STEP(alloc(&L->col, nnz + 8, L, "col allocation"));
@@ -422,11 +414,9 @@ sqz_status sqz_create_layer(const sqz_layer_desc* desc, void* stream, sqz_layer_
                         (h_flag & 2) ? " rowptr[N]!=nnz" : "", (h_flag & 4) ? " rowptr decreasing" : "",
                         (h_flag & 8) ? " column outside [0,K)" : "");
         }
-        h_rowptr.resize(n + 1);
-        SQZ_CUDA_STEP(cudaMemcpy(h_rowptr.data(), L->rowptr, (n + 1) * 4, cudaMemcpyDeviceToHost), "rowptr readback");
     }
     L->fused_ok = L->n_out > 0 && L->k_in > 0 && L->k_in % 16 == 0;
-    if (L->fused_ok) SQZ_STEP(build_native(L, h_rowptr, s));
+    if (L->fused_ok) SQZ_STEP(build_native(L, s));
     SQZ_CUDA_STEP(cudaStreamSynchronize(s), "layer creation");
 #undef SQZ_STEP
 #undef SQZ_CUDA_STEP

@@ -73,6 +73,11 @@ SMALL = [
     (300, 4128, 3, 2000, 16, False, False),
     (257, 4104, 4, 1500, 7, False, False),
     (64, 2048, 3, 0, 16, False, False),
+    # fewer units than warps per CTA, tiles shared by several CTAs
+    (500, 2048, 3, 400, 1, False, False),
+    (4096, 256, 4, 100, 1, False, True),
+    (2000, 512, 3, 300, 4, True, False),
+    (1000, 1024, 4, 900, 9, False, False),
 ]
 
 
