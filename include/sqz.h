@@ -82,7 +82,7 @@ typedef struct {
     int32_t bits;           /* 3 or 4                                                 */
     const uint32_t* codes;  /* [n_out][k_in*bits/32]; may be NULL when N*K == 0        */
     const uint16_t* lut;    /* [n_out][1<<bits] fp16 bits; may be NULL when N == 0     */
-    int64_t nnz;            /* outliers, 0 <= nnz <= INT32_MAX                        */
+    int64_t nnz;            /* outliers, 0 <= nnz <= INT32_MAX - 64                   */
     const int32_t* rowptr;  /* [n_out+1]; may be NULL when nnz == 0                   */
     const int32_t* col;     /* [nnz];     may be NULL when nnz == 0                   */
     const uint16_t* val;    /* [nnz] fp16 bits; may be NULL when nnz == 0             */
@@ -144,15 +144,18 @@ SQZ_API sqz_status sqz_gemv_host(sqz_layer_t layer, const uint16_t* x_host, int3
 SQZ_API sqz_status sqz_debug_dequant(sqz_layer_t layer, uint16_t* w_out, void* stream);
 
 /* Multiply-accumulate unit of the fused kernel (sqz_layer_set_mac). */
-#define SQZ_MAC_TENSOR_CORES 0 /* mma.sync m16n8k16, fp32 accumulate (default)       */
-#define SQZ_MAC_CUDA_CORES 1   /* fma.rn.f32.f16 on the CUDA cores, batch 1 only    */
+#define SQZ_MAC_TENSOR_CORES 0 /* mma.sync m16n8k16, fp32 accumulate (default)        */
+#define SQZ_MAC_CUDA_CORES 1   /* fma.rn.f32.f16 on the CUDA cores, batch 1 only     */
+#define SQZ_MAC_MIXED 2        /* even k16-steps on the tensor cores, odd steps on   */
+                               /* the CUDA cores, batch 1 only                       */
 
 /*
  * Choose the unit that performs the multiply-accumulates of the dense part.
- * Both give results within the same bound; the CUDA-core variant exists to
- * compare the two on the same decode and data path (it applies to batch-1
- * calls; other batches keep the tensor cores).  Not thread-safe against
- * concurrent sqz_gemv calls on the same handle.
+ * All give results within the same bound (fp16 products are exact in fp32,
+ * accumulation is fp32; only the order of the additions differs); the
+ * choice applies to batch-1 calls, larger batches always use the tensor
+ * cores.  Not thread-safe against concurrent sqz_gemv calls on the same
+ * handle.
  * Errors: SQZ_ERR_INVALID_ARG.
  */
 SQZ_API sqz_status sqz_layer_set_mac(sqz_layer_t layer, int32_t mac);

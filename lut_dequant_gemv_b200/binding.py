@@ -27,6 +27,7 @@ SQZ_ERR_TIMEOUT = 5
 SQZ_MAX_BATCH = 16
 SQZ_MAC_TENSOR_CORES = 0
 SQZ_MAC_CUDA_CORES = 1
+SQZ_MAC_MIXED = 2
 
 STATUS_NAMES = {0: "SQZ_OK", 1: "SQZ_ERR_INVALID_ARG", 2: "SQZ_ERR_UNSUPPORTED", 3: "SQZ_ERR_CUDA",
                 4: "SQZ_ERR_OOM", 5: "SQZ_ERR_TIMEOUT"}

@@ -7,21 +7,27 @@
 // Work decomposition
 //   * Rows are grouped in tiles of 16 (the M of an m16n8k16 MMA); columns in
 //     super-groups of 256 (16 k16-steps).  A unit = (tile, super-group).
-//   * Each CTA owns a contiguous run of whole tiles (runs differ by at most
-//     one tile; grid = min(tiles, 2 CTAs per SM)) and its warps split the
-//     CTA's units into equal contiguous ranges.  A tile is therefore
-//     finished inside one CTA: the warps' partial sums are added in warp
-//     order in shared memory -- deterministic, no global atomics.
-//     Consecutive calls overlap through programmatic dependent launch, so
-//     SMs that finish early start the next call's loads.
+//   * One CTA of 16 warps per SM.  Each CTA owns a contiguous run of whole
+//     tiles (runs differ by at most one tile) and its warps split the CTA's
+//     units into equal contiguous ranges, so a tile is finished inside one
+//     CTA: no global atomics, no second pass.
+//   * A tile held by several warps is finished by the warp that flushes its
+//     part last (a shared-memory arrival counter): it adds the parts in warp
+//     order -- deterministic -- and writes y while the other warps keep
+//     decoding.  There is no CTA-wide barrier after the dense loop.
 //
-// Streaming: the codes are read with coalesced 128-bit loads straight into
-// registers.  Each warp issues the loads of its first units before waiting
-// for the previous kernel in the stream (programmatic dependent launch:
-// the weights never depend on it), then keeps a fixed number of units in
-// flight while it decodes.  The LUT planes and the CTA's CSR slices are
-// bulk-copied (TMA, 1-D) into shared memory, x after the wait; the waits
-// on those copies are bounded and record a status bit instead of hanging.
+// Streaming: every warp streams its units through a private ring of
+// shared-memory stages with asynchronous 16-byte copies (cp.async, one
+// commit group per unit), keeping stages-1 units in flight while it
+// decodes.  The copies are asynchronous on purpose: a CTA barrier waits for
+// the outstanding ordinary loads of the threads that reach it, but not for
+// asynchronous copies, so the barriers of the prologue never wait for the
+// code stream.  Before waiting for the previous kernel of the stream
+// (programmatic dependent launch; the weights never depend on it) a CTA
+// requests its LUT planes, rowptr slice and sparse entries (bulk copies) and
+// the first code unit of every warp; x is requested right after the wait and
+// ahead of the remaining code units.  Waits on the bulk copies are bounded
+// and record a status bit instead of hanging.
 //
 // Decode (kernel-native code layout, built by repack_codes_kernel): for each
 // k16-step a lane holds 4 codes of row g and 4 of row g+8 (g = lane/4) at
@@ -30,17 +36,28 @@
 // gathers the bytes of four weights at once and a second `prmt` interleaves
 // them into fp16 pairs, which are exactly the A fragment of the MMA once
 // the MMA's k order is permuted to match (the same permutation is applied
-// to x, so the product is unchanged).
+// to x, so the product is unchanged).  The byte permutes run on the integer
+// ALU pipe, which bounds the dense part; shifts are written as high
+// multiplies so that they run on the FMA pipe instead.
 //
-// MAC: fp16 x fp16 products are exact in fp32; accumulation is fp32, either
-// on the tensor cores (mma.sync m16n8k16, batch columns in N) or on the CUDA
-// cores (mixed-precision fma.rn.f32.f16, batch 1 only).
+// Padding instead of ragged paths: columns past K inside the last
+// super-group carry, per row, the code of a finite LUT entry, and x is zero
+// there in shared memory, so every unit is a full 16-step unit and the
+// padded products are exact zeros.
 //
-// Sparse part: the CSR entries of the rows whose tiles start in a CTA are
-// split evenly over the CTA's threads (a fixed number of nonzeros per
-// thread, independent of how skewed the rows are).  Each thread sums its
-// entries per row; rows cut at thread boundaries are combined in thread
-// order -- the balanced scheme of the pages, made deterministic.
+// MAC: fp16 x fp16 products are exact in fp32; accumulation is fp32, on the
+// tensor cores (mma.sync m16n8k16, batch columns in N), on the CUDA cores
+// (mixed-precision fma.rn.f32.f16, batch 1) or split between both (even
+// steps on the tensor cores, odd steps on the CUDA cores, batch 1).
+//
+// Sparse part: the CSR entries of the rows of a CTA's tiles are split evenly
+// over its threads (a fixed number of nonzeros per thread, independent of
+// how skewed the rows are) -- the balanced scheme of the pages.  Each thread
+// sums its share per row before entering the dense loop, while the code
+// units are in flight, and signals an mbarrier; no CTA barrier follows.
+// The warp that finishes a tile waits on that mbarrier and adds to each row
+// the interior sum and then the pieces of the threads whose shares cut the
+// row, in thread order (deterministic).
 #pragma once
 
 #include <type_traits>
@@ -50,18 +67,29 @@
 namespace sqz {
 namespace tc {
 
-constexpr int kWarps = 8;
+constexpr int kWarps = 16;
 constexpr int kThreads = kWarps * 32;
-constexpr int kCtasPerSm = 2;
-constexpr int kCsrThreads = kThreads;  // threads that share the sparse part
+// Threads sharing the sparse part: all of them while the per-thread pieces
+// are small (up to 8 batch columns), half of them for 16 columns.  Batch 1
+// and batches up to 8 split the entries identically (same sums per column).
+__host__ __device__ constexpr int csr_threads_for(int cm) { return cm <= 8 ? 512 : 256; }
 constexpr int kTileRows = 16;
-constexpr int kSgSteps = 16;   // k16-steps per super-group
-constexpr int kSgCols = 256;   // columns per super-group
+constexpr int kSgSteps = 16;      // k16-steps per super-group
+constexpr int kSgCols = 256;      // columns per super-group
+constexpr int kMaxCtas = 512;     // CTAs per launch (one per SM)
+constexpr int kMinStages = 2;     // shared-memory stages per warp (units in flight + 1)
+constexpr int kMaxStages = 6;
+constexpr int kPreWait = 2;       // code units per warp requested before waiting for the previous kernel
+constexpr int kCsrCap = 4096;     // CSR entries per CTA staged in shared memory, at most (more: read from global)
 constexpr uint32_t kSuspendNs = 1000000u;  // 1 ms per poll
 constexpr uint32_t kWaitLimit = 2000u;
-constexpr int kCsrCap = 2048;  // CSR entries per CTA staged in shared memory
 
 constexpr int kStatusWaitTimeout = 1;
+
+// Multiply-accumulate units (template argument MAC).
+constexpr int kMacTensor = 0;
+constexpr int kMacCuda = 1;
+constexpr int kMacMixed = 2;
 
 template <int BITS>
 struct Fmt;
@@ -70,28 +98,28 @@ struct Fmt<3> {
     static constexpr int kVecs = 3;        // uint4 per lane per super-group
     static constexpr int kSgBytes = 1536;  // 16 rows x 256 cols x 3 bits
     static constexpr int kLutBytes = 16;   // per row: 8 low bytes, 8 high bytes
-    static constexpr int kDepth = 4;       // units a warp keeps in flight (registers)
 };
 template <>
 struct Fmt<4> {
     static constexpr int kVecs = 4;
     static constexpr int kSgBytes = 2048;
     static constexpr int kLutBytes = 32;   // 16 low bytes, 16 high bytes
-    static constexpr int kDepth = 3;
 };
 
 // ------------------------------------------------------------ shared plan
 // Sizes that the host (for the launch) and the kernel (to carve shared
 // memory) must agree on.
 struct Plan {
-    int64_t units;      // ntiles * nsg
-    int grid;           // CTAs
-    int ctiles_max;     // max tiles touched by one CTA
-    int x_stride;       // shared-memory row stride of x, in halves
-    int cm;             // batch columns carried by the sparse part and the combine (1 or 8*NT)
+    int grid;        // CTAs
+    int ctiles_max;  // max tiles owned by one CTA
+    int x_stride;    // shared-memory row stride of x, in halves
+    int x_cols;      // columns of x kept in shared memory (nsg * 256; zero past K)
+    int cm;          // batch columns carried by the sparse part and the combine (1 or 8*NT)
+    int stages;      // shared-memory stages of each warp's code ring
+    int csr_cap;     // CSR entries of a CTA that are staged in shared memory (more: read from global)
     // byte offsets
-    int off_x, off_lut, off_rp, off_col, off_val, off_head, off_tail, off_headrow, off_tailrow, off_rowsum, off_ctile,
-        off_slots, off_wrange, off_tinfo, total;
+    int off_x, off_lut, off_rp, off_rowsum, off_head, off_tail, off_headrow, off_tailrow, off_slots, off_wrange,
+        off_tinfo, off_cnt, off_col, off_val, off_ring, total;
 };
 
 __host__ __device__ inline int round_up(int v, int m) { return (v + m - 1) / m * m; }
@@ -99,52 +127,73 @@ __host__ __device__ inline int round_up(int v, int m) { return (v + m - 1) / m *
 // First tile of CTA c when `ntiles` tiles are split over `grid` CTAs.
 __host__ __device__ inline int tile_begin(int ntiles, int grid, int c) { return (int)((int64_t)ntiles * c / grid); }
 
-// `ctas`: CTAs the device keeps resident (kCtasPerSm per SM).
-__host__ __device__ inline Plan make_plan(int bits, int n_out, int k_in, int batch, int nt, bool single, int ctas) {
+// CTAs of a launch: one per SM, at most one per tile.
+__host__ __device__ inline int grid_size(int n_out, int sms) {
+    const int ntiles = (n_out + kTileRows - 1) / kTileRows;
+    const int g = ntiles < sms ? ntiles : sms;
+    return g < 1 ? 1 : g;
+}
+
+// `budget`: shared memory a CTA may use.  After the fixed part, the code
+// ring gets kMinStages stages per warp, the CSR staging area what is left up
+// to kCsrCap entries, and the ring more stages (up to kMaxStages) from the
+// rest; total > budget when not even kMinStages fit.
+__host__ __device__ inline Plan make_plan(int bits, int n_out, int k_in, int batch, int nt, bool single, int sms,
+                                          int budget) {
     Plan P{};
     const int ntiles = (n_out + kTileRows - 1) / kTileRows;
-    const int nsteps = k_in / 16;
+    const int nsteps = (k_in + 15) / 16;
     const int nsg = (nsteps + kSgSteps - 1) / kSgSteps;
     const int lut_bytes = bits == 3 ? 16 : 32;
-    P.units = (int64_t)ntiles * nsg;
-    P.grid = ntiles < ctas ? ntiles : ctas;
-    if (P.grid < 1) P.grid = 1;
+    P.grid = grid_size(n_out, sms);
     P.ctiles_max = (ntiles + P.grid - 1) / P.grid;
     P.cm = single ? 1 : 8 * nt;
+    P.x_cols = nsg * kSgCols;
     // x rows: stride = 32 (mod 128) bytes keeps the batch rows of one
     // fragment load in different banks.
-    int xs_bytes = round_up(k_in * 2, 128) + 32;
+    const int xs_bytes = round_up(P.x_cols * 2, 128) + 32;
     P.x_stride = xs_bytes / 2;
-    int off = 128;  // three mbarriers, CSR bounds
+    const int rows = P.ctiles_max * kTileRows;
+    int off = 128;  // two mbarriers
     P.off_x = off;
     off += round_up(batch * xs_bytes, 128);
     P.off_lut = off;
-    off += round_up(P.ctiles_max * kTileRows * lut_bytes, 128);
-    const int csr_rows = P.ctiles_max * kTileRows;
+    off += round_up(rows * lut_bytes, 128);
     P.off_rp = off;
-    off += round_up((csr_rows + 8) * 4, 128);
-    P.off_col = off;
-    off += (kCsrCap + 8) * 4;
-    P.off_val = off;
-    off += (kCsrCap + 16) * 2;  // a slice starts up to 7 entries early and is rounded up to 8
-    P.off_head = off;
-    off += kCsrThreads * P.cm * 4;
-    P.off_tail = off;
-    off += kCsrThreads * P.cm * 4;
-    P.off_headrow = off;
-    off += kCsrThreads * 4;
-    P.off_tailrow = off;
-    off += kCsrThreads * 4;
+    off += round_up((rows + 8) * 4, 128);
     P.off_rowsum = off;
-    off += round_up(csr_rows * P.cm * 4, 128);
-    P.off_ctile = off;
-    off += P.ctiles_max * kTileRows * P.cm * 4;
+    off += round_up(rows * P.cm * 4, 128);
+    // the sparse pieces of the threads and the warps' parts of shared tiles
+    const int ct = csr_threads_for(P.cm);
+    P.off_head = off;
+    P.off_tail = off + ct * P.cm * 4;
+    P.off_headrow = P.off_tail + ct * P.cm * 4;
+    P.off_tailrow = P.off_headrow + ct * 4;
+    off += round_up(2 * ct * P.cm * 4 + 2 * ct * 4, 128);
     P.off_slots = off;
-    off += kWarps * 2 * kTileRows * P.cm * 4;
+    off += round_up(kWarps * 2 * kTileRows * P.cm * 4, 128);
     P.off_wrange = off;
-    off += kWarps * 3 * 4;
+    off += round_up(kWarps * 3 * 4, 16);
     P.off_tinfo = off;
     off += round_up(P.ctiles_max * 4, 16);
+    P.off_cnt = off;
+    off += round_up(P.ctiles_max * 4, 16);
+    off = round_up(off, 128);
+    const int sg_bytes = bits == 3 ? 1536 : 2048;
+    const int ring_min = kMinStages * kWarps * sg_bytes;
+    int cap = (budget - off - ring_min - 512) / 6;  // 4-byte column + 2-byte value per entry
+    cap = cap > kCsrCap ? kCsrCap : cap;
+    P.csr_cap = cap < 0 ? 0 : cap & ~7;
+    P.off_col = off;  // a slice starts up to 3 entries early and is rounded up to 4
+    off += round_up((P.csr_cap + 8) * 4, 128);
+    P.off_val = off;  // up to 7 entries early, rounded up to 8
+    off += round_up((P.csr_cap + 16) * 2, 128);
+    P.off_ring = off;
+    int stages = (budget - off) / (kWarps * sg_bytes);
+    if (stages > kMaxStages) stages = kMaxStages;
+    if (stages < kMinStages) stages = kMinStages;
+    P.stages = stages;
+    off += stages * kWarps * sg_bytes;
     P.total = off;
     return P;
 }
@@ -155,15 +204,18 @@ struct Params {
     const int32_t* rowptr;   // canonical CSR (device copies owned by the layer)
     const int32_t* col;
     const uint16_t* val;
-    int64_t nnz;
     const uint16_t* x;
     int64_t ldx;
     uint16_t* y;
     int64_t ldy;
     int* status;             // error bits (bounded waits that gave up)
-    int n_out, k_in, nsteps, nsg, ntiles, batch;
+    int n_out, k_in, nsg, ntiles, batch;
+    int has_csr;             // the layer has outliers
     int x_bulk;              // 1: every x row is 16-byte aligned -> bulk copies
     Plan plan;
+    // CSR entries of the rows of CTA c: [csr_cta[c], csr_cta[c+1]); all zero
+    // when the layer has no outliers.
+    int32_t csr_cta[kMaxCtas + 1];
 };
 
 // ------------------------------------------------------------- PTX helpers
@@ -171,6 +223,11 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)_
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+// Arrive (release at CTA scope: the thread's earlier shared-memory writes are
+// visible to a thread whose wait on this phase succeeds).
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
@@ -202,7 +259,25 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
         "l"(src), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
 }
-__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+// Asynchronous 16-byte global -> shared copy (L2 only), its commit group and
+// the wait for all but the newest n groups of this thread.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_newest(int n) {
+    switch (n) {
+        case 0: cp_async_wait<0>(); break;
+        case 1: cp_async_wait<1>(); break;
+        case 2: cp_async_wait<2>(); break;
+        case 3: cp_async_wait<3>(); break;
+        default: cp_async_wait<4>(); break;
+    }
+}
 __device__ __forceinline__ void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
 // Programmatic dependent launch: let the next kernel of the stream start
 // (its CTAs may begin on SMs this grid leaves), and wait until the previous
@@ -236,8 +311,8 @@ __device__ __forceinline__ Tab4 load_tab4(const uint8_t* row) {
     return Tab4{a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 }
 
-// Four 3-bit codes in the nibbles of sel (bit 3 of each nibble clear) ->
-// fp16 pairs (w0,w1) and (w2,w3).
+// Four 3-bit codes in the low four nibbles of sel (bit 3 of each nibble
+// clear; bits 16..31 are ignored by prmt) -> fp16 pairs (w0,w1), (w2,w3).
 __device__ __forceinline__ void dec3(const Tab3& t, uint32_t sel, uint32_t& w01, uint32_t& w23) {
     const uint32_t lo = prmt(t.l0, t.l1, sel);
     const uint32_t hi = prmt(t.h0, t.h1, sel);
@@ -254,19 +329,15 @@ __device__ __forceinline__ void dec4(const Tab4& t, uint32_t s7, uint32_t pick, 
     w23 = prmt(lo, hi, 0x7362);
 }
 
-// Selectors of one 3-bit quad (steps 4q..4q+3) from the lane's 3 words:
-// step j<3 uses bits 0..2 of the nibbles of word j; step 3's codes are
-// spread over bit 3 of the nibbles of the three words (bit j of the code
-// in word j).  Low 16 bits: row g; high 16 bits: row g+8.
+// 3-bit quad: a lane's words w0, w1, w2 hold the codes of steps 4q, 4q+1,
+// 4q+2 in bits 0..2 of their nibbles; bit 3 of nibble n of word j is bit j
+// of the step-(4q+3) code at nibble n.  Low 16 bits: row g; high: row g+8.
+__device__ __forceinline__ uint32_t sel3_main(uint32_t w) { return w & 0x77777777u; }
 __device__ __forceinline__ uint32_t sel3_extra(uint32_t w0, uint32_t w1, uint32_t w2) {
     return ((w0 >> 3) & 0x11111111u) | ((w1 >> 2) & 0x22222222u) | ((w2 >> 1) & 0x44444444u);
 }
 
-// Decode one k16-step of a lane from its selector word(s): a0/a2 = row g
-// pairs, a1/a3 = row g+8 pairs.  3-bit: `m` holds the codes of row g in its
-// low 16 bits and of row g+8 in its high 16 bits, bit 3 of every nibble
-// clear.  4-bit: the step word `w`; bit 3 of a nibble selects the upper
-// half of the table.
+// Decode one k16-step of a lane: a0/a2 = row g pairs, a1/a3 = row g+8 pairs.
 __device__ __forceinline__ void decode3(const Tab3& tg, const Tab3& tg8, uint32_t m, uint32_t& a0, uint32_t& a1,
                                         uint32_t& a2, uint32_t& a3) {
     dec3(tg, m, a0, a2);
@@ -280,14 +351,13 @@ __device__ __forceinline__ void decode4(const Tab4& tg, const Tab4& tg8, uint32_
     dec4(tg8, m >> 16, pk >> 16, a1, a3);
 }
 
-// Step `st` (0..15) of a lane's super-group words.  3-bit: word 4q+j (j < 3)
-// is stored as such; step 4q+3 is rebuilt from bit 3 of the three words.
+// Step `st` (0..15) of a lane's super-group words (dequant export).
 template <int BITS, class TAB>
 __device__ __forceinline__ void decode_step(const TAB& tg, const TAB& tg8, const uint32_t* w, int st, uint32_t& a0,
                                             uint32_t& a1, uint32_t& a2, uint32_t& a3) {
     if constexpr (BITS == 3) {
         const int q = st >> 2, j = st & 3;
-        const uint32_t m = j < 3 ? (w[3 * q + j] & 0x77777777u) : sel3_extra(w[3 * q], w[3 * q + 1], w[3 * q + 2]);
+        const uint32_t m = j < 3 ? sel3_main(w[3 * q + j]) : sel3_extra(w[3 * q], w[3 * q + 1], w[3 * q + 2]);
         decode3(tg, tg8, m, a0, a1, a2, a3);
     } else {
         decode4(tg, tg8, w[st], a0, a1, a2, a3);
@@ -324,13 +394,23 @@ __device__ __forceinline__ uint32_t canon_code(const uint32_t* codes, int64_t wp
     return v & ((1u << BITS) - 1u);
 }
 
+// Code stored for the columns past K of a row: an entry whose value is
+// finite, so that its product with the zero x there is an exact zero.
+template <int BITS>
+__device__ __forceinline__ uint32_t pad_code(const uint16_t* lut, int row) {
+    constexpr int L = 1 << BITS;
+    for (int e = 0; e < L; ++e)
+        if ((lut[(int64_t)row * L + e] & 0x7c00u) != 0x7c00u) return (uint32_t)e;
+    return 0u;
+}
+
 // One thread per output word of the kernel-native layout.
 template <int BITS>
-__global__ void repack_codes_kernel(const uint32_t* __restrict__ canon, int32_t n_out, int32_t k_in, int nsg,
-                                    int64_t total_words, uint32_t* __restrict__ out) {
+__global__ void repack_codes_kernel(const uint32_t* __restrict__ canon, const uint16_t* __restrict__ lut,
+                                    int32_t n_out, int32_t k_in, int nsg, int64_t total_words,
+                                    uint32_t* __restrict__ out) {
     using F = Fmt<BITS>;
     const int64_t wpr = (int64_t)k_in * BITS / 32;
-    const int nsteps = k_in / 16;
     for (int64_t wi = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; wi < total_words;
          wi += (int64_t)gridDim.x * blockDim.x) {
         const int64_t unit = wi / (F::kVecs * 128);
@@ -339,20 +419,21 @@ __global__ void repack_codes_kernel(const uint32_t* __restrict__ canon, int32_t 
         const int lw = 4 * m + e;  // word index within the lane's list
         const int tile = (int)(unit / nsg), sg = (int)(unit % nsg);
         const int g = lane >> 2, t4 = lane & 3;
-        auto code_or0 = [&](int n, int step) -> uint32_t {
+        auto code_of = [&](int n, int step) -> uint32_t {
             const int row = tile * kTileRows + g + 8 * (n >> 2);
-            const int gstep = sg * kSgSteps + step;
-            if (row >= n_out || gstep >= nsteps) return 0u;
-            return canon_code<BITS>(canon, wpr, row, gstep * 16 + 4 * t4 + (n & 3));
+            if (row >= n_out) return 0u;  // padding rows: their LUT rows are zero
+            const int k = (sg * kSgSteps + step) * 16 + 4 * t4 + (n & 3);
+            if (k >= k_in) return pad_code<BITS>(lut, row);
+            return canon_code<BITS>(canon, wpr, row, k);
         };
         uint32_t word = 0;
         if constexpr (BITS == 4) {
-            for (int n = 0; n < 8; ++n) word |= code_or0(n, lw) << (4 * n);
+            for (int n = 0; n < 8; ++n) word |= code_of(n, lw) << (4 * n);
         } else {
             const int q = lw / 3, j = lw % 3;
             for (int n = 0; n < 8; ++n) {
-                const uint32_t c = code_or0(n, 4 * q + j);
-                const uint32_t x = (code_or0(n, 4 * q + 3) >> j) & 1u;
+                const uint32_t c = code_of(n, 4 * q + j);
+                const uint32_t x = (code_of(n, 4 * q + 3) >> j) & 1u;
                 word |= (c | (x << 3)) << (4 * n);
             }
         }
@@ -375,6 +456,16 @@ __global__ void repack_lut_kernel(const uint16_t* __restrict__ lut, int32_t n_ou
     }
 }
 
+// CSR entry range of each CTA's rows: out[c] = rowptr[first row of CTA c],
+// c = 0..grid (the last value is rowptr[n_out]).
+__global__ void csr_cta_bounds_kernel(const int32_t* __restrict__ rowptr, int32_t n_out, int ntiles, int grid,
+                                      int32_t* __restrict__ out) {
+    for (int c = blockIdx.x * blockDim.x + threadIdx.x; c <= grid; c += gridDim.x * blockDim.x) {
+        const int64_t r = (int64_t)tile_begin(ntiles, grid, c) * kTileRows;
+        out[c] = rowptr[r < n_out ? r : n_out];
+    }
+}
+
 // Dequantized weights from the kernel-native layout, with the GEMV's own
 // decoder: w_out[row][k] = lut[row][code(row,k)].
 template <int BITS>
@@ -384,7 +475,6 @@ __global__ void dequant_native_kernel(const uint8_t* __restrict__ codes, const u
     using F = Fmt<BITS>;
     using TAB = typename std::conditional<BITS == 3, Tab3, Tab4>::type;
     const int lane = threadIdx.x & 31, g = lane >> 2, t4 = lane & 3;
-    const int nsteps = k_in / 16;
     const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
     for (int64_t u = warp0; u < units; u += nwarps) {
@@ -406,11 +496,10 @@ __global__ void dequant_native_kernel(const uint8_t* __restrict__ codes, const u
         }
 #pragma unroll
         for (int st = 0; st < kSgSteps; ++st) {
-            const int gstep = sg * kSgSteps + st;
-            if (gstep >= nsteps) break;
             uint32_t a0, a1, a2, a3;
             decode_step<BITS>(tg, tg8, w, st, a0, a1, a2, a3);
-            const int k = gstep * 16 + 4 * t4;
+            const int k = (sg * kSgSteps + st) * 16 + 4 * t4;  // columns k..k+3 (k_in is a multiple of 8)
+            if (k >= k_in) continue;
             if (rg < n_out) {
                 uint32_t* o = reinterpret_cast<uint32_t*>(w_out + (int64_t)rg * k_in + k);
                 o[0] = a0, o[1] = a2;
@@ -424,16 +513,20 @@ __global__ void dequant_native_kernel(const uint8_t* __restrict__ codes, const u
 }
 
 // ------------------------------------------------------------ main kernel
-// SB: batch 1 (one column carried through the sparse part and the combine).
-template <int BITS, int NT, bool TC, bool SB>
-__global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_fused_kernel(const __grid_constant__ Params p) {
+// MAC: kMacTensor / kMacCuda / kMacMixed.  SB: batch 1 (one column carried
+// through the sparse part and the combine).
+template <int BITS, int NT, int MAC, bool SB>
+__global__ void __launch_bounds__(kThreads, 1) gemv_fused_kernel(const __grid_constant__ Params p) {
     using F = Fmt<BITS>;
     using TAB = typename std::conditional<BITS == 3, Tab3, Tab4>::type;
     constexpr int BM = 8 * NT;              // batch columns of the MMA accumulators
     constexpr int CM = SB ? 1 : BM;         // batch columns carried after the dense loop
     constexpr int TE = kTileRows * CM;      // elements of one tile's result
-    constexpr int D = F::kDepth;            // units in flight per warp
+    constexpr int V = F::kVecs;
+    constexpr int CT = csr_threads_for(CM);  // threads sharing the sparse part
+    static_assert(CT <= kThreads, "sparse part runs on the CTA's threads");
     static_assert(!SB || NT == 1, "single-batch variant uses one n-tile");
+    static_assert(MAC == kMacTensor || SB, "CUDA-core multiply-accumulates carry one batch column");
     extern __shared__ __align__(128) uint8_t smem[];
     const Plan& P = p.plan;
 
@@ -445,150 +538,309 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_fused_kernel(const 
     const int nsg = p.nsg;
     const int t_first = tile_begin(p.ntiles, G, c), t_end = tile_begin(p.ntiles, G, c + 1);
     const int ctiles = t_end - t_first;
-    const int u0 = t_first * nsg, u1 = t_end * nsg;  // whole tiles
-    const int cn = u1 - u0;
+    const int u0 = t_first * nsg, cn = ctiles * nsg;  // the CTA's units: [u0, u0 + cn)
     const int wu0 = u0 + cn * warp / kWarps, wu1 = u0 + cn * (warp + 1) / kWarps;
     const int nwu = wu1 - wu0;
-    const int wfirst = nwu > 0 ? wu0 / nsg : -1;
+    const int wfirst = nwu > 0 ? wu0 / nsg : -1;  // first tile of this warp
 
-    // ---- code prefetch: the first D units of this warp, straight into
-    // registers (coalesced: each 128-bit load of the warp reads 512
-    // consecutive bytes); weights never depend on the previous kernel
-    uint4 R[D][F::kVecs];
-#pragma unroll
-    for (int j = 0; j < D; ++j) {
-        if (j < nwu) {
-            const uint8_t* src = p.codes + (int64_t)(wu0 + j) * F::kSgBytes + lane * 16;
-#pragma unroll
-            for (int m = 0; m < F::kVecs; ++m) R[j][m] = ldg_stream_u128(src + m * 512);
-        }
-    }
+    // ---- rows of the CTA's tiles (their CSR entry range is read where it
+    // is used: an indexed parameter load takes long, and nothing before the
+    // wait for x needs it except the copy of the CSR slices)
+    const int ra = min(p.n_out, t_first * kTileRows);
+    const int nrows = min(p.n_out, t_end * kTileRows) - ra;
+    const bool layer_csr = p.has_csr != 0;
 
-    uint64_t* lbar = reinterpret_cast<uint64_t*>(smem);      // LUT planes
-    uint64_t* cbar = reinterpret_cast<uint64_t*>(smem) + 1;  // CSR slices
-    uint64_t* xbar = reinterpret_cast<uint64_t*>(smem) + 2;  // x
-    int* s_bounds = reinterpret_cast<int*>(smem + 32);       // CSR entries [p0, p1) of the CTA's rows
+    uint64_t* lbar = reinterpret_cast<uint64_t*>(smem);      // LUT planes + rowptr slice
+    uint64_t* xbar = reinterpret_cast<uint64_t*>(smem) + 1;  // x
+    uint64_t* cbar = reinterpret_cast<uint64_t*>(smem) + 2;  // CSR slices
+    uint64_t* rbar = reinterpret_cast<uint64_t*>(smem) + 3;  // sparse pieces written (CT arrivals)
     uint16_t* xs = reinterpret_cast<uint16_t*>(smem + P.off_x);
     uint8_t* luts = smem + P.off_lut;
+    float* s_rowsum = reinterpret_cast<float*>(smem + P.off_rowsum);
     float* s_head = reinterpret_cast<float*>(smem + P.off_head);
     float* s_tail = reinterpret_cast<float*>(smem + P.off_tail);
     int* s_headrow = reinterpret_cast<int*>(smem + P.off_headrow);
     int* s_tailrow = reinterpret_cast<int*>(smem + P.off_tailrow);
-    float* s_rowsum = reinterpret_cast<float*>(smem + P.off_rowsum);
-    float* s_ctile = reinterpret_cast<float*>(smem + P.off_ctile);
     float* s_slots = reinterpret_cast<float*>(smem + P.off_slots);
     int* s_wrange = reinterpret_cast<int*>(smem + P.off_wrange);  // [warp] = {first unit, end unit, first tile}
-    int* s_tinfo = reinterpret_cast<int*>(smem + P.off_tinfo);    // [tile] = {mask of warps holding parts}
-
-    // ---- rows of the CTA's tiles and their outliers
-    const int ra = min(p.n_out, t_first * kTileRows);
-    const int nrows = min(p.n_out, t_end * kTileRows) - ra;
-    const bool has_csr = p.nnz > 0 && nrows > 0;
+    int* s_tinfo = reinterpret_cast<int*>(smem + P.off_tinfo);    // [tile] = mask of warps holding parts
+    int* s_cnt = reinterpret_cast<int*>(smem + P.off_cnt);        // [tile] = parts flushed so far
     const int rp_off = ra & 3;
+    const int* s_rp = reinterpret_cast<const int*>(smem + P.off_rp) + rp_off;  // s_rp[i] = rowptr[ra + i]
 
-    // ---- barriers, warp ranges, per-tile contributor masks
+    // ---- weights, independent of the previous kernel: LUT planes of the
+    // CTA's tiles, the rowptr slice and the CSR entries of its rows
+    if (tid == 0) {
+        mbar_init(lbar, 1);
+        mbar_init(xbar, 1);
+        mbar_init(cbar, 1);
+        mbar_init(rbar, CT);
+        fence_mbar_init();
+        const uint32_t lut_bytes = (uint32_t)ctiles * kTileRows * F::kLutBytes;
+        const uint32_t rp_bytes = layer_csr ? (uint32_t)round_up(nrows + 1 + rp_off, 4) * 4 : 0u;
+        mbar_expect_tx(lbar, lut_bytes + rp_bytes);
+        bulk_g2s(luts, p.lutp + (int64_t)t_first * kTileRows * F::kLutBytes, lut_bytes, lbar);
+        if (rp_bytes) bulk_g2s(smem + P.off_rp, p.rowptr + (ra - rp_off), rp_bytes, lbar);
+        const int q0 = p.csr_cta[c], nz = p.csr_cta[c + 1] - q0;
+        const bool csr_in_smem = nz > 0 && nz <= P.csr_cap;
+        const uint32_t col_bytes = csr_in_smem ? (uint32_t)round_up(nz + (q0 & 3), 4) * 4 : 0u;
+        const uint32_t val_bytes = csr_in_smem ? (uint32_t)round_up(nz + (q0 & 7), 8) * 2 : 0u;
+        mbar_expect_tx(cbar, col_bytes + val_bytes);
+        if (col_bytes) bulk_g2s(smem + P.off_col, p.col + (q0 - (q0 & 3)), col_bytes, cbar);
+        if (val_bytes) bulk_g2s(smem + P.off_val, p.val + (q0 - (q0 & 7)), val_bytes, cbar);
+    }
+
+    // ---- this warp's code ring: unit wu0+i goes to stage i % S; one commit
+    // group per unit (empty past the warp's range) keeps the group count
+    // uniform.  Each lane copies and later reads only its own 16-byte
+    // pieces (coalesced: a warp-wide copy covers 512 consecutive bytes).
+    const int S = P.stages, D = S - 1;
+    uint8_t* ring = smem + P.off_ring + warp * S * F::kSgBytes + lane * 16;
+    auto issue = [&](int i, int stage) {
+        if (i < nwu) {
+            const uint8_t* src = p.codes + (int64_t)(wu0 + i) * F::kSgBytes + lane * 16;
+            uint8_t* dst = ring + stage * F::kSgBytes;
+#pragma unroll
+            for (int m = 0; m < V; ++m) cp_async16(dst + m * 512, src + m * 512);
+        }
+        cp_async_commit();
+    };
+    const int pre = D < kPreWait ? D : kPreWait;
+    for (int j = 0; j < pre; ++j) issue(j, j);
+
+    // ---- bookkeeping: warp ranges, contributors and arrival counters per
+    // tile, zeroed sparse sums, zero x past K
     if (lane == 0) {
         s_wrange[warp * 3] = wu0;
         s_wrange[warp * 3 + 1] = wu1;
         s_wrange[warp * 3 + 2] = wfirst;
     }
-    if (tid == 0) {
-        mbar_init(lbar, 1);
-        mbar_init(cbar, 1);
-        mbar_init(xbar, 1);
-    }
     for (int tl = tid; tl < ctiles; tl += kThreads) {
         const int ta_u = (t_first + tl) * nsg, tb_u = ta_u + nsg;
-        // warps holding a part of the tile (a warp range may be empty when
-        // the CTA has fewer units than warps)
         int mask = 0;
         for (int wv = 0; wv < kWarps; ++wv) {
             const int a = u0 + cn * wv / kWarps, b = u0 + cn * (wv + 1) / kWarps;
             if (max(a, ta_u) < min(b, tb_u)) mask |= 1 << wv;
         }
         s_tinfo[tl] = mask;
+        s_cnt[tl] = 0;
     }
-    if (has_csr) {
+    if (layer_csr) {
         for (int i = tid; i < nrows * CM; i += kThreads) s_rowsum[i] = 0.f;
-        s_headrow[tid] = -1;
-        s_tailrow[tid] = -1;
+        if (tid < CT) {
+            s_headrow[tid] = -1;
+            s_tailrow[tid] = -1;
+        }
     }
-    fence_mbar_init();
+    const int B = p.batch;
+    const int pad = P.x_cols - p.k_in;
+    for (int i = tid; i < B * pad; i += kThreads) {
+        const int b = i / pad;
+        xs[b * P.x_stride + p.k_in + (i - b * pad)] = 0;
+    }
     __syncthreads();
 
-    // ---- weights that do not depend on the previous kernel: the LUT planes
-    // of the CTA's tiles, then (after reading the CTA's rowptr bounds) its
-    // CSR slices, which are only needed after the dense part
-    if (tid == 0) {
-        const uint32_t lut_bytes = (uint32_t)ctiles * kTileRows * F::kLutBytes;
-        mbar_expect_tx(lbar, lut_bytes);
-        bulk_g2s(luts, p.lutp + (int64_t)t_first * kTileRows * F::kLutBytes, lut_bytes, lbar);
-        const int q0 = has_csr ? p.rowptr[ra] : 0, q1 = has_csr ? p.rowptr[ra + nrows] : 0;
-        s_bounds[0] = q0;
-        s_bounds[1] = q1;
-        const int nzz = q1 - q0;
-        const bool in_smem = has_csr && nzz <= kCsrCap;
-        const uint32_t rp_bytes = has_csr ? (uint32_t)round_up(nrows + 1 + rp_off, 4) * 4 : 0u;
-        const uint32_t col_bytes = in_smem ? (uint32_t)round_up(nzz + (q0 & 3), 4) * 4 : 0u;
-        const uint32_t val_bytes = in_smem ? (uint32_t)round_up(nzz + (q0 & 7), 8) * 2 : 0u;
-        mbar_expect_tx(cbar, rp_bytes + col_bytes + val_bytes);
-        if (rp_bytes) bulk_g2s(smem + P.off_rp, p.rowptr + (ra - rp_off), rp_bytes, cbar);
-        if (col_bytes) bulk_g2s(smem + P.off_col, p.col + (q0 - (q0 & 3)), col_bytes, cbar);
-        if (val_bytes) bulk_g2s(smem + P.off_val, p.val + (q0 - (q0 & 7)), val_bytes, cbar);
-    }
-
-    // ---- x and y may be written or read by the previous kernel of the
-    // stream: wait for it to finish
+    // ---- x may be written by the previous kernel of the stream: wait for it
     pdl_wait_previous();
     if (tid == 0) {
         if (p.x_bulk) {
-            mbar_expect_tx(xbar, (uint32_t)p.batch * p.k_in * 2);
-            for (int b = 0; b < p.batch; ++b) bulk_g2s(xs + b * P.x_stride, p.x + b * p.ldx, p.k_in * 2, xbar);
+            mbar_expect_tx(xbar, (uint32_t)B * p.k_in * 2);
+            for (int b = 0; b < B; ++b) bulk_g2s(xs + b * P.x_stride, p.x + b * p.ldx, p.k_in * 2, xbar);
         } else {
             mbar_expect_tx(xbar, 0);
         }
     }
     if (!p.x_bulk) {
-        for (int i = tid; i < p.batch * p.k_in; i += kThreads) {
+        for (int i = tid; i < B * p.k_in; i += kThreads) {
             const int b = i / p.k_in, k = i - b * p.k_in;
             xs[b * P.x_stride + k] = p.x[b * p.ldx + k];
         }
     }
-    const bool got_l = mbar_wait(lbar, 0), got_x = mbar_wait(xbar, 0);
-    const bool ok = __syncthreads_and(got_l && got_x ? 1 : 0) != 0;
-    if (!ok && tid == 0) atomicOr(p.status, kStatusWaitTimeout);
+    // ---- the rest of the first D units
+    for (int j = pre; j < D; ++j) issue(j, j);
+    // Each thread waits for the copies itself (an mbarrier wait makes the
+    // bulk-copied bytes visible to it); only x copied by the threads needs a
+    // barrier.
+    const bool got_l = mbar_wait(lbar, 0), got_x = mbar_wait(xbar, 0), got_c = mbar_wait(cbar, 0);
+    if (!(got_l && got_x && got_c)) atomicOr(p.status, kStatusWaitTimeout);
+    if (!p.x_bulk) __syncthreads();
+
+    // ---- the CTA's CSR entries [q0, q1), a fixed share e_per per thread
+    const int q0 = p.csr_cta[c], q1 = p.csr_cta[c + 1];
+    const int nz = q1 - q0;
+    const bool has_csr = nz > 0;
+    const bool csr_in_smem = has_csr && nz <= P.csr_cap;
+    const int e_per = has_csr ? (int)(((int64_t)nz + CT - 1) / CT) : 1;
+    const int ca = tid < CT ? (int)min((int64_t)q1, (int64_t)q0 + (int64_t)tid * e_per) : q1;
+    const int cb = (int)min((int64_t)q1, (int64_t)ca + e_per);
+
+    // ---- sparse part: a fixed share of nonzeros per thread (balanced).
+    // Each thread sums its entries per row: the first and last rows it
+    // touches go to head/tail pieces, rows it holds entirely to s_rowsum;
+    // then it arrives on rbar.  No CTA barrier: the warp that finishes a
+    // tile waits on rbar and combines the pieces of the tile's rows.
+    const int* csr_col = csr_in_smem ? reinterpret_cast<const int*>(smem + P.off_col) + (q0 & 3) - q0 : p.col;
+    const uint16_t* csr_val =
+        csr_in_smem ? reinterpret_cast<const uint16_t*>(smem + P.off_val) + (q0 & 7) - q0 : p.val;
+    if (has_csr && ca < cb) {
+        // row (relative to ra) containing entry ca: largest r with s_rp[r] <= ca
+        int lo = 0, hi = nrows - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (s_rp[mid] <= ca) lo = mid; else hi = mid - 1;
+        }
+        int cur = lo;
+        int nxt = s_rp[cur + 1];
+        bool first = true;
+        float acc[CM];
+#pragma unroll
+        for (int b = 0; b < CM; ++b) acc[b] = 0.f;
+        auto emit = [&](bool last) {
+            float* dstp;
+            if (first) {
+                s_headrow[tid] = cur;
+                dstp = s_head + tid * CM;
+            } else if (last) {
+                s_tailrow[tid] = cur;
+                dstp = s_tail + tid * CM;
+            } else {
+                dstp = s_rowsum + cur * CM;
+            }
+#pragma unroll
+            for (int b = 0; b < CM; ++b) dstp[b] = acc[b];
+        };
+        for (int base = ca; base < cb; base += 8) {
+            int cc[8];
+            uint32_t vh[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int q = base + j;
+                const bool in = q < cb;
+                cc[j] = in ? csr_col[q] : 0;
+                vh[j] = in ? (uint32_t)csr_val[q] : 0u;
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int q = base + j;
+                if (q >= cb) break;
+                while (q >= nxt) {
+                    emit(false);
+                    first = false;
+#pragma unroll
+                    for (int b = 0; b < CM; ++b) acc[b] = 0.f;
+                    ++cur;
+                    nxt = s_rp[cur + 1];
+                }
+                const float v = h2f((uint16_t)vh[j]);
+#pragma unroll
+                for (int b = 0; b < CM; ++b)
+                    if (SB || b < B) acc[b] = fmaf(v, h2f(xs[b * P.x_stride + cc[j]]), acc[b]);
+            }
+        }
+        emit(true);
+    }
+    if (has_csr && tid < CT) mbar_arrive(rbar);
+
+    if (nwu == 0) return;
+
+    // The sparse sum of row ra+i, batch column col: the interior sum, then
+    // the pieces of the threads whose shares cut the row, in thread order.
+    bool csr_ready = !has_csr;
+    auto csr_row_sum = [&](int i, int col) -> float {
+        if (!has_csr) return 0.f;
+        if (!csr_ready) {
+            if (!mbar_wait(rbar, 0)) atomicOr(p.status, kStatusWaitTimeout);
+            csr_ready = true;
+        }
+        const int rs = s_rp[i], re = s_rp[i + 1];
+        float cs = s_rowsum[i * CM + col];
+        if (re > rs) {
+            const int tau_a = (rs - q0) / e_per, tau_b = min(CT - 1, (re - 1 - q0) / e_per);
+            for (int tau = tau_a; tau <= tau_b; ++tau) {
+                if (s_headrow[tau] == i) cs += s_head[tau * CM + col];
+                if (s_tailrow[tau] == i) cs += s_tail[tau * CM + col];
+            }
+        }
+        return cs;
+    };
 
     // ---- dense part
-    const int B = p.batch;
     const int xrow = (g < B) ? g : 0;  // batch column of this lane's B fragment (n = g)
     const int xrow2 = (NT == 2 && g + 8 < B) ? g + 8 : 0;
     TAB tg, tg8;
     float d0[NT][4], d1[NT][4];
     float f0 = 0.f, f1 = 0.f;  // CUDA-core accumulators (rows g, g+8)
-    int tile = -1;
+    int tile = wfirst;
+    int sg = wu0 - wfirst * nsg;
 
-    // Hand this warp's part of `tile` to the CTA (shared memory).
+    auto start_tile = [&]() {
+        const uint8_t* lt = luts + (tile - t_first) * kTileRows * F::kLutBytes;
+        if constexpr (BITS == 3) {
+            tg = load_tab3(lt + g * F::kLutBytes);
+            tg8 = load_tab3(lt + (g + 8) * F::kLutBytes);
+        } else {
+            tg = load_tab4(lt + g * F::kLutBytes);
+            tg8 = load_tab4(lt + (g + 8) * F::kLutBytes);
+        }
+#pragma unroll
+        for (int n = 0; n < NT; ++n)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) d0[n][q] = d1[n][q] = 0.f;
+        f0 = f1 = 0.f;
+    };
+
+    // y for (row, batch column) = dense value + the row's sparse sum.
+    auto out = [&](int row, int col, float v) {
+        if (row < p.n_out && col < B) p.y[col * p.ldy + row] = f2h_rn(v + csr_row_sum(row - ra, col));
+    };
+
+    // Hand this warp's part of `tile` over: written out directly when the
+    // warp holds the whole tile, otherwise into its slot; the last warp to
+    // arrive adds the slots in warp order and writes y.
     auto flush_tile = [&]() {
         float rr[NT][4];
-        if constexpr (TC) {
+        if constexpr (MAC != kMacCuda) {
 #pragma unroll
             for (int n = 0; n < NT; ++n)
 #pragma unroll
                 for (int q = 0; q < 4; ++q) rr[n][q] = d0[n][q] + d1[n][q];
-        } else {
+        }
+        if constexpr (MAC != kMacTensor) {
             f0 += __shfl_xor_sync(0xffffffffu, f0, 1);
             f0 += __shfl_xor_sync(0xffffffffu, f0, 2);
             f1 += __shfl_xor_sync(0xffffffffu, f1, 1);
             f1 += __shfl_xor_sync(0xffffffffu, f1, 2);
-            rr[0][0] = f0;
-            rr[0][1] = 0.f;
-            rr[0][2] = f1;
-            rr[0][3] = 0.f;
+            if constexpr (MAC == kMacCuda) {
+                rr[0][0] = f0;
+                rr[0][2] = f1;
+                rr[0][1] = rr[0][3] = 0.f;
+            } else {
+                rr[0][0] += f0;
+                rr[0][2] += f1;
+            }
         }
         const int tl = tile - t_first;
+        const int row0 = tile * kTileRows;
         const int mask = s_tinfo[tl];
-        const bool excl = (mask & (mask - 1)) == 0;  // this warp is the tile's only contributor
-        float* dst = excl ? s_ctile + tl * TE : s_slots + (warp * 2 + (tile == wfirst ? 0 : 1)) * TE;
+        if ((mask & (mask - 1)) == 0) {
+            if constexpr (SB) {
+                if (t4 == 0) {
+                    out(row0 + g, 0, rr[0][0]);
+                    out(row0 + g + 8, 0, rr[0][2]);
+                }
+            } else {
+#pragma unroll
+                for (int n = 0; n < NT; ++n) {
+                    const int col = 8 * n + 2 * t4;
+                    out(row0 + g, col, rr[n][0]);
+                    out(row0 + g, col + 1, rr[n][1]);
+                    out(row0 + g + 8, col, rr[n][2]);
+                    out(row0 + g + 8, col + 1, rr[n][3]);
+                }
+            }
+            return;
+        }
+        float* dst = s_slots + (warp * 2 + (tile == wfirst ? 0 : 1)) * TE;
         if constexpr (SB) {
             if (t4 == 0) {
                 dst[g] = rr[0][0];
@@ -604,222 +856,107 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_fused_kernel(const 
                 dst[(g + 8) * CM + col + 1] = rr[n][3];
             }
         }
+        __syncwarp();
+        int arrived = 0;
+        if (lane == 0) {
+            __threadfence_block();
+            arrived = atomicAdd(s_cnt + tl, 1) + 1;
+        }
+        arrived = __shfl_sync(0xffffffffu, arrived, 0);
+        if (arrived == __popc(mask)) {
+            __threadfence_block();
+            for (int e = lane; e < TE; e += 32) {
+                const int row_l = e / CM, col = e - row_l * CM;
+                float sum = 0.f;
+                for (int mm = mask; mm; mm &= mm - 1) {
+                    const int wv = __ffs(mm) - 1;
+                    sum += s_slots[(wv * 2 + (tile == s_wrange[wv * 3 + 2] ? 0 : 1)) * TE + e];
+                }
+                out(row0 + row_l, col, sum);
+            }
+        }
     };
 
     // Decode and multiply-accumulate one unit (16 rows x 256 columns).
-    auto process = [&](const uint4 (&v)[F::kVecs], int unit) {
-        const int ut = unit / nsg;
-        if (ut != tile) {
-            if (tile >= 0) flush_tile();
-            tile = ut;
-            const uint8_t* lt = luts + (tile - t_first) * kTileRows * F::kLutBytes;
-            if constexpr (BITS == 3) {
-                tg = load_tab3(lt + g * F::kLutBytes);
-                tg8 = load_tab3(lt + (g + 8) * F::kLutBytes);
-            } else {
-                tg = load_tab4(lt + g * F::kLutBytes);
-                tg8 = load_tab4(lt + (g + 8) * F::kLutBytes);
-            }
-#pragma unroll
-            for (int n = 0; n < NT; ++n)
-#pragma unroll
-                for (int q = 0; q < 4; ++q) d0[n][q] = d1[n][q] = 0.f;
-            f0 = f1 = 0.f;
-        }
-        uint32_t w[4 * F::kVecs];
-#pragma unroll
-        for (int m = 0; m < F::kVecs; ++m) w[4 * m] = v[m].x, w[4 * m + 1] = v[m].y, w[4 * m + 2] = v[m].z, w[4 * m + 3] = v[m].w;
-        const int step0 = (unit - tile * nsg) * kSgSteps;
-        const int nvalid = min(kSgSteps, p.nsteps - step0);
+    auto process = [&](const uint4 (&v)[V], int sgi) {
         // x fragment source: batch rows >= B read row 0 (those MMA columns
         // are never written out), so every lane loads unconditionally
-        const uint16_t* xb0 = xs + xrow * P.x_stride + step0 * 16 + 4 * t4;
-        const uint16_t* xb1 = xs + xrow2 * P.x_stride + step0 * 16 + 4 * t4;
+        const uint16_t* xb0 = xs + xrow * P.x_stride + sgi * kSgCols + 4 * t4;
+        const uint16_t* xb1 = xs + xrow2 * P.x_stride + sgi * kSgCols + 4 * t4;
         auto mac = [&](int st, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3) {
-            if constexpr (TC) {
-                const uint2 xv = *reinterpret_cast<const uint2*>(xb0 + st * 16);
-                if (st & 1)
+            const uint2 xv = *reinterpret_cast<const uint2*>(xb0 + st * 16);
+            const bool on_tc = MAC == kMacTensor || (MAC == kMacMixed && (st & 1) == 0);
+            if (on_tc) {
+                const int chain = MAC == kMacTensor ? (st & 1) : ((st >> 1) & 1);
+                if (chain)
                     mma16816(d1[0], a0, a1, a2, a3, xv.x, xv.y);
                 else
                     mma16816(d0[0], a0, a1, a2, a3, xv.x, xv.y);
                 if constexpr (NT == 2) {
                     const uint2 xw = *reinterpret_cast<const uint2*>(xb1 + st * 16);
-                    if (st & 1)
+                    if (chain)
                         mma16816(d1[1], a0, a1, a2, a3, xw.x, xw.y);
                     else
                         mma16816(d0[1], a0, a1, a2, a3, xw.x, xw.y);
                 }
             } else {
-                const uint2 xv = *reinterpret_cast<const uint2*>(xb0 + st * 16);
                 fma2_mixed(f0, a0, xv.x);
                 fma2_mixed(f0, a2, xv.y);
                 fma2_mixed(f1, a1, xv.x);
                 fma2_mixed(f1, a3, xv.y);
             }
         };
-        if (nvalid == kSgSteps) {
+        uint32_t w[4 * V];
+#pragma unroll
+        for (int m = 0; m < V; ++m) w[4 * m] = v[m].x, w[4 * m + 1] = v[m].y, w[4 * m + 2] = v[m].z, w[4 * m + 3] = v[m].w;
+        if constexpr (BITS == 3) {
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                if constexpr (BITS == 3) {
-                    const uint32_t w0 = w[3 * q], w1 = w[3 * q + 1], w2 = w[3 * q + 2];
-                    uint32_t a0, a1, a2, a3;
-                    decode3(tg, tg8, w0 & 0x77777777u, a0, a1, a2, a3);
-                    mac(4 * q, a0, a1, a2, a3);
-                    decode3(tg, tg8, w1 & 0x77777777u, a0, a1, a2, a3);
-                    mac(4 * q + 1, a0, a1, a2, a3);
-                    decode3(tg, tg8, w2 & 0x77777777u, a0, a1, a2, a3);
-                    mac(4 * q + 2, a0, a1, a2, a3);
-                    decode3(tg, tg8, sel3_extra(w0, w1, w2), a0, a1, a2, a3);
-                    mac(4 * q + 3, a0, a1, a2, a3);
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        uint32_t a0, a1, a2, a3;
-                        decode4(tg, tg8, w[4 * q + j], a0, a1, a2, a3);
-                        mac(4 * q + j, a0, a1, a2, a3);
-                    }
-                }
+                const uint32_t w0 = w[3 * q], w1 = w[3 * q + 1], w2 = w[3 * q + 2];
+                const uint32_t m0 = sel3_main(w0), m1 = sel3_main(w1), m2 = sel3_main(w2);
+                uint32_t a0, a1, a2, a3;
+                decode3(tg, tg8, m0, a0, a1, a2, a3);
+                mac(4 * q, a0, a1, a2, a3);
+                decode3(tg, tg8, m1, a0, a1, a2, a3);
+                mac(4 * q + 1, a0, a1, a2, a3);
+                decode3(tg, tg8, m2, a0, a1, a2, a3);
+                mac(4 * q + 2, a0, a1, a2, a3);
+                decode3(tg, tg8, sel3_extra(w0, w1, w2), a0, a1, a2, a3);
+                mac(4 * q + 3, a0, a1, a2, a3);
             }
         } else {
-            // ragged last super-group (K % 256 != 0): steps < nvalid only
 #pragma unroll
             for (int st = 0; st < kSgSteps; ++st) {
-                if (st < nvalid) {
-                    uint32_t a0, a1, a2, a3;
-                    decode_step<BITS>(tg, tg8, w, st, a0, a1, a2, a3);
-                    mac(st, a0, a1, a2, a3);
-                }
+                uint32_t a0, a1, a2, a3;
+                decode4(tg, tg8, w[st], a0, a1, a2, a3);
+                mac(st, a0, a1, a2, a3);
             }
         }
     };
 
-    // Software pipeline over the warp's units: slot j holds unit base+j; it
-    // is refilled with unit base+j+D as soon as its words are taken.
-    for (int base = 0; base < nwu; base += D) {
+    start_tile();
+    // Units in order: wait for unit i's group, read its stage, refill the
+    // stage freed by unit i-1 with unit i+D, decode.
+    int s_read = 0, s_fill = D;
+#pragma unroll 1
+    for (int i = 0; i < nwu; ++i) {
+        cp_async_wait_newest(D - 1);
+        uint4 v[V];
+        const uint8_t* src = ring + s_read * F::kSgBytes;
 #pragma unroll
-        for (int j = 0; j < D; ++j) {
-            const int i = base + j;
-            if (i < nwu) {
-                uint4 v[F::kVecs];
-#pragma unroll
-                for (int m = 0; m < F::kVecs; ++m) v[m] = R[j][m];
-                if (i + D < nwu) {
-                    const uint8_t* src = p.codes + (int64_t)(wu0 + i + D) * F::kSgBytes + lane * 16;
-#pragma unroll
-                    for (int m = 0; m < F::kVecs; ++m) R[j][m] = ldg_stream_u128(src + m * 512);
-                }
-                process(v, wu0 + i);
+        for (int m = 0; m < V; ++m) v[m] = *reinterpret_cast<const uint4*>(src + m * 512);
+        issue(i + D, s_fill);
+        s_read = s_read + 1 == S ? 0 : s_read + 1;
+        s_fill = s_fill + 1 == S ? 0 : s_fill + 1;
+        process(v, sg);
+        if (++sg == nsg || i + 1 == nwu) {
+            flush_tile();
+            if (i + 1 < nwu) {
+                ++tile;
+                sg = 0;
+                start_tile();
             }
         }
-    }
-    if (tile >= 0) flush_tile();
-
-    // ---- sparse part: a fixed share of nonzeros per thread (balanced);
-    // its slices were copied while the dense part ran
-    const bool got_c = mbar_wait(cbar, 0);
-    if (!got_c && lane == 0) atomicOr(p.status, kStatusWaitTimeout);
-    const int* s_rp = reinterpret_cast<const int*>(smem + P.off_rp) + rp_off;
-    const int p0 = s_bounds[0], p1 = s_bounds[1];
-    const int nz = p1 - p0;
-    const bool csr_smem = has_csr && nz <= kCsrCap;
-    const int* csr_col = csr_smem ? reinterpret_cast<const int*>(smem + P.off_col) + (p0 & 3) - p0 : p.col;
-    const uint16_t* csr_val =
-        csr_smem ? reinterpret_cast<const uint16_t*>(smem + P.off_val) + (p0 & 7) - p0 : p.val;
-    const int e_per = has_csr ? max(1, (nz + kCsrThreads - 1) / kCsrThreads) : 1;
-    if (has_csr && got_c) {
-        const int a = p0 + tid * e_per;
-        const int b_end = min(p1, a + e_per);
-        if (a < b_end) {
-            // row (relative to ra) containing entry a: largest r with s_rp[r] <= a
-            int lo = 0, hi = nrows - 1;
-            while (lo < hi) {
-                const int mid = (lo + hi + 1) >> 1;
-                if (s_rp[mid] <= a) lo = mid; else hi = mid - 1;
-            }
-            int cur = lo;
-            int nxt = s_rp[cur + 1];
-            bool first = true;
-            float acc[CM];
-#pragma unroll
-            for (int b = 0; b < CM; ++b) acc[b] = 0.f;
-            auto emit = [&](bool last) {
-                float* dstp;
-                if (first) {
-                    s_headrow[tid] = cur;
-                    dstp = s_head + tid * CM;
-                } else if (last) {
-                    s_tailrow[tid] = cur;
-                    dstp = s_tail + tid * CM;
-                } else {
-                    dstp = s_rowsum + cur * CM;
-                }
-#pragma unroll
-                for (int b = 0; b < CM; ++b) dstp[b] = acc[b];
-            };
-            for (int base = a; base < b_end; base += 8) {
-                int cc[8];
-                float vv[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int q = base + j;
-                    cc[j] = q < b_end ? csr_col[q] : 0;
-                    vv[j] = q < b_end ? h2f(csr_val[q]) : 0.f;
-                }
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int q = base + j;
-                    if (q >= b_end) break;
-                    while (q >= nxt) {
-                        emit(false);
-                        first = false;
-#pragma unroll
-                        for (int b = 0; b < CM; ++b) acc[b] = 0.f;
-                        ++cur;
-                        nxt = s_rp[cur + 1];
-                    }
-#pragma unroll
-                    for (int b = 0; b < CM; ++b)
-                        if (SB || b < B) acc[b] = fmaf(vv[j], h2f(xs[b * P.x_stride + cc[j]]), acc[b]);
-                }
-            }
-            emit(true);
-        }
-    }
-    __syncthreads();  // every warp's dense parts and every sparse partial are in shared memory
-
-    // ---- finish the CTA's tiles: sum the warps' parts in warp order, add
-    // the rows' nonzeros (interior sums plus the pieces of the threads whose
-    // shares cut a row, in thread order) and write y
-    for (int idx = tid; idx < ctiles * TE; idx += kThreads) {
-        const int tl = idx / TE, e = idx - tl * TE;
-        const int tile_i = t_first + tl;
-        const int row_l = e / CM, col = e - row_l * CM;
-        const int mask = s_tinfo[tl];
-        float sum;
-        if ((mask & (mask - 1)) == 0) {
-            sum = s_ctile[idx];
-        } else {
-            sum = 0.f;
-            for (int mm = mask; mm; mm &= mm - 1) {
-                const int wv = __ffs(mm) - 1;
-                sum += s_slots[(wv * 2 + (tile_i == s_wrange[wv * 3 + 2] ? 0 : 1)) * TE + e];
-            }
-        }
-        const int row = tile_i * kTileRows + row_l;
-        if (has_csr && row < ra + nrows) {
-            const int i = row - ra;
-            const int rs = s_rp[i], re = s_rp[i + 1];
-            float cs = s_rowsum[i * CM + col];
-            if (re > rs) {
-                const int tau_a = (rs - p0) / e_per, tau_b = min(kCsrThreads - 1, (re - 1 - p0) / e_per);
-                for (int tau = tau_a; tau <= tau_b; ++tau) {
-                    if (s_headrow[tau] == i) cs += s_head[tau * CM + col];
-                    if (s_tailrow[tau] == i) cs += s_tail[tau * CM + col];
-                }
-            }
-            sum += cs;
-        }
-        if (row < p.n_out && col < B) p.y[col * p.ldy + row] = f2h_rn(sum);
     }
 }
 

@@ -72,10 +72,9 @@ struct sqz_layer {
     int device = 0;
     int sm_count = 148;
     int smem_optin = 232448;
-    int smem_per_sm = 233472;
     int mac = SQZ_MAC_TENSOR_CORES;
-    // The fused kernel works on whole k16-steps: K % 16 == 0 (4-bit layers
-    // with K % 16 == 8 use the row-per-warp kernel).
+    // The fused kernel serves every layer with N > 0 and K > 0 (columns past
+    // K are padded inside the kernel-native layout).
     bool fused_ok = false;
     // canonical copies (row-per-warp kernel for requests the fused kernel
     // cannot stage in shared memory)
@@ -89,6 +88,8 @@ struct sqz_layer {
     // kernel-native layout for the fused kernel
     int ntiles = 0, nsteps = 0, nsg = 0;
     int64_t units = 0;
+    int grid = 0;                     // CTAs of a fused launch (one per SM)
+    std::vector<int32_t> csr_cta;     // [grid + 1]: CSR entry range of each CTA's rows
     uint8_t* codes_native = nullptr;  // [ntiles][nsg][sg_bytes]
     uint8_t* lut_native = nullptr;    // [ntiles*16][2 << bits] byte planes
     int* status = nullptr;            // [1]
@@ -136,7 +137,7 @@ sqz_status check_desc(const sqz_layer_desc* d) {
     if (d->k_in % kmult != 0)
         return fail(SQZ_ERR_INVALID_ARG, "k_in=%d must be a multiple of %d for %d-bit codes (whole words per row)",
                     d->k_in, kmult, d->bits);
-    if (d->nnz < 0 || d->nnz > INT32_MAX) return fail(SQZ_ERR_INVALID_ARG, "nnz=%lld out of range", (long long)d->nnz);
+    if (d->nnz < 0 || d->nnz > INT32_MAX - 64) return fail(SQZ_ERR_INVALID_ARG, "nnz=%lld out of range", (long long)d->nnz);
     if ((int64_t)d->n_out * d->k_in > 0 && !d->codes) return fail(SQZ_ERR_INVALID_ARG, "codes is NULL");
     if (d->n_out > 0 && !d->lut) return fail(SQZ_ERR_INVALID_ARG, "lut is NULL");
     if (d->nnz > 0 && (!d->rowptr || !d->col || !d->val))
@@ -180,33 +181,37 @@ void dispatch_rowwarp(const sqz_layer* L, const uint16_t* x, int32_t batch, int6
 }
 
 // ------------------------------------------------------------ fused kernel
-template <int BITS, int NT, bool TC, bool SB>
+template <int BITS, int NT, int MAC, bool SB>
 sqz_status set_smem_attr(int bytes) {
-    SQZ_CUDA_TRY(cudaFuncSetAttribute(sqz::tc::gemv_fused_kernel<BITS, NT, TC, SB>,
+    SQZ_CUDA_TRY(cudaFuncSetAttribute(sqz::tc::gemv_fused_kernel<BITS, NT, MAC, SB>,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, bytes),
                  "cudaFuncSetAttribute");
     return SQZ_OK;
 }
 
-sqz_status prepare_fused_kernels(int optin) {
+template <int BITS>
+sqz_status prepare_fused_bits(int optin) {
+    using namespace sqz::tc;
     sqz_status st;
-    if ((st = set_smem_attr<3, 1, true, true>(optin)) != SQZ_OK) return st;
-    if ((st = set_smem_attr<3, 1, true, false>(optin)) != SQZ_OK) return st;
-    if ((st = set_smem_attr<3, 2, true, false>(optin)) != SQZ_OK) return st;
-    if ((st = set_smem_attr<4, 1, true, true>(optin)) != SQZ_OK) return st;
-    if ((st = set_smem_attr<4, 1, true, false>(optin)) != SQZ_OK) return st;
-    if ((st = set_smem_attr<4, 2, true, false>(optin)) != SQZ_OK) return st;
-    if ((st = set_smem_attr<3, 1, false, true>(optin)) != SQZ_OK) return st;
-    if ((st = set_smem_attr<4, 1, false, true>(optin)) != SQZ_OK) return st;
+    if ((st = set_smem_attr<BITS, 1, kMacTensor, true>(optin)) != SQZ_OK) return st;
+    if ((st = set_smem_attr<BITS, 1, kMacTensor, false>(optin)) != SQZ_OK) return st;
+    if ((st = set_smem_attr<BITS, 2, kMacTensor, false>(optin)) != SQZ_OK) return st;
+    if ((st = set_smem_attr<BITS, 1, kMacCuda, true>(optin)) != SQZ_OK) return st;
+    if ((st = set_smem_attr<BITS, 1, kMacMixed, true>(optin)) != SQZ_OK) return st;
     return SQZ_OK;
+}
+
+sqz_status prepare_fused_kernels(int optin) {
+    sqz_status st = prepare_fused_bits<3>(optin);
+    return st != SQZ_OK ? st : prepare_fused_bits<4>(optin);
 }
 
 // Plan for a call, or false when the fused kernel cannot stage x.
 bool fused_plan(const sqz_layer* L, int batch, sqz::tc::Plan* out) {
     const int nt = batch > 8 ? 2 : 1;
     sqz::tc::Plan P =
-        sqz::tc::make_plan(L->bits, L->n_out, L->k_in, batch, nt, batch == 1, sqz::tc::kCtasPerSm * L->sm_count);
-    if (P.total > L->smem_optin) return false;
+        sqz::tc::make_plan(L->bits, L->n_out, L->k_in, batch, nt, batch == 1, L->sm_count, L->smem_optin);
+    if (P.total > L->smem_optin || P.grid != L->grid) return false;
     *out = P;
     return true;
 }
@@ -214,7 +219,7 @@ bool fused_plan(const sqz_layer* L, int batch, sqz::tc::Plan* out) {
 // Launch with programmatic stream serialization: the kernel may start while
 // the previous kernel of the stream is still running; it prefetches only
 // weights before it waits for that kernel (griddepcontrol.wait).
-template <int BITS, int NT, bool TC, bool SB>
+template <int BITS, int NT, int MAC, bool SB>
 cudaError_t launch_fused(const sqz::tc::Params& prm, cudaStream_t s) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)prm.plan.grid);
@@ -226,7 +231,19 @@ cudaError_t launch_fused(const sqz::tc::Params& prm, cudaStream_t s) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, sqz::tc::gemv_fused_kernel<BITS, NT, TC, SB>, prm);
+    return cudaLaunchKernelEx(&cfg, sqz::tc::gemv_fused_kernel<BITS, NT, MAC, SB>, prm);
+}
+
+// Batch 1 takes the requested multiply-accumulate unit; larger batches the
+// tensor cores (one or two n-tiles of 8 batch columns).
+template <int BITS>
+cudaError_t launch_fused_bits(const sqz::tc::Params& prm, int batch, int mac, cudaStream_t s) {
+    using namespace sqz::tc;
+    if (batch > 8) return launch_fused<BITS, 2, kMacTensor, false>(prm, s);
+    if (batch > 1) return launch_fused<BITS, 1, kMacTensor, false>(prm, s);
+    if (mac == SQZ_MAC_CUDA_CORES) return launch_fused<BITS, 1, kMacCuda, true>(prm, s);
+    if (mac == SQZ_MAC_MIXED) return launch_fused<BITS, 1, kMacMixed, true>(prm, s);
+    return launch_fused<BITS, 1, kMacTensor, true>(prm, s);
 }
 
 sqz_status gemv_impl(const sqz_layer* L, const uint16_t* x, int32_t batch, int64_t ldx, uint16_t* y, int64_t ldy,
@@ -240,7 +257,6 @@ sqz_status gemv_impl(const sqz_layer* L, const uint16_t* x, int32_t batch, int64
         prm.rowptr = L->rowptr;
         prm.col = L->col;
         prm.val = L->val;
-        prm.nnz = L->nnz;
         prm.x = x;
         prm.ldx = ldx;
         prm.y = y;
@@ -248,25 +264,15 @@ sqz_status gemv_impl(const sqz_layer* L, const uint16_t* x, int32_t batch, int64
         prm.status = L->status;
         prm.n_out = L->n_out;
         prm.k_in = L->k_in;
-        prm.nsteps = L->nsteps;
         prm.nsg = L->nsg;
         prm.ntiles = L->ntiles;
         prm.batch = batch;
+        prm.has_csr = L->nnz > 0;
         prm.x_bulk = (reinterpret_cast<uintptr_t>(x) % 16 == 0) && (ldx % 8 == 0) && (L->k_in % 8 == 0);
         prm.plan = P;
-        const bool cuda_cores = L->mac == SQZ_MAC_CUDA_CORES && batch == 1;
-        cudaError_t e;
-        if (L->bits == 3) {
-            if (cuda_cores) e = launch_fused<3, 1, false, true>(prm, s);
-            else if (batch > 8) e = launch_fused<3, 2, true, false>(prm, s);
-            else if (batch > 1) e = launch_fused<3, 1, true, false>(prm, s);
-            else e = launch_fused<3, 1, true, true>(prm, s);
-        } else {
-            if (cuda_cores) e = launch_fused<4, 1, false, true>(prm, s);
-            else if (batch > 8) e = launch_fused<4, 2, true, false>(prm, s);
-            else if (batch > 1) e = launch_fused<4, 1, true, false>(prm, s);
-            else e = launch_fused<4, 1, true, true>(prm, s);
-        }
+        std::memcpy(prm.csr_cta, L->csr_cta.data(), sizeof(int32_t) * L->csr_cta.size());
+        const cudaError_t e = L->bits == 3 ? launch_fused_bits<3>(prm, batch, L->mac, s)
+                                           : launch_fused_bits<4>(prm, batch, L->mac, s);
         SQZ_CUDA_TRY(e, "fused gemv launch");
     } else if (L->bits == 3) {
         dispatch_rowwarp<3>(L, x, batch, ldx, y, ldy, s);
@@ -281,8 +287,9 @@ sqz_status gemv_impl(const sqz_layer* L, const uint16_t* x, int32_t batch, int64
 sqz_status build_native(sqz_layer* L, cudaStream_t s) {
     using namespace sqz::tc;
     L->ntiles = (L->n_out + kTileRows - 1) / kTileRows;
-    L->nsteps = L->k_in / 16;
+    L->nsteps = (L->k_in + 15) / 16;
     L->nsg = (L->nsteps + kSgSteps - 1) / kSgSteps;
+    L->grid = grid_size(L->n_out, L->sm_count);
     L->units = (int64_t)L->ntiles * L->nsg;
     const int sg_bytes = L->bits == 3 ? 1536 : 2048;
     const int lut_row = 2 << L->bits;
@@ -296,13 +303,11 @@ sqz_status build_native(sqz_layer* L, cudaStream_t s) {
         int64_t blocks = (words + 255) / 256;
         if (blocks > (int64_t)L->sm_count * 16) blocks = (int64_t)L->sm_count * 16;
         if (L->bits == 3)
-            sqz::tc::repack_codes_kernel<3><<<(unsigned)blocks, 256, 0, s>>>(L->codes, L->n_out, L->k_in, L->nsg,
-                                                                             words,
-                                                                             reinterpret_cast<uint32_t*>(L->codes_native));
+            repack_codes_kernel<3><<<(unsigned)blocks, 256, 0, s>>>(L->codes, L->lut, L->n_out, L->k_in, L->nsg, words,
+                                                                    reinterpret_cast<uint32_t*>(L->codes_native));
         else
-            sqz::tc::repack_codes_kernel<4><<<(unsigned)blocks, 256, 0, s>>>(L->codes, L->n_out, L->k_in, L->nsg,
-                                                                             words,
-                                                                             reinterpret_cast<uint32_t*>(L->codes_native));
+            repack_codes_kernel<4><<<(unsigned)blocks, 256, 0, s>>>(L->codes, L->lut, L->n_out, L->k_in, L->nsg, words,
+                                                                    reinterpret_cast<uint32_t*>(L->codes_native));
         SQZ_CUDA_TRY(cudaGetLastError(), "repack codes");
     }
     if (L->ntiles > 0) {
@@ -313,6 +318,20 @@ sqz_status build_native(sqz_layer* L, cudaStream_t s) {
         else
             sqz::tc::repack_lut_kernel<4><<<blocks, 256, 0, s>>>(L->lut, L->n_out, rows, L->lut_native);
         SQZ_CUDA_TRY(cudaGetLastError(), "repack lut");
+    }
+    // CSR entry range of every CTA's rows, passed with each launch
+    L->csr_cta.assign((size_t)L->grid + 1, 0);
+    if (L->nnz > 0) {
+        if (L->grid > kMaxCtas) return fail(SQZ_ERR_UNSUPPORTED, "%d CTAs exceed the fused kernel's %d", L->grid, kMaxCtas);
+        int32_t* d_b = nullptr;
+        SQZ_CUDA_TRY(cudaMalloc(&d_b, sizeof(int32_t) * (L->grid + 1)), "CTA bounds allocation");
+        csr_cta_bounds_kernel<<<(L->grid + 256) / 256, 256, 0, s>>>(L->rowptr, L->n_out, L->ntiles, L->grid, d_b);
+        cudaError_t e = cudaGetLastError();
+        if (e == cudaSuccess)
+            e = cudaMemcpyAsync(L->csr_cta.data(), d_b, sizeof(int32_t) * (L->grid + 1), cudaMemcpyDeviceToHost, s);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+        cudaFree(d_b);
+        SQZ_CUDA_TRY(e, "CTA bounds");
     }
     return SQZ_OK;
 }
@@ -337,12 +356,6 @@ sqz_status sqz_create_layer(const sqz_layer_desc* desc, void* stream, sqz_layer_
     L->wpr = (int64_t)desc->k_in * desc->bits / 32;
     L->sm_count = sm_count_of_current_device();
     L->smem_optin = max_smem_optin();
-    {
-        int dev = 0, v = 0;
-        if (cudaGetDevice(&dev) == cudaSuccess &&
-            cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) == cudaSuccess && v > 0)
-            L->smem_per_sm = v;
-    }
     cudaGetDevice(&L->device);
 
     const size_t n = (size_t)desc->n_out, lut_n = n << desc->bits, code_n = n * (size_t)L->wpr;
@@ -415,7 +428,7 @@ sqz_status sqz_create_layer(const sqz_layer_desc* desc, void* stream, sqz_layer_
                         (h_flag & 8) ? " column outside [0,K)" : "");
         }
     }
-    L->fused_ok = L->n_out > 0 && L->k_in > 0 && L->k_in % 16 == 0;
+    L->fused_ok = L->n_out > 0 && L->k_in > 0 && sqz::tc::grid_size(L->n_out, L->sm_count) <= sqz::tc::kMaxCtas;
     if (L->fused_ok) SQZ_STEP(build_native(L, s));
     SQZ_CUDA_STEP(cudaStreamSynchronize(s), "layer creation");
 #undef SQZ_STEP
@@ -486,7 +499,7 @@ sqz_status sqz_layer_info(sqz_layer_t layer, int32_t* n_out, int32_t* k_in, int3
 
 sqz_status sqz_layer_set_mac(sqz_layer_t layer, int32_t mac) {
     if (!layer) return fail(SQZ_ERR_INVALID_ARG, "layer is NULL");
-    if (mac != SQZ_MAC_TENSOR_CORES && mac != SQZ_MAC_CUDA_CORES)
+    if (mac != SQZ_MAC_TENSOR_CORES && mac != SQZ_MAC_CUDA_CORES && mac != SQZ_MAC_MIXED)
         return fail(SQZ_ERR_INVALID_ARG, "unknown MAC unit %d", mac);
     layer->mac = mac;
     return SQZ_OK;

@@ -265,21 +265,93 @@ def test_fp16_yardstick(B, orc):
     assert_close(yd.cpu().numpy().view(np.uint16), ref, bound)
 
 
+@pytest.mark.parametrize("mac", ["cuda", "mixed"])
 @pytest.mark.parametrize("wl", ["llama7b-q-4bit", "llama7b-up-3bit"])
-def test_cuda_core_mac_matches_oracle(B, orc, wl):
-    """The CUDA-core multiply-accumulate variant (batch 1) meets the same
-    bound as the tensor-core one."""
+def test_mac_variants_match_oracle(B, orc, wl, mac):
+    """The CUDA-core and the split tensor/CUDA-core multiply-accumulate
+    variants (batch 1) meet the same bound as the tensor-core one."""
     shape = synth.workloads()[wl][0]
     L = synth.layer_for(shape)
     x = synth.x_for(shape)
     layer = upload(B, L)
     y_tc = gpu_gemv(B, layer, x)
-    B.sqz_layer_set_mac(layer, B.SQZ_MAC_CUDA_CORES)
-    y_cc = gpu_gemv(B, layer, x)
+    B.sqz_layer_set_mac(layer, B.SQZ_MAC_CUDA_CORES if mac == "cuda" else B.SQZ_MAC_MIXED)
+    y_v = gpu_gemv(B, layer, x)
     y_ref, bound = orc.gemv_layer(L, x)
-    assert_close(y_cc, y_ref, bound, "cuda cores")
+    assert_close(y_v, y_ref, bound, mac)
     assert_close(y_tc, y_ref, bound, "tensor cores")
     assert B.sqz_layer_status(layer) == 0
+    # a batch > 1 call keeps the tensor cores whatever the choice
+    x3 = synth.make_x(3, shape.k_in, seed=12)
+    y_ref3, bound3 = orc.gemv_layer(L, x3)
+    assert_close(gpu_gemv(B, layer, x3), y_ref3, bound3, "batch 3")
+
+
+@pytest.mark.parametrize("bits,k_in", [(3, 288), (3, 4128), (4, 264), (4, 1000)])
+@pytest.mark.parametrize("mac", ["tensor", "mixed"])
+def test_padded_columns_with_nonfinite_lut_entries(B, orc, bits, k_in, mac):
+    """K not a multiple of 256: the columns past K inside the last
+    super-group are padding.  Rows whose LUT holds inf/NaN entries that no
+    real code selects must still give finite, exact results (the padding
+    must not pick a non-finite entry), and the dequantized export must stay
+    bit-exact."""
+    n_out = 70
+    L = make_small(61 + k_in, n_out, k_in, bits, 50)
+    rng = np.random.default_rng(k_in)
+    nlev = 1 << bits
+    lut = L.lut.copy()
+    lut[::3, 0] = 0x7C00   # +inf
+    lut[1::3, 0] = 0xFC00  # -inf
+    lut[1::3, 1] = 0x7E00  # NaN
+    lut[2::3, :nlev - 1] = 0x7C00  # only the last entry finite
+    # codes: rows 0,1 (mod 3) never use entries 0/1, rows 2 (mod 3) only the last
+    codes_mat = rng.integers(2, nlev, size=(n_out, k_in))
+    codes_mat[2::3] = nlev - 1
+    bitsarr = ((codes_mat[:, :, None] >> np.arange(bits)) & 1).reshape(n_out, -1)
+    words = np.packbits(bitsarr.astype(np.uint8), axis=1, bitorder="little").view("<u4")
+    Lx = synth.Layer(n_out, k_in, bits, np.ascontiguousarray(words), lut, L.rowptr, L.col, L.val)
+    layer = upload(B, Lx)
+    if mac == "mixed":
+        B.sqz_layer_set_mac(layer, B.SQZ_MAC_MIXED)
+    for batch in (1, 3):
+        x = synth.make_x(batch, k_in, seed=batch)
+        y = gpu_gemv(B, layer, x)
+        y_ref, bound = orc.gemv_layer(Lx, x)
+        assert np.isfinite(y_ref).all()
+        assert_close(y, y_ref, bound, f"batch {batch}")
+    w = torch.empty((n_out, k_in), dtype=torch.int16, device="cuda")
+    B.sqz_debug_dequant(layer, w)
+    torch.cuda.synchronize()
+    assert np.array_equal(w.cpu().numpy().view(np.uint16), orc.dequant(Lx.codes, Lx.lut, n_out, k_in, bits))
+
+
+def test_chained_calls_read_the_previous_output(B, orc):
+    """Back-to-back calls on one stream where each call's x is the previous
+    call's y: a launch may start before the previous kernel ends, and must
+    still read x only after that kernel has written it."""
+    dims = [4096, 1024, 2048, 4096, 512]
+    layers, hosts = [], []
+    for i in range(len(dims) - 1):
+        L = make_small(70 + i, dims[i + 1], dims[i], 3 if i % 2 == 0 else 4, dims[i + 1] * 3)
+        hosts.append(L)
+        layers.append(upload(B, L))
+    x0 = synth.make_x(1, dims[0], seed=4)
+    bufs = [torch.from_numpy(x0.view(np.int16)).cuda()]
+    for d in dims[1:]:
+        bufs.append(torch.full((1, d), 0x7E00, dtype=torch.int16, device="cuda"))
+    torch.cuda.synchronize()
+    for rep in range(3):
+        for i, layer in enumerate(layers):
+            B.sqz_gemv(layer, bufs[i], bufs[i + 1])
+        torch.cuda.synchronize()
+        x = x0
+        for i, L in enumerate(hosts):
+            y = bufs[i + 1].cpu().numpy().view(np.uint16)
+            y_ref, bound = orc.gemv_layer(L, x)
+            assert_close(y, y_ref, bound, f"rep {rep} layer {i}")
+            x = y  # the next layer's input is what the GPU produced
+        for b in bufs[1:]:
+            b.fill_(0x7E00)
 
 
 def test_status_word_clear_after_runs(B):
