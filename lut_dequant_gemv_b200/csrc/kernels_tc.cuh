@@ -9,8 +9,10 @@
 //     super-groups of 256 (16 k16-steps).  A unit = (tile, super-group).
 //   * One CTA of 16 warps per SM.  Each CTA owns a contiguous run of whole
 //     tiles (runs differ by at most one tile) and its warps split the CTA's
-//     units into equal contiguous ranges, so a tile is finished inside one
-//     CTA: no global atomics, no second pass.
+//     units into contiguous ranges (equal, except that the eight warps that
+//     also sum the sparse part take one unit less each when there is one),
+//     so a tile is finished inside one CTA: no global atomics, no second
+//     pass.
 //   * A tile held by several warps is finished by the warp that flushes its
 //     part last (a shared-memory arrival counter): it adds the parts in warp
 //     order -- deterministic -- and writes y while the other warps keep
@@ -51,8 +53,9 @@
 // steps on the tensor cores, odd steps on the CUDA cores, batch 1).
 //
 // Sparse part: the CSR entries of the rows of a CTA's tiles are split evenly
-// over its threads (a fixed number of nonzeros per thread, independent of
-// how skewed the rows are) -- the balanced scheme of the pages.  Each thread
+// over 256 of its threads (a fixed number of nonzeros per thread,
+// independent of how skewed the rows are) -- the balanced scheme of the
+// pages.  Each thread
 // sums its share per row before entering the dense loop, while the code
 // units are in flight, and signals an mbarrier; no CTA barrier follows.
 // The warp that finishes a tile waits on that mbarrier and adds to each row
@@ -67,19 +70,26 @@
 namespace sqz {
 namespace tc {
 
-constexpr int kWarps = 16;
+constexpr int kWarps = 12;
 constexpr int kThreads = kWarps * 32;
-// Threads sharing the sparse part: all of them while the per-thread pieces
-// are small (up to 8 batch columns), half of them for 16 columns.  Batch 1
-// and batches up to 8 split the entries identically (same sums per column).
-__host__ __device__ constexpr int csr_threads_for(int cm) { return cm <= 8 ? 512 : 256; }
+// Two CTAs fit on an SM: while one call's CTA decodes, the next call's CTA
+// (programmatic dependent launch) already streams its own weights in.
+constexpr int kCtasPerSm = 2;
+constexpr int kCsrThreads = 256;  // threads sharing the sparse part (warps 0-7; the same split for every batch)
+constexpr int kCsrWarps = kCsrThreads / 32;
+static_assert(kCsrWarps <= kWarps, "the sparse part runs on the CTA's first warps");
+// Dense units that each sparse warp hands to a non-sparse warp when the
+// layer has outliers: the sparse share delays a warp's dense start by about
+// one unit's decode time.
+constexpr int kCsrUnitShift = 1;
 constexpr int kTileRows = 16;
 constexpr int kSgSteps = 16;      // k16-steps per super-group
 constexpr int kSgCols = 256;      // columns per super-group
 constexpr int kMaxCtas = 512;     // CTAs per launch (one per SM)
 constexpr int kMinStages = 2;     // shared-memory stages per warp (units in flight + 1)
-constexpr int kMaxStages = 6;
-constexpr int kPreWait = 2;       // code units per warp requested before waiting for the previous kernel
+constexpr int kMaxStages = 16;
+constexpr int kPreWait = 2;       // code units per warp requested before waiting for the previous kernel;
+                                  // the rest of the first ring follows once x has landed
 constexpr int kCsrCap = 4096;     // CSR entries per CTA staged in shared memory, at most (more: read from global)
 constexpr uint32_t kSuspendNs = 1000000u;  // 1 ms per poll
 constexpr uint32_t kWaitLimit = 2000u;
@@ -124,8 +134,23 @@ struct Plan {
 
 __host__ __device__ inline int round_up(int v, int m) { return (v + m - 1) / m * m; }
 
-// First tile of CTA c when `ntiles` tiles are split over `grid` CTAs.
-__host__ __device__ inline int tile_begin(int ntiles, int grid, int c) { return (int)((int64_t)ntiles * c / grid); }
+// First tile of CTA c when `ntiles` tiles are split over `grid` CTAs: the
+// first ntiles % grid CTAs take one tile more (32-bit arithmetic only).
+__host__ __device__ inline int tile_begin(int ntiles, int grid, int c) {
+    const int q = ntiles / grid, r = ntiles - q * grid;
+    return c * q + (c < r ? c : r);
+}
+
+// First unit of warp w among a CTA's units [u0, u0 + cn): an even split,
+// except that the sparse warps (0..kCsrWarps-1) give `shift` units each to
+// the other warps (spread evenly over them).
+__host__ __device__ inline int warp_unit_begin(int u0, int cn, int w, int shift) {
+    if (cn < 4 * kWarps || kCsrWarps == kWarps) shift = 0;
+    const int moved = kCsrWarps * shift;
+    const int base = cn - moved;
+    const int extra = w > kCsrWarps ? moved * (w - kCsrWarps) / (kWarps - kCsrWarps) : 0;
+    return u0 + base * w / kWarps + extra;
+}
 
 // CTAs of a launch: one per SM, at most one per tile.
 __host__ __device__ inline int grid_size(int n_out, int sms) {
@@ -164,7 +189,7 @@ __host__ __device__ inline Plan make_plan(int bits, int n_out, int k_in, int bat
     P.off_rowsum = off;
     off += round_up(rows * P.cm * 4, 128);
     // the sparse pieces of the threads and the warps' parts of shared tiles
-    const int ct = csr_threads_for(P.cm);
+    const int ct = kCsrThreads;
     P.off_head = off;
     P.off_tail = off + ct * P.cm * 4;
     P.off_headrow = P.off_tail + ct * P.cm * 4;
@@ -198,8 +223,15 @@ __host__ __device__ inline Plan make_plan(int bits, int n_out, int k_in, int bat
     return P;
 }
 
+// The fields read first sit together at the start (parameter reads that
+// miss the constant cache are slow at kernel start).
 struct Params {
     const uint8_t* codes;    // [ntiles][nsg][sg_bytes], kernel-native layout
+    int n_out, k_in, nsg, ntiles, batch;
+    int has_csr;             // the layer has outliers
+    int x_bulk;              // 1: every x row is 16-byte aligned -> bulk copies
+    int pad_;
+    Plan plan;
     const uint8_t* lutp;     // [ntiles*16][lut_bytes], byte planes
     const int32_t* rowptr;   // canonical CSR (device copies owned by the layer)
     const int32_t* col;
@@ -209,10 +241,6 @@ struct Params {
     uint16_t* y;
     int64_t ldy;
     int* status;             // error bits (bounded waits that gave up)
-    int n_out, k_in, nsg, ntiles, batch;
-    int has_csr;             // the layer has outliers
-    int x_bulk;              // 1: every x row is 16-byte aligned -> bulk copies
-    Plan plan;
     // CSR entries of the rows of CTA c: [csr_cta[c], csr_cta[c+1]); all zero
     // when the layer has no outliers.
     int32_t csr_cta[kMaxCtas + 1];
@@ -271,11 +299,13 @@ __device__ __forceinline__ void cp_async_wait() {
 }
 __device__ __forceinline__ void cp_async_wait_newest(int n) {
     switch (n) {
-        case 0: cp_async_wait<0>(); break;
-        case 1: cp_async_wait<1>(); break;
-        case 2: cp_async_wait<2>(); break;
-        case 3: cp_async_wait<3>(); break;
-        default: cp_async_wait<4>(); break;
+#define SQZ_WAIT_CASE(k) \
+    case k: cp_async_wait<k>(); break;
+        SQZ_WAIT_CASE(0) SQZ_WAIT_CASE(1) SQZ_WAIT_CASE(2) SQZ_WAIT_CASE(3) SQZ_WAIT_CASE(4) SQZ_WAIT_CASE(5)
+        SQZ_WAIT_CASE(6) SQZ_WAIT_CASE(7) SQZ_WAIT_CASE(8) SQZ_WAIT_CASE(9) SQZ_WAIT_CASE(10) SQZ_WAIT_CASE(11)
+        SQZ_WAIT_CASE(12) SQZ_WAIT_CASE(13)
+#undef SQZ_WAIT_CASE
+        default: cp_async_wait<14>(); break;
     }
 }
 __device__ __forceinline__ void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
@@ -516,15 +546,14 @@ __global__ void dequant_native_kernel(const uint8_t* __restrict__ codes, const u
 // MAC: kMacTensor / kMacCuda / kMacMixed.  SB: batch 1 (one column carried
 // through the sparse part and the combine).
 template <int BITS, int NT, int MAC, bool SB>
-__global__ void __launch_bounds__(kThreads, 1) gemv_fused_kernel(const __grid_constant__ Params p) {
+__global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_fused_kernel(const __grid_constant__ Params p) {
     using F = Fmt<BITS>;
     using TAB = typename std::conditional<BITS == 3, Tab3, Tab4>::type;
     constexpr int BM = 8 * NT;              // batch columns of the MMA accumulators
     constexpr int CM = SB ? 1 : BM;         // batch columns carried after the dense loop
     constexpr int TE = kTileRows * CM;      // elements of one tile's result
     constexpr int V = F::kVecs;
-    constexpr int CT = csr_threads_for(CM);  // threads sharing the sparse part
-    static_assert(CT <= kThreads, "sparse part runs on the CTA's threads");
+    constexpr int CT = kCsrThreads;
     static_assert(!SB || NT == 1, "single-batch variant uses one n-tile");
     static_assert(MAC == kMacTensor || SB, "CUDA-core multiply-accumulates carry one batch column");
     extern __shared__ __align__(128) uint8_t smem[];
@@ -539,7 +568,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_fused_kernel(const __grid_co
     const int t_first = tile_begin(p.ntiles, G, c), t_end = tile_begin(p.ntiles, G, c + 1);
     const int ctiles = t_end - t_first;
     const int u0 = t_first * nsg, cn = ctiles * nsg;  // the CTA's units: [u0, u0 + cn)
-    const int wu0 = u0 + cn * warp / kWarps, wu1 = u0 + cn * (warp + 1) / kWarps;
+    const int shift = p.has_csr ? kCsrUnitShift : 0;
+    const int wu0 = warp_unit_begin(u0, cn, warp, shift), wu1 = warp_unit_begin(u0, cn, warp + 1, shift);
     const int nwu = wu1 - wu0;
     const int wfirst = nwu > 0 ? wu0 / nsg : -1;  // first tile of this warp
 
@@ -619,7 +649,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_fused_kernel(const __grid_co
         const int ta_u = (t_first + tl) * nsg, tb_u = ta_u + nsg;
         int mask = 0;
         for (int wv = 0; wv < kWarps; ++wv) {
-            const int a = u0 + cn * wv / kWarps, b = u0 + cn * (wv + 1) / kWarps;
+            const int a = warp_unit_begin(u0, cn, wv, shift), b = warp_unit_begin(u0, cn, wv + 1, shift);
             if (max(a, ta_u) < min(b, tb_u)) mask |= 1 << wv;
         }
         s_tinfo[tl] = mask;
@@ -656,14 +686,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_fused_kernel(const __grid_co
             xs[b * P.x_stride + k] = p.x[b * p.ldx + k];
         }
     }
-    // ---- the rest of the first D units
-    for (int j = pre; j < D; ++j) issue(j, j);
     // Each thread waits for the copies itself (an mbarrier wait makes the
     // bulk-copied bytes visible to it); only x copied by the threads needs a
     // barrier.
     const bool got_l = mbar_wait(lbar, 0), got_x = mbar_wait(xbar, 0), got_c = mbar_wait(cbar, 0);
     if (!(got_l && got_x && got_c)) atomicOr(p.status, kStatusWaitTimeout);
     if (!p.x_bulk) __syncthreads();
+    // ---- the rest of the first D units (after x, which they would delay)
+    for (int j = pre; j < D; ++j) issue(j, j);
 
     // ---- the CTA's CSR entries [q0, q1), a fixed share e_per per thread
     const int q0 = p.csr_cta[c], q1 = p.csr_cta[c + 1];

@@ -72,6 +72,7 @@ struct sqz_layer {
     int device = 0;
     int sm_count = 148;
     int smem_optin = 232448;
+    int smem_budget = 232448;  // shared memory of one fused CTA (kCtasPerSm of them share an SM)
     int mac = SQZ_MAC_TENSOR_CORES;
     // The fused kernel serves every layer with N > 0 and K > 0 (columns past
     // K are padded inside the kernel-native layout).
@@ -206,14 +207,20 @@ sqz_status prepare_fused_kernels(int optin) {
     return st != SQZ_OK ? st : prepare_fused_bits<4>(optin);
 }
 
-// Plan for a call, or false when the fused kernel cannot stage x.
+// Plan for a call, or false when the fused kernel cannot stage x.  A call
+// first gets an SM's share (two CTAs per SM, so the next call's CTA can
+// stream its weights while this one computes); one whose x does not fit
+// there gets a whole SM.
 bool fused_plan(const sqz_layer* L, int batch, sqz::tc::Plan* out) {
     const int nt = batch > 8 ? 2 : 1;
-    sqz::tc::Plan P =
-        sqz::tc::make_plan(L->bits, L->n_out, L->k_in, batch, nt, batch == 1, L->sm_count, L->smem_optin);
-    if (P.total > L->smem_optin || P.grid != L->grid) return false;
-    *out = P;
-    return true;
+    for (int budget : {L->smem_budget, L->smem_optin}) {
+        sqz::tc::Plan P = sqz::tc::make_plan(L->bits, L->n_out, L->k_in, batch, nt, batch == 1, L->sm_count, budget);
+        if (P.total <= budget && P.grid == L->grid) {
+            *out = P;
+            return true;
+        }
+    }
+    return false;
 }
 
 // Launch with programmatic stream serialization: the kernel may start while
@@ -250,30 +257,43 @@ sqz_status gemv_impl(const sqz_layer* L, const uint16_t* x, int32_t batch, int64
                      cudaStream_t s) {
     if (L->n_out == 0) return SQZ_OK;
     sqz::tc::Plan P;
-    if (L->fused_ok && fused_plan(L, batch, &P)) {
-        sqz::tc::Params prm{};
-        prm.codes = L->codes_native;
-        prm.lutp = L->lut_native;
-        prm.rowptr = L->rowptr;
-        prm.col = L->col;
-        prm.val = L->val;
-        prm.x = x;
-        prm.ldx = ldx;
-        prm.y = y;
-        prm.ldy = ldy;
-        prm.status = L->status;
-        prm.n_out = L->n_out;
-        prm.k_in = L->k_in;
-        prm.nsg = L->nsg;
-        prm.ntiles = L->ntiles;
-        prm.batch = batch;
-        prm.has_csr = L->nnz > 0;
-        prm.x_bulk = (reinterpret_cast<uintptr_t>(x) % 16 == 0) && (ldx % 8 == 0) && (L->k_in % 8 == 0);
-        prm.plan = P;
-        std::memcpy(prm.csr_cta, L->csr_cta.data(), sizeof(int32_t) * L->csr_cta.size());
-        const cudaError_t e = L->bits == 3 ? launch_fused_bits<3>(prm, batch, L->mac, s)
-                                           : launch_fused_bits<4>(prm, batch, L->mac, s);
-        SQZ_CUDA_TRY(e, "fused gemv launch");
+    // Columns per launch: the whole batch when its x fits in shared memory,
+    // else chunks of 8, 4, 2 or 1 columns (each launch reads the weights).
+    int chunk = batch;
+    bool fits = L->fused_ok && fused_plan(L, chunk, &P);
+    while (L->fused_ok && !fits && chunk > 1) {
+        chunk = chunk > 8 ? 8 : chunk / 2;
+        fits = fused_plan(L, chunk, &P);
+    }
+    if (fits) {
+        for (int b0 = 0; b0 < batch; b0 += chunk) {
+            const int nb = batch - b0 < chunk ? batch - b0 : chunk;
+            if (nb != chunk && !fused_plan(L, nb, &P)) return fail(SQZ_ERR_UNSUPPORTED, "no fused plan for %d columns", nb);
+            const uint16_t* xc = x + (int64_t)b0 * ldx;
+            sqz::tc::Params prm{};
+            prm.codes = L->codes_native;
+            prm.lutp = L->lut_native;
+            prm.rowptr = L->rowptr;
+            prm.col = L->col;
+            prm.val = L->val;
+            prm.x = xc;
+            prm.ldx = ldx;
+            prm.y = y + (int64_t)b0 * ldy;
+            prm.ldy = ldy;
+            prm.status = L->status;
+            prm.n_out = L->n_out;
+            prm.k_in = L->k_in;
+            prm.nsg = L->nsg;
+            prm.ntiles = L->ntiles;
+            prm.batch = nb;
+            prm.has_csr = L->nnz > 0;
+            prm.x_bulk = (reinterpret_cast<uintptr_t>(xc) % 16 == 0) && (ldx % 8 == 0) && (L->k_in % 8 == 0);
+            prm.plan = P;
+            std::memcpy(prm.csr_cta, L->csr_cta.data(), sizeof(int32_t) * L->csr_cta.size());
+            const cudaError_t e = L->bits == 3 ? launch_fused_bits<3>(prm, nb, L->mac, s)
+                                               : launch_fused_bits<4>(prm, nb, L->mac, s);
+            SQZ_CUDA_TRY(e, "fused gemv launch");
+        }
     } else if (L->bits == 3) {
         dispatch_rowwarp<3>(L, x, batch, ldx, y, ldy, s);
     } else {
@@ -356,6 +376,16 @@ sqz_status sqz_create_layer(const sqz_layer_desc* desc, void* stream, sqz_layer_
     L->wpr = (int64_t)desc->k_in * desc->bits / 32;
     L->sm_count = sm_count_of_current_device();
     L->smem_optin = max_smem_optin();
+    {
+        // an SM's shared memory split between kCtasPerSm CTAs, less the 1 KiB
+        // the hardware reserves per CTA
+        int dev = 0, per_sm = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess)
+            per_sm = 233472;
+        const int share = per_sm / sqz::tc::kCtasPerSm - 1024;
+        L->smem_budget = share < L->smem_optin ? share : L->smem_optin;
+    }
     cudaGetDevice(&L->device);
 
     const size_t n = (size_t)desc->n_out, lut_n = n << desc->bits, code_n = n * (size_t)L->wpr;
