@@ -670,6 +670,43 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_fused_kernel(const 
     }
     __syncthreads();
 
+    // ---- the CTA's CSR entries [q0, q1), a fixed share e_per per thread
+    const int q0 = p.csr_cta[c], q1 = p.csr_cta[c + 1];
+    const int nz = q1 - q0;
+    const bool has_csr = nz > 0;
+    const bool csr_in_smem = has_csr && nz <= P.csr_cap;
+    const int e_per = has_csr ? (int)(((int64_t)nz + CT - 1) / CT) : 1;
+    const int ca = tid < CT ? (int)min((int64_t)q1, (int64_t)q0 + (int64_t)tid * e_per) : q1;
+    const int cb = (int)min((int64_t)q1, (int64_t)ca + e_per);
+    const int* csr_col = csr_in_smem ? reinterpret_cast<const int*>(smem + P.off_col) + (q0 & 3) - q0 : p.col;
+    const uint16_t* csr_val =
+        csr_in_smem ? reinterpret_cast<const uint16_t*>(smem + P.off_val) + (q0 & 7) - q0 : p.val;
+    // The part of a thread's sparse share that does not need x -- the row of
+    // its first entry and its first entries -- is done before the wait for
+    // the previous kernel, while that kernel still computes.
+    int cur = 0, nxt = 0;
+    int cc[8];
+    uint32_t vh[8];
+    bool got_early = true;
+    if (has_csr && ca < cb) {
+        got_early = mbar_wait(lbar, 0) && mbar_wait(cbar, 0);
+        // row (relative to ra) containing entry ca: largest r with s_rp[r] <= ca
+        int lo = 0, hi = nrows - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (s_rp[mid] <= ca) lo = mid; else hi = mid - 1;
+        }
+        cur = lo;
+        nxt = s_rp[cur + 1];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int q = ca + j;
+            const bool in = q < cb;
+            cc[j] = in ? csr_col[q] : 0;
+            vh[j] = in ? (uint32_t)csr_val[q] : 0u;
+        }
+    }
+
     // ---- x may be written by the previous kernel of the stream: wait for it
     pdl_wait_previous();
     if (tid == 0) {
@@ -690,37 +727,17 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_fused_kernel(const 
     // bulk-copied bytes visible to it); only x copied by the threads needs a
     // barrier.
     const bool got_l = mbar_wait(lbar, 0), got_x = mbar_wait(xbar, 0), got_c = mbar_wait(cbar, 0);
-    if (!(got_l && got_x && got_c)) atomicOr(p.status, kStatusWaitTimeout);
+    if (!(got_l && got_x && got_c && got_early)) atomicOr(p.status, kStatusWaitTimeout);
     if (!p.x_bulk) __syncthreads();
     // ---- the rest of the first D units (after x, which they would delay)
     for (int j = pre; j < D; ++j) issue(j, j);
-
-    // ---- the CTA's CSR entries [q0, q1), a fixed share e_per per thread
-    const int q0 = p.csr_cta[c], q1 = p.csr_cta[c + 1];
-    const int nz = q1 - q0;
-    const bool has_csr = nz > 0;
-    const bool csr_in_smem = has_csr && nz <= P.csr_cap;
-    const int e_per = has_csr ? (int)(((int64_t)nz + CT - 1) / CT) : 1;
-    const int ca = tid < CT ? (int)min((int64_t)q1, (int64_t)q0 + (int64_t)tid * e_per) : q1;
-    const int cb = (int)min((int64_t)q1, (int64_t)ca + e_per);
 
     // ---- sparse part: a fixed share of nonzeros per thread (balanced).
     // Each thread sums its entries per row: the first and last rows it
     // touches go to head/tail pieces, rows it holds entirely to s_rowsum;
     // then it arrives on rbar.  No CTA barrier: the warp that finishes a
     // tile waits on rbar and combines the pieces of the tile's rows.
-    const int* csr_col = csr_in_smem ? reinterpret_cast<const int*>(smem + P.off_col) + (q0 & 3) - q0 : p.col;
-    const uint16_t* csr_val =
-        csr_in_smem ? reinterpret_cast<const uint16_t*>(smem + P.off_val) + (q0 & 7) - q0 : p.val;
     if (has_csr && ca < cb) {
-        // row (relative to ra) containing entry ca: largest r with s_rp[r] <= ca
-        int lo = 0, hi = nrows - 1;
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (s_rp[mid] <= ca) lo = mid; else hi = mid - 1;
-        }
-        int cur = lo;
-        int nxt = s_rp[cur + 1];
         bool first = true;
         float acc[CM];
 #pragma unroll
@@ -740,14 +757,14 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_fused_kernel(const 
             for (int b = 0; b < CM; ++b) dstp[b] = acc[b];
         };
         for (int base = ca; base < cb; base += 8) {
-            int cc[8];
-            uint32_t vh[8];
+            if (base != ca) {
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const int q = base + j;
-                const bool in = q < cb;
-                cc[j] = in ? csr_col[q] : 0;
-                vh[j] = in ? (uint32_t)csr_val[q] : 0u;
+                for (int j = 0; j < 8; ++j) {
+                    const int q = base + j;
+                    const bool in = q < cb;
+                    cc[j] = in ? csr_col[q] : 0;
+                    vh[j] = in ? (uint32_t)csr_val[q] : 0u;
+                }
             }
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
