@@ -123,13 +123,16 @@ struct Plan {
     int grid;        // CTAs
     int ctiles_max;  // max tiles owned by one CTA
     int x_stride;    // shared-memory row stride of x, in halves
-    int x_cols;      // columns of x kept in shared memory (nsg * 256; zero past K)
+    int x_cols;      // columns of x kept in a shared-memory buffer (chunk_sg * 256; zero past K)
+    int passes;      // passes over K (1, or more when x is staged in K chunks)
+    int chunk_sg;    // super-groups of x per pass
+    int xbufs;       // x buffers (2 when passes > 1: the next chunk loads during a pass)
     int cm;          // batch columns carried by the sparse part and the combine (1 or 8*NT)
     int stages;      // shared-memory stages of each warp's code ring
     int csr_cap;     // CSR entries of a CTA that are staged in shared memory (more: read from global)
     // byte offsets
     int off_x, off_lut, off_rp, off_rowsum, off_head, off_tail, off_headrow, off_tailrow, off_slots, off_wrange,
-        off_tinfo, off_cnt, off_col, off_val, off_ring, total;
+        off_tinfo, off_cnt, off_col, off_val, off_acc, off_ring, total;
 };
 
 __host__ __device__ inline int round_up(int v, int m) { return (v + m - 1) / m * m; }
@@ -163,8 +166,10 @@ __host__ __device__ inline int grid_size(int n_out, int sms) {
 // ring gets kMinStages stages per warp, the CSR staging area what is left up
 // to kCsrCap entries, and the ring more stages (up to kMaxStages) from the
 // rest; total > budget when not even kMinStages fit.
+// `passes` > 1 stages x in K chunks of chunk_sg super-groups (two buffers)
+// and keeps per-tile sums in shared memory between passes.
 __host__ __device__ inline Plan make_plan(int bits, int n_out, int k_in, int batch, int nt, bool single, int sms,
-                                          int budget) {
+                                          int budget, int passes = 1) {
     Plan P{};
     const int ntiles = (n_out + kTileRows - 1) / kTileRows;
     const int nsteps = (k_in + 15) / 16;
@@ -173,7 +178,11 @@ __host__ __device__ inline Plan make_plan(int bits, int n_out, int k_in, int bat
     P.grid = grid_size(n_out, sms);
     P.ctiles_max = (ntiles + P.grid - 1) / P.grid;
     P.cm = single ? 1 : 8 * nt;
-    P.x_cols = nsg * kSgCols;
+    P.passes = passes < 1 ? 1 : (passes > nsg ? nsg : passes);
+    P.chunk_sg = (nsg + P.passes - 1) / P.passes;
+    P.passes = (nsg + P.chunk_sg - 1) / P.chunk_sg;
+    P.xbufs = P.passes > 1 ? 2 : 1;
+    P.x_cols = P.chunk_sg * kSgCols;
     // x rows: stride = 32 (mod 128) bytes keeps the batch rows of one
     // fragment load in different banks.
     const int xs_bytes = round_up(P.x_cols * 2, 128) + 32;
@@ -181,7 +190,7 @@ __host__ __device__ inline Plan make_plan(int bits, int n_out, int k_in, int bat
     const int rows = P.ctiles_max * kTileRows;
     int off = 128;  // two mbarriers
     P.off_x = off;
-    off += round_up(batch * xs_bytes, 128);
+    off += P.xbufs * round_up(batch * xs_bytes, 128);
     P.off_lut = off;
     off += round_up(rows * lut_bytes, 128);
     P.off_rp = off;
@@ -204,6 +213,8 @@ __host__ __device__ inline Plan make_plan(int bits, int n_out, int k_in, int bat
     P.off_cnt = off;
     off += round_up(P.ctiles_max * 4, 16);
     off = round_up(off, 128);
+    P.off_acc = off;  // per-tile sums across passes
+    if (P.passes > 1) off += round_up(rows * P.cm * 4, 128);
     const int sg_bytes = bits == 3 ? 1536 : 2048;
     const int ring_min = kMinStages * kWarps * sg_bytes;
     int cap = (budget - off - ring_min - 512) / 6;  // 4-byte column + 2-byte value per entry
@@ -308,6 +319,7 @@ __device__ __forceinline__ void cp_async_wait_newest(int n) {
         default: cp_async_wait<14>(); break;
     }
 }
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ __forceinline__ void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
 // Programmatic dependent launch: let the next kernel of the stream start
 // (its CTAs may begin on SMs this grid leaves), and wait until the previous
@@ -584,7 +596,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_fused_kernel(const 
     uint64_t* xbar = reinterpret_cast<uint64_t*>(smem) + 1;  // x
     uint64_t* cbar = reinterpret_cast<uint64_t*>(smem) + 2;  // CSR slices
     uint64_t* rbar = reinterpret_cast<uint64_t*>(smem) + 3;  // sparse pieces written (CT arrivals)
+    uint64_t* xbar1 = reinterpret_cast<uint64_t*>(smem) + 4;  // second x buffer (several passes)
     uint16_t* xs = reinterpret_cast<uint16_t*>(smem + P.off_x);
+    const int PS = P.passes, CS = P.chunk_sg;
+    const int xbuf_h = round_up(p.batch * P.x_stride * 2, 128) / 2;  // halves per x buffer
     uint8_t* luts = smem + P.off_lut;
     float* s_rowsum = reinterpret_cast<float*>(smem + P.off_rowsum);
     float* s_head = reinterpret_cast<float*>(smem + P.off_head);
@@ -605,6 +620,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_fused_kernel(const 
         mbar_init(xbar, 1);
         mbar_init(cbar, 1);
         mbar_init(rbar, CT);
+        mbar_init(xbar1, 1);
         fence_mbar_init();
         const uint32_t lut_bytes = (uint32_t)ctiles * kTileRows * F::kLutBytes;
         const uint32_t rp_bytes = layer_csr ? (uint32_t)round_up(nrows + 1 + rp_off, 4) * 4 : 0u;
@@ -626,17 +642,39 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_fused_kernel(const 
     // pieces (coalesced: a warp-wide copy covers 512 consecutive bytes).
     const int S = P.stages, D = S - 1;
     uint8_t* ring = smem + P.off_ring + warp * S * F::kSgBytes + lane * 16;
-    auto issue = [&](int i, int stage) {
-        if (i < nwu) {
-            const uint8_t* src = p.codes + (int64_t)(wu0 + i) * F::kSgBytes + lane * 16;
+    // Several passes over K: pass q covers super-groups [q*CS, q*CS + cs(q)) of
+    // every tile of the CTA; its ctiles*cs(q) units are split evenly over the
+    // warps.  One pass: the warp's units are [wu0, wu1).
+    auto pass_cs = [&](int q) { return min(CS, nsg - q * CS); };
+    auto prange = [&](int q, int w, int& a, int& b) {
+        const int n = ctiles * pass_cs(q);
+        a = n * w / kWarps;
+        b = n * (w + 1) / kWarps;
+    };
+    auto pass_unit = [&](int q, int j) {
+        const int cs = pass_cs(q), tl = j / cs;
+        return (t_first + tl) * nsg + q * CS + (j - tl * cs);
+    };
+    // producer cursor over this warp's unit sequence (all passes in order)
+    int pq = 0, pj = wu0 - u0, pend = wu1 - u0;
+    if (PS > 1) {
+        prange(0, warp, pj, pend);
+        while (pj >= pend && ++pq < PS) prange(pq, warp, pj, pend);
+    }
+    auto issue = [&](int stage) {
+        if (pq < PS) {
+            const int unit = PS == 1 ? u0 + pj : pass_unit(pq, pj);
+            const uint8_t* src = p.codes + (int64_t)unit * F::kSgBytes + lane * 16;
             uint8_t* dst = ring + stage * F::kSgBytes;
 #pragma unroll
             for (int m = 0; m < V; ++m) cp_async16(dst + m * 512, src + m * 512);
+            ++pj;
+            while (pj >= pend && ++pq < PS) prange(pq, warp, pj, pend);
         }
         cp_async_commit();
     };
     const int pre = D < kPreWait ? D : kPreWait;
-    for (int j = 0; j < pre; ++j) issue(j, j);
+    for (int j = 0; j < pre; ++j) issue(j);
 
     // ---- bookkeeping: warp ranges, contributors and arrival counters per
     // tile, zeroed sparse sums, zero x past K
@@ -663,11 +701,19 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_fused_kernel(const 
         }
     }
     const int B = p.batch;
-    const int pad = P.x_cols - p.k_in;
-    for (int i = tid; i < B * pad; i += kThreads) {
-        const int b = i / pad;
-        xs[b * P.x_stride + p.k_in + (i - b * pad)] = 0;
-    }
+    // columns of x chunk q (the last one may be short; its buffer is zero past K)
+    auto chunk_len = [&](int q) { return min(CS * kSgCols, p.k_in - q * CS * kSgCols); };
+    auto zero_pad = [&](int q) {
+        uint16_t* xb = xs + (q & 1) * xbuf_h;
+        const int len = chunk_len(q), pad = P.x_cols - len;
+        for (int i = tid; i < B * pad; i += kThreads) {
+            const int b = i / pad;
+            xb[b * P.x_stride + len + (i - b * pad)] = 0;
+        }
+    };
+    if (PS <= 2) zero_pad(PS - 1);
+    if (PS > 1)
+        for (int i = tid; i < ctiles * TE; i += kThreads) reinterpret_cast<float*>(smem + P.off_acc)[i] = 0.f;
     __syncthreads();
 
     // ---- the CTA's CSR entries [q0, q1), a fixed share e_per per thread
@@ -709,20 +755,27 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_fused_kernel(const 
 
     // ---- x may be written by the previous kernel of the stream: wait for it
     pdl_wait_previous();
-    if (tid == 0) {
+    // x chunk q into buffer q % 2: bulk copies issued by thread 0 (x rows
+    // 16-byte aligned), or copied by all threads (then a barrier follows)
+    auto load_chunk = [&](int q) {
+        uint64_t* bar = (q & 1) ? xbar1 : xbar;
+        uint16_t* xb = xs + (q & 1) * xbuf_h;
+        const int k0 = q * CS * kSgCols, len = chunk_len(q);
         if (p.x_bulk) {
-            mbar_expect_tx(xbar, (uint32_t)B * p.k_in * 2);
-            for (int b = 0; b < B; ++b) bulk_g2s(xs + b * P.x_stride, p.x + b * p.ldx, p.k_in * 2, xbar);
+            if (tid == 0) {
+                mbar_expect_tx(bar, (uint32_t)B * len * 2);
+                for (int b = 0; b < B; ++b) bulk_g2s(xb + b * P.x_stride, p.x + b * p.ldx + k0, len * 2, bar);
+            }
         } else {
-            mbar_expect_tx(xbar, 0);
+            if (tid == 0) mbar_expect_tx(bar, 0);
+            for (int i = tid; i < B * len; i += kThreads) {
+                const int b = i / len, k = i - b * len;
+                xb[b * P.x_stride + k] = p.x[b * p.ldx + k0 + k];
+            }
         }
-    }
-    if (!p.x_bulk) {
-        for (int i = tid; i < B * p.k_in; i += kThreads) {
-            const int b = i / p.k_in, k = i - b * p.k_in;
-            xs[b * P.x_stride + k] = p.x[b * p.ldx + k];
-        }
-    }
+    };
+    load_chunk(0);
+    if (PS > 1) load_chunk(1);
     // Each thread waits for the copies itself (an mbarrier wait makes the
     // bulk-copied bytes visible to it); only x copied by the threads needs a
     // barrier.
@@ -730,7 +783,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_fused_kernel(const 
     if (!(got_l && got_x && got_c && got_early)) atomicOr(p.status, kStatusWaitTimeout);
     if (!p.x_bulk) __syncthreads();
     // ---- the rest of the first D units (after x, which they would delay)
-    for (int j = pre; j < D; ++j) issue(j, j);
+    for (int j = pre; j < D; ++j) issue(j);
 
     // ---- sparse part: a fixed share of nonzeros per thread (balanced).
     // Each thread sums its entries per row: the first and last rows it
@@ -781,14 +834,16 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_fused_kernel(const 
                 const float v = h2f((uint16_t)vh[j]);
 #pragma unroll
                 for (int b = 0; b < CM; ++b)
-                    if (SB || b < B) acc[b] = fmaf(v, h2f(xs[b * P.x_stride + cc[j]]), acc[b]);
+                    if (SB || b < B) {
+                        // x of column cc[j]: staged in shared memory, or (x in K chunks) from L2
+                        const uint16_t xv = PS == 1 ? xs[b * P.x_stride + cc[j]] : __ldg(p.x + b * p.ldx + cc[j]);
+                        acc[b] = fmaf(v, h2f(xv), acc[b]);
+                    }
             }
         }
         emit(true);
     }
     if (has_csr && tid < CT) mbar_arrive(rbar);
-
-    if (nwu == 0) return;
 
     // The sparse sum of row ra+i, batch column col: the interior sum, then
     // the pieces of the threads whose shares cut the row, in thread order.
@@ -925,11 +980,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_fused_kernel(const 
     };
 
     // Decode and multiply-accumulate one unit (16 rows x 256 columns).
-    auto process = [&](const uint4 (&v)[V], int sgi) {
-        // x fragment source: batch rows >= B read row 0 (those MMA columns
-        // are never written out), so every lane loads unconditionally
-        const uint16_t* xb0 = xs + xrow * P.x_stride + sgi * kSgCols + 4 * t4;
-        const uint16_t* xb1 = xs + xrow2 * P.x_stride + sgi * kSgCols + 4 * t4;
+    auto process = [&](const uint4 (&v)[V], int sgi, const uint16_t* xbuf) {
+        // x fragment source (super-group sgi of the x buffer): batch rows >= B
+        // read row 0 (those MMA columns are never written out), so every lane
+        // loads unconditionally
+        const uint16_t* xb0 = xbuf + xrow * P.x_stride + sgi * kSgCols + 4 * t4;
+        const uint16_t* xb1 = xbuf + xrow2 * P.x_stride + sgi * kSgCols + 4 * t4;
         auto mac = [&](int st, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3) {
             const uint2 xv = *reinterpret_cast<const uint2*>(xb0 + st * 16);
             const bool on_tc = MAC == kMacTensor || (MAC == kMacMixed && (st & 1) == 0);
@@ -981,6 +1037,104 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_fused_kernel(const 
         }
     };
 
+
+    // ---- several passes over K (x staged chunk by chunk): per pass, each
+    // warp decodes its share of the pass's units; a tile's part that a warp
+    // holds whole is added to the tile's sum at once, shared parts go to the
+    // warps' slots and are added in warp order after a CTA barrier (the same
+    // order every call); the next chunk of x then loads into the buffer the
+    // pass used.  After the last pass the tile sums get their sparse sums and
+    // are written out.
+    if (!SB && PS > 1) {  // (batch 1 always takes one pass)
+        float* s_acc = reinterpret_cast<float*>(smem + P.off_acc);
+        int s_read = 0, s_fill = D;
+        for (int q = 0; q < PS; ++q) {
+            const int cs = pass_cs(q);
+            int a, b;
+            prange(q, warp, a, b);
+            const uint16_t* xq = xs + (q & 1) * xbuf_h;
+            if (!mbar_wait((q & 1) ? xbar1 : xbar, (uint32_t)((q >> 1) & 1))) atomicOr(p.status, kStatusWaitTimeout);
+            int cur = -1;  // CTA-local tile of the accumulators
+            auto flush_pass = [&]() {
+                float rr[NT][4];
+#pragma unroll
+                for (int n = 0; n < NT; ++n)
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) rr[n][r] = d0[n][r] + d1[n][r];
+                const int lo = cur * cs, hi = lo + cs;
+                const bool whole = a <= lo && b >= hi;
+                float* dst = whole ? s_acc + cur * TE : s_slots + (warp * 2 + (cur == a / cs ? 0 : 1)) * TE;
+#pragma unroll
+                for (int n = 0; n < NT; ++n) {
+                    const int col = 8 * n + 2 * t4;
+                    if (whole) {
+                        dst[g * CM + col] += rr[n][0];
+                        dst[g * CM + col + 1] += rr[n][1];
+                        dst[(g + 8) * CM + col] += rr[n][2];
+                        dst[(g + 8) * CM + col + 1] += rr[n][3];
+                    } else {
+                        dst[g * CM + col] = rr[n][0];
+                        dst[g * CM + col + 1] = rr[n][1];
+                        dst[(g + 8) * CM + col] = rr[n][2];
+                        dst[(g + 8) * CM + col + 1] = rr[n][3];
+                    }
+                }
+            };
+#pragma unroll 1
+            for (int j = a; j < b; ++j) {
+                cp_async_wait_newest(D - 1);
+                uint4 v[V];
+                const uint8_t* src = ring + s_read * F::kSgBytes;
+#pragma unroll
+                for (int m = 0; m < V; ++m) v[m] = *reinterpret_cast<const uint4*>(src + m * 512);
+                issue(s_fill);
+                s_read = s_read + 1 == S ? 0 : s_read + 1;
+                s_fill = s_fill + 1 == S ? 0 : s_fill + 1;
+                const int tl = j / cs;
+                if (tl != cur) {
+                    if (cur >= 0) flush_pass();
+                    cur = tl;
+                    tile = t_first + tl;
+                    start_tile();
+                }
+                process(v, j - tl * cs, xq);
+            }
+            if (cur >= 0) flush_pass();
+            __syncthreads();
+            // shared tiles of this pass: the parts, in warp order
+            for (int idx = tid; idx < ctiles * TE; idx += kThreads) {
+                const int tl = idx / TE, e = idx - tl * TE;
+                const int lo = tl * cs, hi = lo + cs;
+                int parts = 0;
+                float sum = 0.f;
+                for (int w = 0; w < kWarps; ++w) {
+                    int aw, bw;
+                    prange(q, w, aw, bw);
+                    if (max(aw, lo) < min(bw, hi)) {
+                        ++parts;
+                        sum += s_slots[(w * 2 + (tl == aw / cs ? 0 : 1)) * TE + e];
+                    }
+                }
+                if (parts > 1) s_acc[idx] += sum;
+            }
+            // chunk q+2 into the buffer this pass used
+            if (q + 2 < PS) {
+                if (q + 2 == PS - 1) zero_pad(q + 2);
+                if (tid == 0) fence_proxy_async();
+                load_chunk(q + 2);
+            }
+            __syncthreads();
+        }
+        for (int idx = tid; idx < ctiles * TE; idx += kThreads) {
+            const int tl = idx / TE, e = idx - tl * TE;
+            const int row_l = e / CM, col = e - row_l * CM;
+            out((t_first + tl) * kTileRows + row_l, col, s_acc[idx]);
+        }
+        return;
+    }
+
+    if (nwu == 0) return;
+
     start_tile();
     // Units in order: wait for unit i's group, read its stage, refill the
     // stage freed by unit i-1 with unit i+D, decode.
@@ -992,10 +1146,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_fused_kernel(const 
         const uint8_t* src = ring + s_read * F::kSgBytes;
 #pragma unroll
         for (int m = 0; m < V; ++m) v[m] = *reinterpret_cast<const uint4*>(src + m * 512);
-        issue(i + D, s_fill);
+        issue(s_fill);
         s_read = s_read + 1 == S ? 0 : s_read + 1;
         s_fill = s_fill + 1 == S ? 0 : s_fill + 1;
-        process(v, sg);
+        process(v, sg, xs);
         if (++sg == nsg || i + 1 == nwu) {
             flush_tile();
             if (i + 1 < nwu) {

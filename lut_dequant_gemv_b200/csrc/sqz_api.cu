@@ -210,7 +210,8 @@ sqz_status prepare_fused_kernels(int optin) {
 // Plan for a call, or false when the fused kernel cannot stage x.  A call
 // first gets an SM's share (two CTAs per SM, so the next call's CTA can
 // stream its weights while this one computes); one whose x does not fit
-// there gets a whole SM.
+// there gets a whole SM; a batch whose x does not fit at all is staged in K
+// chunks (several passes, fewest first).
 bool fused_plan(const sqz_layer* L, int batch, sqz::tc::Plan* out) {
     const int nt = batch > 8 ? 2 : 1;
     for (int budget : {L->smem_budget, L->smem_optin}) {
@@ -219,6 +220,25 @@ bool fused_plan(const sqz_layer* L, int batch, sqz::tc::Plan* out) {
             *out = P;
             return true;
         }
+    }
+    if (batch > 1) {
+        // fewest passes that still leave a ring of 4 stages per warp, else the
+        // fewest passes that fit at all
+        bool have = false;
+        for (int passes = 2; passes <= L->nsg; ++passes) {
+            sqz::tc::Plan P =
+                sqz::tc::make_plan(L->bits, L->n_out, L->k_in, batch, nt, false, L->sm_count, L->smem_optin, passes);
+            if (P.passes != passes || P.total > L->smem_optin || P.grid != L->grid) continue;
+            if (!have) {
+                *out = P;
+                have = true;
+            }
+            if (P.stages >= 4) {
+                *out = P;
+                return true;
+            }
+        }
+        return have;
     }
     return false;
 }

@@ -325,6 +325,26 @@ def test_padded_columns_with_nonfinite_lut_entries(B, orc, bits, k_in, mac):
     assert np.array_equal(w.cpu().numpy().view(np.uint16), orc.dequant(Lx.codes, Lx.lut, n_out, k_in, bits))
 
 
+@pytest.mark.parametrize("n_out,k_in,bits,batch,ldx_pad", [
+    (200, 8288, 3, 16, 0),   # x staged in K chunks; the last chunk is short
+    (150, 12000, 4, 12, 0),
+    (96, 9216, 3, 9, 1),     # x rows not 16-byte aligned: copied by the threads
+    (300, 6144, 4, 16, 0),
+])
+def test_batches_whose_x_is_staged_in_chunks(B, orc, n_out, k_in, bits, batch, ldx_pad):
+    """Batches whose activations do not fit in shared memory at once: x is
+    staged chunk by chunk over several passes and per-tile sums are kept
+    between them.  Same tolerance, and bit-identical from run to run."""
+    L = make_small(90 + k_in, n_out, k_in, bits, n_out * 12)
+    x = synth.make_x(batch, k_in, seed=batch)
+    layer = upload(B, L)
+    y = gpu_gemv(B, layer, x, ldx=k_in + ldx_pad)
+    y_ref, bound = orc.gemv_layer(L, x)
+    assert_close(y, y_ref, bound, f"{n_out}x{k_in} b{bits} B{batch}")
+    assert np.array_equal(y, gpu_gemv(B, layer, x, ldx=k_in + ldx_pad))
+    assert B.sqz_layer_status(layer) == 0
+
+
 def test_chained_calls_read_the_previous_output(B, orc):
     """Back-to-back calls on one stream where each call's x is the previous
     call's y: a launch may start before the previous kernel ends, and must
