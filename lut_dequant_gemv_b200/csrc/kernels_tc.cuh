@@ -77,7 +77,7 @@ constexpr int kThreads = kWarps * 32;
 constexpr int kCtasPerSm = 2;
 constexpr int kCsrThreads = 256;  // threads sharing the sparse part (warps 0-7; the same split for every batch)
 constexpr int kCsrWarps = kCsrThreads / 32;
-static_assert(kCsrWarps <= kWarps, "the sparse part runs on the CTA's first warps");
+static_assert(kCsrWarps <= kWarps && kWarps <= 16, "the sparse part runs on the CTA's first warps; warp masks are 16 bits");
 // Dense units that each sparse warp hands to a non-sparse warp when the
 // layer has outliers: the sparse share delays a warp's dense start by about
 // one unit's decode time.
@@ -88,6 +88,7 @@ constexpr int kSgCols = 256;      // columns per super-group
 constexpr int kMaxCtas = 512;     // CTAs per launch (one per SM)
 constexpr int kMinStages = 2;     // shared-memory stages per warp (units in flight + 1)
 constexpr int kMaxStages = 16;
+constexpr int kRingStages = 4;    // ring depth reserved before the CSR staging area
 constexpr int kPreWait = 2;       // code units per warp requested before waiting for the previous kernel;
                                   // the rest of the first ring follows once x has landed
 constexpr int kCsrCap = 4096;     // CSR entries per CTA staged in shared memory, at most (more: read from global)
@@ -216,7 +217,9 @@ __host__ __device__ inline Plan make_plan(int bits, int n_out, int k_in, int bat
     P.off_acc = off;  // per-tile sums across passes
     if (P.passes > 1) off += round_up(rows * P.cm * 4, 128);
     const int sg_bytes = bits == 3 ? 1536 : 2048;
-    const int ring_min = kMinStages * kWarps * sg_bytes;
+    // the CSR staging area takes what is left after a ring of kRingStages
+    // (up to kCsrCap entries; entries beyond it are read from global memory)
+    const int ring_min = kRingStages * kWarps * sg_bytes;
     int cap = (budget - off - ring_min - 512) / 6;  // 4-byte column + 2-byte value per entry
     cap = cap > kCsrCap ? kCsrCap : cap;
     P.csr_cap = cap < 0 ? 0 : cap & ~7;
@@ -1100,22 +1103,30 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_fused_kernel(const 
                 process(v, j - tl * cs, xq);
             }
             if (cur >= 0) flush_pass();
+            // per tile of this pass: the warps holding parts (bits 0-15) and
+            // which of them used their second slot (bits 16-31)
+            for (int tl = tid; tl < ctiles; tl += kThreads) {
+                const int lo = tl * cs, hi = lo + cs;
+                int info = 0;
+                for (int w = 0; w < kWarps; ++w) {
+                    int aw, bw;
+                    prange(q, w, aw, bw);
+                    if (max(aw, lo) < min(bw, hi)) info |= (1 << w) | ((tl == aw / cs ? 0 : 1) << (16 + w));
+                }
+                s_tinfo[tl] = info;
+            }
             __syncthreads();
             // shared tiles of this pass: the parts, in warp order
             for (int idx = tid; idx < ctiles * TE; idx += kThreads) {
                 const int tl = idx / TE, e = idx - tl * TE;
-                const int lo = tl * cs, hi = lo + cs;
-                int parts = 0;
+                const int info = s_tinfo[tl], mask = info & 0xffff;
+                if ((mask & (mask - 1)) == 0) continue;  // one part: already added
                 float sum = 0.f;
-                for (int w = 0; w < kWarps; ++w) {
-                    int aw, bw;
-                    prange(q, w, aw, bw);
-                    if (max(aw, lo) < min(bw, hi)) {
-                        ++parts;
-                        sum += s_slots[(w * 2 + (tl == aw / cs ? 0 : 1)) * TE + e];
-                    }
+                for (int mm = mask; mm; mm &= mm - 1) {
+                    const int w = __ffs(mm) - 1;
+                    sum += s_slots[(w * 2 + ((info >> (16 + w)) & 1)) * TE + e];
                 }
-                if (parts > 1) s_acc[idx] += sum;
+                s_acc[idx] += sum;
             }
             // chunk q+2 into the buffer this pass used
             if (q + 2 < PS) {
