@@ -55,6 +55,9 @@ def parse():
     p.add_argument("--sweep", action="store_true", help="one JSON line per workload shape")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--seed", type=int, default=0)
+    p.add_argument("--profile-launches", type=int, default=0,
+                   help="for profiler captures: one layer instance of the shape, this many plain launches, "
+                        "no timing and no JSON line")
     return p.parse_args()
 
 
@@ -89,7 +92,7 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload: str, shape_key: str):
+def recorded_traffic(workload: str, shape_key: str, batch: int = 1):
     """DRAM bytes per launch from the committed ncu summary, valid only while
     the kernel sources are unchanged since the capture."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
@@ -102,7 +105,8 @@ def recorded_traffic(workload: str, shape_key: str):
             if not line:
                 continue
             kv = dict(tok.split("=", 1) for tok in line.split())
-            if kv.get("shape") == shape_key and kv.get("source_hash") == want:
+            if (kv.get("shape") == shape_key and kv.get("batch", "1") == str(batch)
+                    and kv.get("source_hash") == want):
                 return int(kv["bytes_per_launch"])
     return None
 
@@ -371,7 +375,7 @@ def run_ours(args):
         yard = {"error": str(e)}
 
     peak, peak_kind = measured_peaks()
-    traffic = recorded_traffic(args.workload, shape.key)
+    traffic = recorded_traffic(args.workload, shape.key, shape.batch)
     line = {
         "metric": METRIC if args.workload == DEFAULT_WORKLOAD else f"dense+sparse GEMV achieved HBM GB/s ({args.workload})",
         "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -447,8 +451,31 @@ def run_sweep(args):
     return 0
 
 
+def run_profile_launches(args):
+    """One layer instance, N back-to-back launches on the default stream (a
+    short, bounded program for an ncu capture of one launch per shape)."""
+    import torch
+
+    from lut_dequant_gemv_b200 import binding as B
+
+    B.lib()
+    shape = shape_for(args)
+    L = synth.layer_for(shape, seed=args.seed)
+    layer = B.create_layer_from_numpy(L.n_out, L.k_in, L.bits, L.codes, L.lut, L.rowptr, L.col, L.val)
+    x = torch.from_numpy(synth.x_for(shape, seed=args.seed).view(np.int16)).cuda()
+    y = torch.empty((shape.batch, shape.n_out), dtype=torch.int16, device="cuda")
+    for _ in range(args.profile_launches):
+        B.sqz_gemv(layer, x, y)
+    torch.cuda.synchronize()
+    print(f"{shape.key} B{shape.batch}: {args.profile_launches} launches", flush=True)
+    layer.close()
+    return 0
+
+
 def main():
     args = parse()
+    if args.profile_launches:
+        return run_profile_launches(args)
     if args.impl == "reference":
         return run_reference(args)
     if args.sweep:
