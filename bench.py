@@ -55,6 +55,8 @@ def parse():
     p.add_argument("--sweep", action="store_true", help="one JSON line per workload shape")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--seed", type=int, default=0)
+    p.add_argument("--csr", choices=("balanced", "rowwise"), default="balanced",
+                   help="sparse scheme of the fused kernel (rowwise: the plain CSR comparison)")
     p.add_argument("--profile-launches", type=int, default=0,
                    help="for profiler captures: one layer instance of the shape, this many plain launches, "
                         "no timing and no JSON line")
@@ -183,7 +185,7 @@ def config_for(args, shape, instances, inst_bytes):
         "workload": f"{args.workload}: " + WORKLOAD_DESC.get(
             args.workload, f"{shape.n_out}x{shape.k_in}, {shape.bits}-bit, {shape.density:.2%} CSR, batch {shape.batch}"),
         "n_out": shape.n_out, "k_in": shape.k_in, "bits": shape.bits, "density": shape.density,
-        "batch": shape.batch, "outliers": shape.dist,
+        "batch": shape.batch, "outliers": shape.dist, "csr_scheme": args.csr,
         "l2": f"inputs larger than L2: {instances} rotating layer instances, {instances * inst_bytes / 1e6:.0f} MB",
         "parallelism": "replicas (independent layers per GPU)",
     }
@@ -281,6 +283,8 @@ def run_ours(args):
         L = L0 if i == 0 else synth.layer_for(shape, seed=args.seed, instance=rank * 1000 + i)
         layers.append(B.create_layer_from_numpy(L.n_out, L.k_in, L.bits, L.codes, L.lut, L.rowptr, L.col, L.val,
                                                 device=dev))
+        if args.csr == "rowwise":
+            B.sqz_layer_set_csr_mode(layers[-1], B.SQZ_CSR_ROWWISE)
         xs.append(torch.from_numpy(synth.x_for(shape, seed=args.seed, instance=rank * 1000 + i).view(np.int16)).to(dev))
         ys.append(torch.empty((shape.batch, shape.n_out), dtype=torch.int16, device=dev))
     nnz = L0.nnz

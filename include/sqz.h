@@ -160,6 +160,24 @@ SQZ_API sqz_status sqz_debug_dequant(sqz_layer_t layer, uint16_t* w_out, void* s
  */
 SQZ_API sqz_status sqz_layer_set_mac(sqz_layer_t layer, int32_t mac);
 
+/* How the fused kernel sums the outliers (sqz_layer_set_csr_mode). */
+#define SQZ_CSR_BALANCED 0 /* equal nonzero shares per thread, pieces combined per row (default) */
+#define SQZ_CSR_ROWWISE 1  /* each row's nonzeros summed by one thread: the plain CSR SpMV     */
+
+/*
+ * Choose the sparse scheme ("SqueezeLLM: Dense-and-Sparse Quantization",
+ * summary page, §3.4 "Balanced Sparse Kernel": the balanced split against
+ * the plain row-per-thread CSR kernel it replaces).  Both give results
+ * within the same bound (only the order of the additions differs); the
+ * row-wise scheme exists to compare the two on skewed outlier
+ * distributions, where its cost follows the longest row of a tile.  In
+ * row-wise mode the dense part always uses the tensor cores (the
+ * sqz_layer_set_mac choice applies to the balanced mode).  Not
+ * thread-safe against concurrent sqz_gemv calls on the same handle.
+ * Errors: SQZ_ERR_INVALID_ARG.
+ */
+SQZ_API sqz_status sqz_layer_set_csr_mode(sqz_layer_t layer, int32_t mode);
+
 /*
  * Read and clear the handle's device status word, ordered on `stream`
  * (synchronises it).  0 means every call so far completed normally; bit 0

@@ -28,6 +28,8 @@ SQZ_MAX_BATCH = 16
 SQZ_MAC_TENSOR_CORES = 0
 SQZ_MAC_CUDA_CORES = 1
 SQZ_MAC_MIXED = 2
+SQZ_CSR_BALANCED = 0
+SQZ_CSR_ROWWISE = 1
 
 STATUS_NAMES = {0: "SQZ_OK", 1: "SQZ_ERR_INVALID_ARG", 2: "SQZ_ERR_UNSUPPORTED", 3: "SQZ_ERR_CUDA",
                 4: "SQZ_ERR_OOM", 5: "SQZ_ERR_TIMEOUT"}
@@ -35,7 +37,7 @@ STATUS_NAMES = {0: "SQZ_OK", 1: "SQZ_ERR_INVALID_ARG", 2: "SQZ_ERR_UNSUPPORTED",
 # Every entry point include/sqz.h declares.
 EXPORTED = ("sqz_create_layer", "sqz_gemv", "sqz_gemv_host", "sqz_debug_dequant", "sqz_layer_info",
             "sqz_destroy", "sqz_fp16_gemv", "sqz_last_error", "sqz_version", "sqz_check_csr_static",
-            "sqz_layer_set_mac", "sqz_layer_status")
+            "sqz_layer_set_mac", "sqz_layer_set_csr_mode", "sqz_layer_status")
 
 
 class SqzError(RuntimeError):
@@ -82,6 +84,8 @@ def lib() -> ctypes.CDLL:
             getattr(L, name).restype = ctypes.c_int
         L.sqz_layer_set_mac.argtypes = [P, i32]
         L.sqz_layer_set_mac.restype = ctypes.c_int
+        L.sqz_layer_set_csr_mode.argtypes = [P, i32]
+        L.sqz_layer_set_csr_mode.restype = ctypes.c_int
         L.sqz_layer_status.argtypes = [P, P, ctypes.POINTER(i32)]
         L.sqz_layer_status.restype = ctypes.c_int
         L.sqz_check_csr_static.argtypes = [P, P, i32, i32, i64, P, ctypes.POINTER(i32)]
@@ -289,6 +293,10 @@ def sqz_check_csr_static(rowptr: Optional[torch.Tensor], col: Optional[torch.Ten
 
 def sqz_layer_set_mac(layer: Layer, mac: int) -> None:
     _check(lib().sqz_layer_set_mac(layer, int(mac)), "sqz_layer_set_mac")
+
+
+def sqz_layer_set_csr_mode(layer: Layer, mode: int) -> None:
+    _check(lib().sqz_layer_set_csr_mode(layer, int(mode)), "sqz_layer_set_csr_mode")
 
 
 def sqz_layer_status(layer: Layer, stream=None) -> int:

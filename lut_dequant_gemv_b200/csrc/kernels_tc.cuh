@@ -244,7 +244,6 @@ struct Params {
     int n_out, k_in, nsg, ntiles, batch;
     int has_csr;             // the layer has outliers
     int x_bulk;              // 1: every x row is 16-byte aligned -> bulk copies
-    int pad_;
     Plan plan;
     const uint8_t* lutp;     // [ntiles*16][lut_bytes], byte planes
     const int32_t* rowptr;   // canonical CSR (device copies owned by the layer)
@@ -560,7 +559,7 @@ __global__ void dequant_native_kernel(const uint8_t* __restrict__ codes, const u
 // ------------------------------------------------------------ main kernel
 // MAC: kMacTensor / kMacCuda / kMacMixed.  SB: batch 1 (one column carried
 // through the sparse part and the combine).
-template <int BITS, int NT, int MAC, bool SB>
+template <int BITS, int NT, int MAC, bool SB, bool RW>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_fused_kernel(const __grid_constant__ Params p) {
     using F = Fmt<BITS>;
     using TAB = typename std::conditional<BITS == 3, Tab3, Tab4>::type;
@@ -726,7 +725,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_fused_kernel(const 
     const bool csr_in_smem = has_csr && nz <= P.csr_cap;
     const int e_per = has_csr ? (int)(((int64_t)nz + CT - 1) / CT) : 1;
     const int ca = tid < CT ? (int)min((int64_t)q1, (int64_t)q0 + (int64_t)tid * e_per) : q1;
-    const int cb = (int)min((int64_t)q1, (int64_t)ca + e_per);
+    const int cb = RW ? ca : (int)min((int64_t)q1, (int64_t)ca + e_per);  // row-wise: no shares
     const int* csr_col = csr_in_smem ? reinterpret_cast<const int*>(smem + P.off_col) + (q0 & 3) - q0 : p.col;
     const uint16_t* csr_val =
         csr_in_smem ? reinterpret_cast<const uint16_t*>(smem + P.off_val) + (q0 & 7) - q0 : p.val;
@@ -845,6 +844,28 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_fused_kernel(const 
             }
         }
         emit(true);
+    }
+    // Row-wise mode (the plain CSR scheme, for comparison): no shares; thread
+    // t sums the whole rows t, t + CT, ... of the CTA into s_rowsum, so the
+    // tile finishers wait for the thread holding the longest row.
+    if (RW && has_csr && tid < CT) {
+        for (int i = tid; i < nrows; i += CT) {
+            float acc[CM];
+#pragma unroll
+            for (int b = 0; b < CM; ++b) acc[b] = 0.f;
+            for (int j = s_rp[i], je = s_rp[i + 1]; j < je; ++j) {
+                const float v = h2f(csr_val[j]);
+                const int cj = csr_col[j];
+#pragma unroll
+                for (int b = 0; b < CM; ++b)
+                    if (SB || b < B) {
+                        const uint16_t xv = PS == 1 ? xs[b * P.x_stride + cj] : __ldg(p.x + b * p.ldx + cj);
+                        acc[b] = fmaf(v, h2f(xv), acc[b]);
+                    }
+            }
+#pragma unroll
+            for (int b = 0; b < CM; ++b) s_rowsum[i * CM + b] = acc[b];
+        }
     }
     if (has_csr && tid < CT) mbar_arrive(rbar);
 

@@ -74,6 +74,7 @@ struct sqz_layer {
     int smem_optin = 232448;
     int smem_budget = 232448;  // shared memory of one fused CTA (kCtasPerSm of them share an SM)
     int mac = SQZ_MAC_TENSOR_CORES;
+    int csr_mode = SQZ_CSR_BALANCED;
     // The fused kernel serves every layer with N > 0 and K > 0 (columns past
     // K are padded inside the kernel-native layout).
     bool fused_ok = false;
@@ -182,9 +183,9 @@ void dispatch_rowwarp(const sqz_layer* L, const uint16_t* x, int32_t batch, int6
 }
 
 // ------------------------------------------------------------ fused kernel
-template <int BITS, int NT, int MAC, bool SB>
+template <int BITS, int NT, int MAC, bool SB, bool RW = false>
 sqz_status set_smem_attr(int bytes) {
-    SQZ_CUDA_TRY(cudaFuncSetAttribute(sqz::tc::gemv_fused_kernel<BITS, NT, MAC, SB>,
+    SQZ_CUDA_TRY(cudaFuncSetAttribute(sqz::tc::gemv_fused_kernel<BITS, NT, MAC, SB, RW>,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, bytes),
                  "cudaFuncSetAttribute");
     return SQZ_OK;
@@ -199,6 +200,9 @@ sqz_status prepare_fused_bits(int optin) {
     if ((st = set_smem_attr<BITS, 2, kMacTensor, false>(optin)) != SQZ_OK) return st;
     if ((st = set_smem_attr<BITS, 1, kMacCuda, true>(optin)) != SQZ_OK) return st;
     if ((st = set_smem_attr<BITS, 1, kMacMixed, true>(optin)) != SQZ_OK) return st;
+    if ((st = set_smem_attr<BITS, 1, kMacTensor, true, true>(optin)) != SQZ_OK) return st;
+    if ((st = set_smem_attr<BITS, 1, kMacTensor, false, true>(optin)) != SQZ_OK) return st;
+    if ((st = set_smem_attr<BITS, 2, kMacTensor, false, true>(optin)) != SQZ_OK) return st;
     return SQZ_OK;
 }
 
@@ -246,7 +250,7 @@ bool fused_plan(const sqz_layer* L, int batch, sqz::tc::Plan* out) {
 // Launch with programmatic stream serialization: the kernel may start while
 // the previous kernel of the stream is still running; it prefetches only
 // weights before it waits for that kernel (griddepcontrol.wait).
-template <int BITS, int NT, int MAC, bool SB>
+template <int BITS, int NT, int MAC, bool SB, bool RW = false>
 cudaError_t launch_fused(const sqz::tc::Params& prm, cudaStream_t s) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)prm.plan.grid);
@@ -258,14 +262,20 @@ cudaError_t launch_fused(const sqz::tc::Params& prm, cudaStream_t s) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, sqz::tc::gemv_fused_kernel<BITS, NT, MAC, SB>, prm);
+    return cudaLaunchKernelEx(&cfg, sqz::tc::gemv_fused_kernel<BITS, NT, MAC, SB, RW>, prm);
 }
 
 // Batch 1 takes the requested multiply-accumulate unit; larger batches the
-// tensor cores (one or two n-tiles of 8 batch columns).
+// tensor cores (one or two n-tiles of 8 batch columns).  The row-wise CSR
+// comparison mode always uses the tensor cores.
 template <int BITS>
-cudaError_t launch_fused_bits(const sqz::tc::Params& prm, int batch, int mac, cudaStream_t s) {
+cudaError_t launch_fused_bits(const sqz::tc::Params& prm, int batch, int mac, int csr_mode, cudaStream_t s) {
     using namespace sqz::tc;
+    if (csr_mode == SQZ_CSR_ROWWISE) {
+        if (batch > 8) return launch_fused<BITS, 2, kMacTensor, false, true>(prm, s);
+        if (batch > 1) return launch_fused<BITS, 1, kMacTensor, false, true>(prm, s);
+        return launch_fused<BITS, 1, kMacTensor, true, true>(prm, s);
+    }
     if (batch > 8) return launch_fused<BITS, 2, kMacTensor, false>(prm, s);
     if (batch > 1) return launch_fused<BITS, 1, kMacTensor, false>(prm, s);
     if (mac == SQZ_MAC_CUDA_CORES) return launch_fused<BITS, 1, kMacCuda, true>(prm, s);
@@ -310,8 +320,8 @@ sqz_status gemv_impl(const sqz_layer* L, const uint16_t* x, int32_t batch, int64
             prm.x_bulk = (reinterpret_cast<uintptr_t>(xc) % 16 == 0) && (ldx % 8 == 0) && (L->k_in % 8 == 0);
             prm.plan = P;
             std::memcpy(prm.csr_cta, L->csr_cta.data(), sizeof(int32_t) * L->csr_cta.size());
-            const cudaError_t e = L->bits == 3 ? launch_fused_bits<3>(prm, nb, L->mac, s)
-                                               : launch_fused_bits<4>(prm, nb, L->mac, s);
+            const cudaError_t e = L->bits == 3 ? launch_fused_bits<3>(prm, nb, L->mac, L->csr_mode, s)
+                                               : launch_fused_bits<4>(prm, nb, L->mac, L->csr_mode, s);
             SQZ_CUDA_TRY(e, "fused gemv launch");
         }
     } else if (L->bits == 3) {
@@ -552,6 +562,13 @@ sqz_status sqz_layer_set_mac(sqz_layer_t layer, int32_t mac) {
     if (mac != SQZ_MAC_TENSOR_CORES && mac != SQZ_MAC_CUDA_CORES && mac != SQZ_MAC_MIXED)
         return fail(SQZ_ERR_INVALID_ARG, "unknown MAC unit %d", mac);
     layer->mac = mac;
+    return SQZ_OK;
+}
+
+sqz_status sqz_layer_set_csr_mode(sqz_layer_t layer, int32_t mode) {
+    if (!layer) return fail(SQZ_ERR_INVALID_ARG, "layer is NULL");
+    if (mode != SQZ_CSR_BALANCED && mode != SQZ_CSR_ROWWISE) return fail(SQZ_ERR_INVALID_ARG, "unknown CSR mode %d", mode);
+    layer->csr_mode = mode;
     return SQZ_OK;
 }
 

@@ -20,7 +20,13 @@ tensor is drawn from the distributions below.
 * Outliers: round(p*N*K) distinct positions drawn uniformly without
   replacement, stored in CSR order (row-major, ascending column); values
   are +-U(0.1, 0.5) (fair sign) or 0.1*t(df=3) clamped to the fp16 range,
-  rounded to fp16.
+  rounded to fp16.  The "skew" distribution draws the same number of
+  outliers with +-U(0.1, 0.5) values but concentrates them on few rows: row
+  counts are multinomial with Zipf weights 1/r over a random order of the
+  rows (capped at K, so the heaviest rows are entirely outliers), columns
+  uniform without replacement within a row -- a stress case for the
+  balanced sparse scheme (the pages state that outliers are unevenly
+  spread over rows).
 * Activations: x ~ N(0, 1) rounded to fp16.
 
 Every tensor comes from its own PCG64 stream keyed by (seed, workload id,
@@ -36,7 +42,7 @@ import numpy as np
 
 FP16_MAX = 65504.0
 
-_TENSOR_IDS = {"lut": 1, "codes": 2, "pos": 3, "sign": 4, "mag": 5, "x": 6}
+_TENSOR_IDS = {"lut": 1, "codes": 2, "pos": 3, "sign": 4, "mag": 5, "x": 6, "rows": 7}
 
 
 def _rng(seed: int, key: str, instance: int, tensor: str) -> np.random.Generator:
@@ -99,7 +105,18 @@ def draw_codes(rng: np.random.Generator, n_out: int, k_in: int, bits: int) -> np
 def draw_outliers(seed: int, key: str, instance: int, n_out: int, k_in: int, density: float,
                   dist: str = "uniform") -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
     nnz = nnz_for(n_out, k_in, density)
-    if nnz:
+    if nnz and dist == "skew":
+        rr = _rng(seed, key, instance, "rows")
+        order = rr.permutation(n_out)
+        w = 1.0 / np.arange(1, n_out + 1)
+        counts = np.zeros(n_out, dtype=np.int64)
+        counts[order] = rr.multinomial(nnz, w / w.sum())
+        counts = np.minimum(counts, k_in)
+        pr = _rng(seed, key, instance, "pos")
+        parts = [i * k_in + np.sort(pr.choice(k_in, size=int(c), replace=False)) for i, c in enumerate(counts) if c]
+        pos = np.concatenate(parts).astype(np.int64) if parts else np.zeros(0, dtype=np.int64)
+        nnz = int(pos.shape[0])
+    elif nnz:
         pos = _rng(seed, key, instance, "pos").choice(n_out * k_in, size=nnz, replace=False)
         pos = np.sort(pos.astype(np.int64))
     else:
@@ -108,7 +125,7 @@ def draw_outliers(seed: int, key: str, instance: int, n_out: int, k_in: int, den
     col = (pos % k_in).astype(np.int32)
     rowptr = np.zeros(n_out + 1, dtype=np.int64)
     np.cumsum(np.bincount(rows, minlength=n_out), out=rowptr[1:])
-    if dist == "uniform":
+    if dist in ("uniform", "skew"):
         sign = _rng(seed, key, instance, "sign").integers(0, 2, size=nnz) * 2 - 1
         mag = _rng(seed, key, instance, "mag").uniform(0.1, 0.5, size=nnz)
         v = sign * mag
@@ -155,7 +172,7 @@ class Shape:
 
 
 def workloads() -> Dict[str, List[Shape]]:
-    """The five synthetic workloads (LLaMA-7B/13B/65B linear-layer shapes)."""
+    """The synthetic workloads (LLaMA-7B/13B/65B linear-layer shapes)."""
     w: Dict[str, List[Shape]] = {}
     w["llama7b-q-4bit"] = [Shape("q_proj", 4096, 4096, 4, 0.0045)]
     w["llama7b-up-3bit"] = [Shape("up_proj", 11008, 4096, 3, 0.0045)]
@@ -170,6 +187,9 @@ def workloads() -> Dict[str, List[Shape]]:
     w["llama13b-batch"] = [Shape(nm, n, k, 3, 0.0045, b) for nm, n, k in
                            (("qkvo", 5120, 5120), ("gate_up", 13824, 5120), ("down", 5120, 13824))
                            for b in (1, 2, 4, 8, 16)]
+    # skewed outliers (same counts as the uniform 0.45 % layers, Zipf rows)
+    w["llama7b-skew"] = [Shape("up_proj", 11008, 4096, 3, 0.0045, 1, "skew"),
+                         Shape("q_proj", 4096, 4096, 4, 0.0045, 1, "skew")]
     return w
 
 

@@ -92,3 +92,9 @@ def test_destroy_accepts_null(lib):
 ])
 def test_fp16_gemv_rejects_bad_arguments(lib, args):
     assert lib.sqz_fp16_gemv(*args, None) == B.SQZ_ERR_INVALID_ARG
+
+
+def test_layer_options_reject_null_handles_and_unknown_values(lib):
+    assert lib.sqz_layer_set_mac(None, 0) == B.SQZ_ERR_INVALID_ARG
+    assert lib.sqz_layer_set_csr_mode(None, B.SQZ_CSR_ROWWISE) == B.SQZ_ERR_INVALID_ARG
+    assert "NULL" in B.sqz_last_error()

@@ -345,6 +345,28 @@ def test_batches_whose_x_is_staged_in_chunks(B, orc, n_out, k_in, bits, batch, l
     assert B.sqz_layer_status(layer) == 0
 
 
+@pytest.mark.parametrize("mode", ["balanced", "rowwise"])
+@pytest.mark.parametrize("wl,idx", [("llama7b-skew", 0), ("llama7b-skew", 1), ("llama7b-up-3bit", 0)])
+def test_csr_schemes_match_oracle(B, orc, wl, idx, mode):
+    """Both sparse schemes -- the balanced split and the plain row-per-thread
+    CSR it replaces -- on uniform and on heavily skewed outliers (Zipf rows,
+    the heaviest entirely outliers), batch 1 and batch 3."""
+    shape = synth.workloads()[wl][idx]
+    L = synth.layer_for(shape)
+    layer = upload(B, L)
+    if mode == "rowwise":
+        B.sqz_layer_set_csr_mode(layer, B.SQZ_CSR_ROWWISE)
+    for batch in (1, 3):
+        x = synth.make_x(batch, shape.k_in, seed=batch, key="csr-modes")
+        y = gpu_gemv(B, layer, x)
+        rows = _rows_for(synth.Shape(shape.name, shape.n_out, shape.k_in, shape.bits, shape.density, batch))
+        y_ref, bound = orc.gemv_layer(L, x, rows=rows)
+        assert_close(y if rows is None else y[:, rows], y_ref, bound, f"{shape.key} {mode} B{batch}")
+    assert B.sqz_layer_status(layer) == 0
+    with pytest.raises(B.SqzError):
+        B.sqz_layer_set_csr_mode(layer, 5)
+
+
 def test_chained_calls_read_the_previous_output(B, orc):
     """Back-to-back calls on one stream where each call's x is the previous
     call's y: a launch may start before the previous kernel ends, and must
