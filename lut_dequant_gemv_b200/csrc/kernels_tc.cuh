@@ -89,6 +89,8 @@ constexpr int kMaxCtas = 512;     // CTAs per launch (one per SM)
 constexpr int kMinStages = 2;     // shared-memory stages per warp (units in flight + 1)
 constexpr int kMaxStages = 16;
 constexpr int kRingStages = 4;    // ring depth reserved before the CSR staging area
+constexpr int kSbStages = 4;      // batch 1: the ring depth, 4 stages (3 when 4 do not fit), so
+                                  // that the wait for a unit's copies is one of two fixed forms
 constexpr int kPreWait = 2;       // code units per warp requested before waiting for the previous kernel;
                                   // the rest of the first ring follows once x has landed
 constexpr int kCsrCap = 4096;     // CSR entries per CTA staged in shared memory, at most (more: read from global)
@@ -219,7 +221,11 @@ __host__ __device__ inline Plan make_plan(int bits, int n_out, int k_in, int bat
     const int sg_bytes = bits == 3 ? 1536 : 2048;
     // the CSR staging area takes what is left after a ring of kRingStages
     // (up to kCsrCap entries; entries beyond it are read from global memory)
-    const int ring_min = kRingStages * kWarps * sg_bytes;
+    // batch 1: a ring of kSbStages stages when it fits beside at least a
+    // small CSR stage, else one stage less
+    int sb_stages = kSbStages;
+    if (single && budget - off - kSbStages * kWarps * sg_bytes - 512 < 6 * 256) sb_stages = kSbStages - 1;
+    const int ring_min = (single ? sb_stages : kRingStages) * kWarps * sg_bytes;
     int cap = (budget - off - ring_min - 512) / 6;  // 4-byte column + 2-byte value per entry
     cap = cap > kCsrCap ? kCsrCap : cap;
     P.csr_cap = cap < 0 ? 0 : cap & ~7;
@@ -231,6 +237,7 @@ __host__ __device__ inline Plan make_plan(int bits, int n_out, int k_in, int bat
     int stages = (budget - off) / (kWarps * sg_bytes);
     if (stages > kMaxStages) stages = kMaxStages;
     if (stages < kMinStages) stages = kMinStages;
+    if (single) stages = sb_stages;
     P.stages = stages;
     off += stages * kWarps * sg_bytes;
     P.total = off;
@@ -600,7 +607,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_fused_kernel(const 
     uint64_t* rbar = reinterpret_cast<uint64_t*>(smem) + 3;  // sparse pieces written (CT arrivals)
     uint64_t* xbar1 = reinterpret_cast<uint64_t*>(smem) + 4;  // second x buffer (several passes)
     uint16_t* xs = reinterpret_cast<uint16_t*>(smem + P.off_x);
-    const int PS = P.passes, CS = P.chunk_sg;
+    const int PS = SB ? 1 : P.passes, CS = P.chunk_sg;  // batch 1 always takes one pass
     const int xbuf_h = round_up(p.batch * P.x_stride * 2, 128) / 2;  // halves per x buffer
     uint8_t* luts = smem + P.off_lut;
     float* s_rowsum = reinterpret_cast<float*>(smem + P.off_rowsum);
@@ -1173,7 +1180,14 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_fused_kernel(const 
     int s_read = 0, s_fill = D;
 #pragma unroll 1
     for (int i = 0; i < nwu; ++i) {
-        cp_async_wait_newest(D - 1);
+        if constexpr (SB) {
+            if (S == kSbStages)
+                cp_async_wait<kSbStages - 2>();
+            else
+                cp_async_wait<kSbStages - 3>();
+        } else {
+            cp_async_wait_newest(D - 1);
+        }
         uint4 v[V];
         const uint8_t* src = ring + s_read * F::kSgBytes;
 #pragma unroll
