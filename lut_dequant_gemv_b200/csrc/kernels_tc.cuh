@@ -989,25 +989,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_fused_kernel(const 
                 dst[(g + 8) * CM + col + 1] = rr[n][3];
             }
         }
-        __syncwarp();
-        int arrived = 0;
-        if (lane == 0) {
-            __threadfence_block();
-            arrived = atomicAdd(s_cnt + tl, 1) + 1;
-        }
-        arrived = __shfl_sync(0xffffffffu, arrived, 0);
-        if (arrived == __popc(mask)) {
-            __threadfence_block();
-            for (int e = lane; e < TE; e += 32) {
-                const int row_l = e / CM, col = e - row_l * CM;
-                float sum = 0.f;
-                for (int mm = mask; mm; mm &= mm - 1) {
-                    const int wv = __ffs(mm) - 1;
-                    sum += s_slots[(wv * 2 + (tile == s_wrange[wv * 3 + 2] ? 0 : 1)) * TE + e];
-                }
-                out(row0 + row_l, col, sum);
-            }
-        }
+        // shared tiles are combined after the loop (one CTA barrier)
     };
 
     // Decode and multiply-accumulate one unit (16 rows x 256 columns).
@@ -1172,11 +1154,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_fused_kernel(const 
         return;
     }
 
-    if (nwu == 0) return;
-
-    start_tile();
     // Units in order: wait for unit i's group, read its stage, refill the
     // stage freed by unit i-1 with unit i+D, decode.
+    if (nwu > 0) start_tile();
     int s_read = 0, s_fill = D;
 #pragma unroll 1
     for (int i = 0; i < nwu; ++i) {
@@ -1204,6 +1184,22 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_fused_kernel(const 
                 start_tile();
             }
         }
+    }
+    // Tiles shared by several warps: once every warp has left the loop, the
+    // warps' parts are added in warp order (the same order for every batch
+    // size) and the rows get their sparse sums.
+    __syncthreads();
+    for (int idx = tid; idx < ctiles * TE; idx += kThreads) {
+        const int tl = idx / TE, e = idx - tl * TE;
+        const int mask = s_tinfo[tl];
+        if ((mask & (mask - 1)) == 0) continue;  // one warp: already written
+        const int row_l = e / CM, col = e - row_l * CM;
+        float sum = 0.f;
+        for (int mm = mask; mm; mm &= mm - 1) {
+            const int wv = __ffs(mm) - 1;
+            sum += s_slots[(wv * 2 + (t_first + tl == s_wrange[wv * 3 + 2] ? 0 : 1)) * TE + e];
+        }
+        out((t_first + tl) * kTileRows + row_l, col, sum);
     }
 }
 
