@@ -457,22 +457,30 @@ def run_sweep(args):
 
 def run_profile_launches(args):
     """One layer instance, N back-to-back launches on the default stream (a
-    short, bounded program for an ncu capture of one launch per shape)."""
+    short, bounded program for an ncu capture of one launch per shape).
+    ``--workload all``: every shape of every workload in turn, N launches
+    each, one layer alive at a time (launch N*s + j of the fused kernel is
+    launch j of shape s, in the order printed)."""
     import torch
 
     from lut_dequant_gemv_b200 import binding as B
 
     B.lib()
-    shape = shape_for(args)
-    L = synth.layer_for(shape, seed=args.seed)
-    layer = B.create_layer_from_numpy(L.n_out, L.k_in, L.bits, L.codes, L.lut, L.rowptr, L.col, L.val)
-    x = torch.from_numpy(synth.x_for(shape, seed=args.seed).view(np.int16)).cuda()
-    y = torch.empty((shape.batch, shape.n_out), dtype=torch.int16, device="cuda")
-    for _ in range(args.profile_launches):
-        B.sqz_gemv(layer, x, y)
-    torch.cuda.synchronize()
-    print(f"{shape.key} B{shape.batch}: {args.profile_launches} launches", flush=True)
-    layer.close()
+    if args.workload == "all":
+        shapes = [(name, i) for name, ss in synth.workloads().items() for i in range(len(ss))]
+    else:
+        shapes = [(args.workload, args.shape_index)]
+    for name, i in shapes:
+        shape = synth.workloads()[name][i]
+        L = synth.layer_for(shape, seed=args.seed)
+        layer = B.create_layer_from_numpy(L.n_out, L.k_in, L.bits, L.codes, L.lut, L.rowptr, L.col, L.val)
+        x = torch.from_numpy(synth.x_for(shape, seed=args.seed).view(np.int16)).cuda()
+        y = torch.empty((shape.batch, shape.n_out), dtype=torch.int16, device="cuda")
+        for _ in range(args.profile_launches):
+            B.sqz_gemv(layer, x, y)
+        torch.cuda.synchronize()
+        print(f"{name} {i} {shape.key} B{shape.batch}: {args.profile_launches} launches", flush=True)
+        layer.close()
     return 0
 
 
