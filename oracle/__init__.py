@@ -52,6 +52,16 @@ def _bind(lib):
     lib.oracle_check_csr.restype = c_int
     lib.oracle_gemv.argtypes = [i32, i32, c_int, P, P, i64, P, P, P, P, i32, i64, P, i64, P, P]
     lib.oracle_gemv.restype = c_int
+    lib.oracle_double_to_half.argtypes = [ctypes.c_double]
+    lib.oracle_double_to_half.restype = ctypes.c_uint16
+    lib.oracle_outliers_per_tail.argtypes = [i64, ctypes.c_double]
+    lib.oracle_outliers_per_tail.restype = i64
+    lib.oracle_select_outliers.argtypes = [i32, i32, P, i64, P]
+    lib.oracle_select_outliers.restype = c_int
+    lib.oracle_kmeans_row.argtypes = [i64, P, c_int, c_int, P]
+    lib.oracle_kmeans_row.restype = c_int
+    lib.oracle_encode.argtypes = [i32, i32, c_int, P, ctypes.c_double, c_int, P, i32, P, P, P, P, P, i64, P, P]
+    lib.oracle_encode.restype = c_int
     return lib
 
 
@@ -134,6 +144,61 @@ class Oracle:
         if rc:
             raise ValueError("oracle_gemv: bad arguments")
         return y, bound
+
+    # ---- encoder (Dense-and-Sparse split + per-row 1-D k-means), fp64
+    def double_to_half(self, v: float) -> int:
+        return int(self.lib.oracle_double_to_half(float(v)))
+
+    def outliers_per_tail(self, n: int, fraction: float) -> int:
+        return int(self.lib.oracle_outliers_per_tail(int(n), float(fraction)))
+
+    def select_outliers(self, w: np.ndarray, m: int) -> np.ndarray:
+        """uint8 marks [n_out, k_in]: 1 for the first m and last m weights in
+        ascending (value, row-major position) order."""
+        w = _c(w, np.uint16)
+        n_out, k_in = w.shape
+        marks = np.empty((n_out, k_in), dtype=np.uint8)
+        if self.lib.oracle_select_outliers(n_out, k_in, _ptr(w), int(m), _ptr(marks)):
+            raise ValueError("oracle_select_outliers: bad arguments")
+        return marks
+
+    def kmeans_row(self, d: np.ndarray, k: int, max_iters: int) -> Tuple[np.ndarray, int]:
+        """(centroids float64 [k], iterations run) of 1-D Lloyd k-means."""
+        d = _c(d, np.float64)
+        c = np.empty(k, dtype=np.float64)
+        it = self.lib.oracle_kmeans_row(int(d.shape[0]), _ptr(d), int(k), int(max_iters), _ptr(c))
+        if it < 0:
+            raise ValueError("oracle_kmeans_row: bad arguments")
+        return c, int(it)
+
+    def encode(self, w: np.ndarray, bits: int, fraction: float, max_iters: int,
+               rows: Optional[np.ndarray] = None):
+        """Encode fp16 weights [n_out, k_in]: returns dict with codes (canonical
+        words of the requested rows), lut (fp16 bits of those rows), rowptr, col,
+        val (S for all rows), iters (per requested row)."""
+        w = _c(w, np.uint16)
+        n_out, k_in = w.shape
+        wpr = self.lib.oracle_words_per_row(k_in, bits)
+        if wpr < 0:
+            raise ValueError("K*bits must be a multiple of 32")
+        rows_c = None if rows is None else _c(rows, np.int32)
+        n_rows = n_out if rows_c is None else int(rows_c.shape[0])
+        cap = 2 * self.outliers_per_tail(n_out * k_in, fraction)
+        codes = np.zeros((n_rows, wpr), dtype=np.uint32)
+        lut = np.zeros((n_rows, 1 << bits), dtype=np.uint16)
+        rowptr = np.zeros(n_out + 1, dtype=np.int32)
+        col = np.zeros(max(cap, 1), dtype=np.int32)
+        val = np.zeros(max(cap, 1), dtype=np.uint16)
+        nnz = ctypes.c_int64(0)
+        iters = np.zeros(n_rows, dtype=np.int32)
+        rc = self.lib.oracle_encode(n_out, k_in, bits, _ptr(w), float(fraction), int(max_iters), _ptr(rows_c), n_rows,
+                                    _ptr(codes), _ptr(lut), _ptr(rowptr), _ptr(col), _ptr(val), max(cap, 1),
+                                    ctypes.byref(nnz), _ptr(iters))
+        if rc:
+            raise ValueError("oracle_encode: bad arguments")
+        n = int(nnz.value)
+        return {"codes": codes, "lut": lut, "rowptr": rowptr, "col": col[:n].copy(), "val": val[:n].copy(),
+                "iters": iters}
 
     def gemv_layer(self, layer, x, rows=None):
         return self.gemv(layer.n_out, layer.k_in, layer.bits, layer.codes, layer.lut, layer.rowptr,

@@ -179,3 +179,242 @@ int oracle_gemv(int32_t n_out, int32_t k_in, int bits, const uint32_t* codes, co
     }
     return ORACLE_OK;
 }
+
+/* ======================================================================
+ * Encoder: Dense-and-Sparse split and per-row 1-D k-means
+ * ("SqueezeLLM: Dense-and-Sparse Quantization", summary page, section
+ * "Sensitivity-Based Non-Uniform Quantization", Equation 1 and the
+ * weighted k-means procedure without the sensitivity weights; section
+ * "The Dense-and-Sparse Decomposition", W = D + S with percentile
+ * thresholds).  Readings taken where the pages leave a step open:
+ *   - the thresholds are order statistics of all N*K weights of the
+ *     layer: with m = floor(fraction * N * K / 2 + 1/2) (at most N*K/2),
+ *     the outliers are the first m and the last m weights in ascending
+ *     order of (value, row-major position); D is W with those positions set
+ *     to +0 and S holds them exactly (CSR, row-major, ascending column);
+ *   - k-means runs per output row on the K values of that row of D (the
+ *     zeros at outlier positions included), k = 2^b centroids initialised
+ *     uniformly over [min, max] of the row (the uniform grid of the page);
+ *   - one Lloyd iteration assigns every value to its nearest centroid
+ *     (|d - c_j| in fp64, the lowest j on a tie) and sets each centroid to
+ *     the mean of its values (sum in ascending column order, then one
+ *     division); a centroid with no values keeps its place; iterations stop
+ *     when no centroid moves or after max_iters;
+ *   - the LUT holds the final centroids rounded to fp16 (to nearest, ties
+ *     to even), and every weight's code is its nearest LUT entry (lowest
+ *     index on a tie);
+ *   - weights must be finite, and K * max|w| < 2^29 (every partial sum of a
+ *     row's fp16 values is then exact in fp64).
+ * ====================================================================== */
+#include <stdlib.h>
+
+/* double -> binary16, round to nearest, ties to even, from the format's
+ * definition (overflow to infinity). */
+uint16_t oracle_double_to_half(double v) {
+    uint16_t sign = (uint16_t)(signbit(v) ? 0x8000u : 0u);
+    double a = fabs(v);
+    if (isnan(v)) return (uint16_t)(sign | 0x7e00u);
+    if (isinf(a)) return (uint16_t)(sign | 0x7c00u);
+    /* largest finite half is 65504; values >= 65520 round to infinity */
+    if (a >= 65520.0) return (uint16_t)(sign | 0x7c00u);
+    int e;
+    (void)frexp(a, &e); /* a = f * 2^e, f in [0.5, 1) */
+    int ex = e - 1;     /* a in [2^ex, 2^(ex+1)) */
+    if (a == 0.0) return sign;
+    if (ex < -14) ex = -14; /* subnormal range: quantum 2^-24 */
+    double q = ldexp(1.0, ex - 10);  /* spacing of halves in this binade */
+    double n = a / q;               /* exact: q is a power of two */
+    double fl = floor(n);
+    double r = n - fl;
+    if (r > 0.5 || (r == 0.5 && fmod(fl, 2.0) == 1.0)) fl += 1.0;
+    double rounded = fl * q;        /* exact */
+    if (rounded >= 65520.0) return (uint16_t)(sign | 0x7c00u);
+    if (rounded < ldexp(1.0, -14)) {
+        return (uint16_t)(sign | (uint16_t)(rounded / ldexp(1.0, -24))); /* subnormal: mantissa only */
+    }
+    int e2;
+    double f2 = frexp(rounded, &e2); /* rounded = f2 * 2^e2 */
+    int biased = e2 - 1 + 15;
+    uint16_t mant = (uint16_t)((f2 * 2.0 - 1.0) * 1024.0);
+    return (uint16_t)(sign | (uint16_t)(biased << 10) | mant);
+}
+
+int64_t oracle_outliers_per_tail(int64_t n, double fraction) {
+    if (n <= 0 || !(fraction >= 0.0)) return 0;
+    int64_t m = (int64_t)floor(fraction * (double)n / 2.0 + 0.5);
+    if (m > n / 2) m = n / 2;
+    return m;
+}
+
+typedef struct {
+    double v;
+    int64_t pos;
+} oracle_vp;
+
+static int oracle_vp_cmp(const void* a, const void* b) {
+    const oracle_vp* x = (const oracle_vp*)a;
+    const oracle_vp* y = (const oracle_vp*)b;
+    if (x->v < y->v) return -1;
+    if (x->v > y->v) return 1;
+    return (x->pos < y->pos) ? -1 : (x->pos > y->pos) ? 1 : 0;
+}
+
+/* marks[p] = 1 where weight p (row-major) is an outlier: the first m and the
+ * last m in ascending (value, position) order. */
+int oracle_select_outliers(int32_t n_out, int32_t k_in, const uint16_t* w, int64_t m, uint8_t* marks) {
+    int64_t n = (int64_t)n_out * k_in;
+    if (n_out < 0 || k_in < 0 || m < 0 || 2 * m > n) return ORACLE_BAD_ARG;
+    memset(marks, 0, (size_t)n);
+    if (m == 0) return ORACLE_OK;
+    oracle_vp* a = (oracle_vp*)malloc((size_t)n * sizeof(oracle_vp));
+    if (!a) return ORACLE_BAD_ARG;
+    for (int64_t p = 0; p < n; ++p) {
+        a[p].v = oracle_half_to_double(w[p]) + 0.0; /* -0 and +0 are one value */
+        a[p].pos = p;
+    }
+    qsort(a, (size_t)n, sizeof(oracle_vp), oracle_vp_cmp);
+    for (int64_t t = 0; t < m; ++t) {
+        marks[a[t].pos] = 1;
+        marks[a[n - 1 - t].pos] = 1;
+    }
+    free(a);
+    return ORACLE_OK;
+}
+
+/* 1-D k-means (Lloyd) of n values, kc centroids; returns the iterations run. */
+int oracle_kmeans_row(int64_t n, const double* d, int kc, int max_iters, double* c) {
+    if (n <= 0 || kc < 2 || kc > 16) return -1;
+    double lo = d[0], hi = d[0];
+    for (int64_t k = 1; k < n; ++k) {
+        if (d[k] < lo) lo = d[k];
+        if (d[k] > hi) hi = d[k];
+    }
+    double step = (hi - lo) / (double)(kc - 1);
+    for (int j = 0; j < kc; ++j) c[j] = lo + (double)j * step;
+    int it = 0;
+    for (; it < max_iters; ++it) {
+        double sum[16];
+        int64_t cnt[16];
+        for (int j = 0; j < kc; ++j) {
+            sum[j] = 0.0;
+            cnt[j] = 0;
+        }
+        for (int64_t k = 0; k < n; ++k) {
+            int best = 0;
+            double bd = fabs(d[k] - c[0]);
+            for (int j = 1; j < kc; ++j) {
+                double dj = fabs(d[k] - c[j]);
+                if (dj < bd) {
+                    bd = dj;
+                    best = j;
+                }
+            }
+            sum[best] += d[k];
+            cnt[best] += 1;
+        }
+        int moved = 0;
+        for (int j = 0; j < kc; ++j) {
+            double nc = cnt[j] ? sum[j] / (double)cnt[j] : c[j];
+            if (nc != c[j]) moved = 1;
+            c[j] = nc;
+        }
+        if (!moved) {
+            ++it;
+            break;
+        }
+    }
+    return it;
+}
+
+/* Encode a layer: outliers to CSR (all rows), then for each requested row
+ * (all rows when rows == NULL) the k-means LUT and the codes.  codes is
+ * [n_rows][K*bits/32] canonical words, lut [n_rows][2^bits]; rowptr, col,
+ * val describe S for all rows (nnz_cap entries available). */
+int oracle_encode(int32_t n_out, int32_t k_in, int bits, const uint16_t* w, double fraction, int max_iters,
+                  const int32_t* rows, int32_t n_rows, uint32_t* codes, uint16_t* lut, int32_t* rowptr, int32_t* col,
+                  uint16_t* val, int64_t nnz_cap, int64_t* nnz_out, int32_t* iters_out) {
+    int64_t wpr = oracle_words_per_row(k_in, bits);
+    if (wpr < 0 || n_out < 1 || k_in < 1 || max_iters < 0) return ORACLE_BAD_ARG;
+    int64_t n = (int64_t)n_out * k_in;
+    double amax = 0.0;
+    for (int64_t p = 0; p < n; ++p) {
+        double v = oracle_half_to_double(w[p]);
+        if (!isfinite(v)) return ORACLE_BAD_ARG;
+        if (fabs(v) > amax) amax = fabs(v);
+    }
+    if (amax * (double)k_in >= ldexp(1.0, 29)) return ORACLE_BAD_ARG;
+    int64_t m = oracle_outliers_per_tail(n, fraction);
+    uint8_t* marks = (uint8_t*)malloc((size_t)n);
+    if (!marks) return ORACLE_BAD_ARG;
+    if (oracle_select_outliers(n_out, k_in, w, m, marks) != ORACLE_OK) {
+        free(marks);
+        return ORACLE_BAD_ARG;
+    }
+    int64_t nnz = 0;
+    rowptr[0] = 0;
+    for (int64_t i = 0; i < n_out; ++i) {
+        for (int64_t k = 0; k < k_in; ++k) {
+            if (!marks[i * k_in + k]) continue;
+            if (nnz >= nnz_cap) {
+                free(marks);
+                return ORACLE_BAD_ARG;
+            }
+            col[nnz] = (int32_t)k;
+            val[nnz] = w[i * k_in + k];
+            ++nnz;
+        }
+        rowptr[i + 1] = (int32_t)nnz;
+    }
+    *nnz_out = nnz;
+    int L = 1 << bits;
+    if (rows == NULL) n_rows = n_out;
+    double* d = (double*)malloc((size_t)k_in * sizeof(double));
+    uint8_t* cm = (uint8_t*)malloc((size_t)k_in);
+    if (!d || !cm) {
+        free(marks);
+        free(d);
+        free(cm);
+        return ORACLE_BAD_ARG;
+    }
+    for (int64_t r = 0; r < n_rows; ++r) {
+        int64_t i = rows ? rows[r] : r;
+        if (i < 0 || i >= n_out) {
+            free(marks);
+            free(d);
+            free(cm);
+            return ORACLE_BAD_ARG;
+        }
+        for (int64_t k = 0; k < k_in; ++k)
+            d[k] = marks[i * k_in + k] ? 0.0 : oracle_half_to_double(w[i * k_in + k]) + 0.0;
+        double c[16];
+        int it = oracle_kmeans_row(k_in, d, L, max_iters, c);
+        if (iters_out) iters_out[r] = it;
+        double lv[16];
+        for (int j = 0; j < L; ++j) {
+            lut[r * L + j] = oracle_double_to_half(c[j]);
+            lv[j] = oracle_half_to_double(lut[r * L + j]);
+        }
+        for (int64_t k = 0; k < k_in; ++k) {
+            int best = 0;
+            double bd = fabs(d[k] - lv[0]);
+            for (int j = 1; j < L; ++j) {
+                double dj = fabs(d[k] - lv[j]);
+                if (dj < bd) {
+                    bd = dj;
+                    best = j;
+                }
+            }
+            cm[k] = (uint8_t)best;
+        }
+        if (oracle_pack(1, k_in, bits, cm, codes + r * wpr) != ORACLE_OK) {
+            free(marks);
+            free(d);
+            free(cm);
+            return ORACLE_BAD_ARG;
+        }
+    }
+    free(marks);
+    free(d);
+    free(cm);
+    return ORACLE_OK;
+}

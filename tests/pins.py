@@ -401,4 +401,167 @@ def pin_csr_checks(orc):
     assert not orc.check_csr(3, 8, rp, np.array([1, -1, 0], dtype=np.int32))
 
 
+# ------------------------------------------------------------ encoder pins ---
+# The encoder ("SqueezeLLM" summary page: Eq. 1 k-means and the
+# Dense-and-Sparse decomposition) checked against numpy's fp16 rounding,
+# numpy's sort, scikit-learn's Lloyd k-means, exact rational arithmetic and
+# the uniform grid the page prints.
+
+def pin_enc_double_to_half_matches_numpy(orc):
+    rng = np.random.default_rng(41)
+    vals = rng.standard_normal(20000) * np.exp(rng.uniform(-22, 12, 20000))
+    edge = [0.0, -0.0, 65504.0, 65519.99, 65520.0, 1e6, 2.0 ** -24, 2.0 ** -25, 1.5 * 2.0 ** -24, 2.0 ** -14,
+            2.0 ** -14 - 2.0 ** -25, 1.0 + 2.0 ** -11, 1.0 + 3 * 2.0 ** -11, 1 / 3, -2.5e-8]
+    vals = np.concatenate([vals, edge, -np.array(edge)])
+    with np.errstate(over="ignore"):
+        want = vals.astype(np.float16).view(np.uint16)
+    got = np.array([orc.double_to_half(v) for v in vals], dtype=np.uint16)
+    assert np.array_equal(got, want), int((got != want).sum())
+
+
+def pin_enc_outlier_tails_page_example(orc):
+    # 0.2th / 99.8th percentiles: 0.4 % of the weights, 0.2 % in each tail
+    assert orc.outliers_per_tail(100000, 0.004) == 200
+    assert orc.outliers_per_tail(1000, 0.0045) == 2  # 2.25 rounds to 2
+    assert orc.outliers_per_tail(1000, 0.005) == 3   # 2.5 rounds up (the reading taken)
+    assert orc.outliers_per_tail(10, 1.0) == 5        # at most half the weights per tail
+
+
+def pin_enc_outlier_selection_is_order_statistics(orc):
+    rng = np.random.default_rng(42)
+    # values from a small set so that the thresholds fall inside runs of ties
+    pool = (np.arange(-40, 41) / 64.0).astype(np.float16)
+    w = rng.choice(pool, size=(24, 96), p=None).astype(np.float16)
+    w[rng.integers(0, 24, 6), rng.integers(0, 96, 6)] = np.float16(-0.0)
+    n = w.size
+    for m in (0, 1, 7, 37, 200):
+        marks = orc.select_outliers(w.view(np.uint16), m).ravel()
+        v = w.astype(np.float64).ravel() + 0.0
+        order = np.lexsort((np.arange(n), v))  # numpy sort by value, then position
+        want = np.zeros(n, dtype=np.uint8)
+        want[order[:m]] = 1
+        want[order[n - m:]] = 1
+        assert np.array_equal(marks, want), m
+        assert int(marks.sum()) == 2 * m
+        if m:
+            lo_sel, hi_sel = order[:m], order[n - m:]
+            rest = v[marks == 0]
+            assert v[lo_sel].max() <= rest.min() and rest.max() <= v[hi_sel].min()
+
+
+def pin_enc_kmeans_page_uniform_init(orc):
+    g = {r[0]: r[1:] for r in read_golden("uniform_grid_3bit.txt")}
+    lo, hi, k = float(g["w_min"][0]), float(g["w_max"][0]), int(g["k"][0])
+    d = np.linspace(lo, hi, 101)
+    c, it = orc.kmeans_row(d, k, 0)
+    assert it == 0
+    assert np.allclose(c, [float(t) for t in g["values"]], atol=5e-4)
+    assert abs((c[1] - c[0]) - float(g["width"][0])) < 5e-4
+
+
+def pin_enc_kmeans_empty_clusters_keep_place(orc):
+    # clusters 1..6 of the grid over [0, 1] get no values: they stay where
+    # they started, the two others settle on the means 0 and 1
+    d = np.array([0.0, 0.0, 0.0, 1.0])
+    c, it = orc.kmeans_row(d, 8, 10)
+    assert it <= 2
+    assert np.allclose(c, np.array([j / 7.0 for j in range(8)]), rtol=0, atol=1e-15)
+    assert c[0] == 0.0 and c[7] == 1.0
+
+
+def pin_enc_kmeans_matches_sklearn(orc):
+    from sklearn.cluster import KMeans
+
+    rng = np.random.default_rng(43)
+    for k in (8, 16):
+        # one tight group of values near each point of the starting grid (no
+        # cluster ever empties, where the two implementations would differ)
+        grid = np.linspace(-0.05, 0.05, k)
+        centres = grid + rng.uniform(-0.2, 0.2, k) * (grid[1] - grid[0])
+        centres[0], centres[-1] = grid[0], grid[-1]
+        d = np.concatenate([c0 + rng.standard_normal(64) * 2e-4 for c0 in centres])
+        d = d.astype(np.float16).astype(np.float64)
+        c, it = orc.kmeans_row(d, k, 100)
+        init = d.min() + np.arange(k) * ((d.max() - d.min()) / (k - 1))
+        km = KMeans(n_clusters=k, init=init.reshape(-1, 1), n_init=1, max_iter=100, tol=0.0,
+                    algorithm="lloyd").fit(d.reshape(-1, 1))
+        ref = np.sort(km.cluster_centers_.ravel())
+        assert it < 100
+        assert np.allclose(np.sort(c), ref, rtol=0, atol=1e-12), (k, np.abs(np.sort(c) - ref).max())
+
+
+def pin_enc_kmeans_fixed_point_exact(orc):
+    rng = np.random.default_rng(44)
+    d = (rng.standard_normal(300) * 0.02).astype(np.float16).astype(np.float64)
+    c, it = orc.kmeans_row(d, 8, 200)
+    assert it < 200
+    cf = [Fraction(x) for x in c]
+    groups = [[] for _ in range(8)]
+    for v in d:
+        fv = Fraction(v)
+        dist = [abs(fv - cj) for cj in cf]
+        groups[dist.index(min(dist))].append(fv)
+    for j in range(8):
+        if groups[j]:
+            mean = sum(groups[j]) / len(groups[j])
+            assert abs(float(mean) - c[j]) <= 2.0 ** -52 * abs(c[j]), j
+
+
+def pin_enc_kmeans_sse_nonincreasing(orc):
+    rng = np.random.default_rng(45)
+    d = (rng.standard_t(4, 512) * 0.02).astype(np.float16).astype(np.float64)
+    prev = None
+    for t in range(0, 8):
+        c, _ = orc.kmeans_row(d, 8, t)
+        sse = float(np.min((d[:, None] - c[None, :]) ** 2, axis=1).sum())
+        if prev is not None:
+            assert sse <= prev * (1 + 1e-12), t
+        prev = sse
+
+
+def pin_enc_codes_are_nearest_fp16_entry(orc):
+    # a wider layer: every code must index the nearest entry of the row's
+    # fp16 LUT (fp16 - fp16 differences are exact in fp64; argmin takes the
+    # lowest index on a tie), which the codes of the unrounded centroids are
+    # not, for values close to a midpoint
+    rng = np.random.default_rng(47)
+    n_out, k_in, bits = 6, 4096, 3
+    w = (rng.standard_normal((n_out, k_in)) * 0.02).astype(np.float16)
+    r = orc.encode(w.view(np.uint16), bits, 0.0045, 30)
+    dense = w.astype(np.float64).copy()
+    for i in range(n_out):
+        dense[i, r["col"][r["rowptr"][i]:r["rowptr"][i + 1]]] = 0.0
+    for i in range(n_out):
+        lut = r["lut"][i].view(np.float16).astype(np.float64)
+        want = np.argmin(np.abs(dense[i][:, None] - lut[None, :]), axis=1)
+        got = np.array(bigint_codes(r["codes"][i], bits, k_in))
+        assert np.array_equal(got, want), (i, int((got != want).sum()))
+
+
+def pin_enc_layer_reconstruction(orc):
+    rng = np.random.default_rng(46)
+    n_out, k_in, frac = 12, 64, 0.03
+    for bits in (3, 4):
+        w = (rng.standard_normal((n_out, k_in)) * 0.02).astype(np.float16)
+        w[rng.integers(0, n_out, 5), rng.integers(0, k_in, 5)] = np.float16(0.7)
+        r = orc.encode(w.view(np.uint16), bits, frac, 40)
+        m = orc.outliers_per_tail(w.size, frac)
+        rowptr, col, val = r["rowptr"], r["col"], r["val"]
+        assert rowptr[0] == 0 and rowptr[-1] == 2 * m and np.all(np.diff(rowptr) >= 0)
+        wv = w.view(np.uint16)
+        outl = np.zeros((n_out, k_in), dtype=bool)
+        for i in range(n_out):
+            cs = col[rowptr[i]:rowptr[i + 1]]
+            assert np.all(np.diff(cs) > 0)
+            assert np.array_equal(val[rowptr[i]:rowptr[i + 1]], wv[i, cs])
+            outl[i, cs] = True
+        for i in range(n_out):
+            lut = [Fraction(float(x)) for x in r["lut"][i].view(np.float16)]
+            codes = bigint_codes(r["codes"][i], bits, k_in)
+            for k in range(k_in):
+                target = Fraction(0) if outl[i, k] else Fraction(float(w[i, k]))
+                dist = [abs(target - e) for e in lut]
+                assert codes[k] == dist.index(min(dist)), (bits, i, k)
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

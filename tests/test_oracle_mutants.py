@@ -25,6 +25,18 @@ MUTANTS = [
     ("code_row_stride", r"codes \+ i \* wpr;\n        for \(int64_t b", "codes + (i % 2) * wpr;\n        for (int64_t b"),
     ("row_end_exclusive", r"j < rowptr\[i \+ 1\]; \+\+j\) \{\n                    double t",
      "j < rowptr[i + 1] - 1; ++j) {\n                    double t"),
+    # encoder
+    ("half_truncates", r"if \(r > 0\.5 \|\| \(r == 0\.5 && fmod\(fl, 2\.0\) == 1\.0\)\) fl \+= 1\.0;", ""),
+    ("half_ties_up", r"r == 0\.5 && fmod\(fl, 2\.0\) == 1\.0", "r == 0.5"),
+    ("one_tail_only", r"marks\[a\[n - 1 - t\]\.pos\] = 1;", ""),
+    ("tail_rounding_floor", r"floor\(fraction \* \(double\)n / 2\.0 \+ 0\.5\)", "floor(fraction * (double)n / 2.0)"),
+    ("ties_by_position_reversed", r"return \(x->pos < y->pos\) \? -1 : \(x->pos > y->pos\) \? 1 : 0;",
+     "return (x->pos < y->pos) ? 1 : (x->pos > y->pos) ? -1 : 0;"),
+    ("init_grid_from_zero", r"c\[j\] = lo \+ \(double\)j \* step;", "c[j] = (double)j * step;"),
+    ("empty_cluster_to_zero", r"cnt\[j\] \? sum\[j\] / \(double\)cnt\[j\] : c\[j\]", "cnt[j] ? sum[j] / (double)cnt[j] : 0.0"),
+    ("mean_over_all_values", r"sum\[j\] / \(double\)cnt\[j\]", "sum[j] / (double)n"),
+    ("outliers_left_in_dense", r"d\[k\] = marks\[i \* k_in \+ k\] \? 0\.0 : ", "d[k] = marks[i * k_in + k] ? oracle_half_to_double(w[i * k_in + k]) : "),
+    ("codes_from_unrounded_centroids", r"lv\[j\] = oracle_half_to_double\(lut\[r \* L \+ j\]\);", "lv[j] = c[j];"),
 ]
 
 
