@@ -242,6 +242,57 @@ SQZ_API sqz_status sqz_fp16_gemv(const uint16_t* w, int32_t n_out, int32_t k_in,
 SQZ_API sqz_status sqz_check_csr_static(const int32_t* rowptr, const int32_t* col, int32_t n_out, int32_t k_in,
                                         int64_t nnz, void* stream, int32_t* flags);
 
+/* ------------------------------------------------------------ encoder ---
+ * Quantize an fp16 weight matrix into the layer format sqz_create_layer
+ * takes ("SqueezeLLM: Dense-and-Sparse Quantization", summary page:
+ * "The Dense-and-Sparse Decomposition", W = D + S with S the weights beyond
+ * two percentile thresholds, kept exactly in CSR; "Sensitivity-Based
+ * Non-Uniform Quantization", Eq. 1: per output row a 1-D k-means over the
+ * row's values gives the 2^bits centroids of the row's LUT, each weight is
+ * stored as the index of its centroid; the sensitivity weighting, which
+ * needs gradients of a real model, is not part of it).
+ *
+ * Definition (every step exact, so the result is unique):
+ *   - m = floor(outlier_fraction * n_out * k_in / 2 + 1/2), at most half
+ *     the weights; the outliers are the first m and the last m weights in
+ *     ascending order of (value, row-major position), -0 and +0 being one
+ *     value (the 0.2th/99.8th percentiles of the page are fraction 0.004);
+ *   - D = W with the outliers set to +0; per row of D, k-means with
+ *     2^bits centroids starting from the uniform grid over [min, max] of the
+ *     row; each Lloyd iteration assigns every value to its nearest centroid
+ *     (|d - c_j| in fp64, the lowest j on a tie) and moves each centroid to
+ *     the mean of its values (an empty centroid stays); it stops when no
+ *     centroid moves or after max_iters iterations;
+ *   - lut = the centroids rounded to fp16 (nearest, ties to even); each
+ *     weight's code = its nearest lut entry (lowest index on a tie), packed
+ *     as sqz_layer_desc.codes (canonical LSB-first bitstream).
+ *
+ * w: device fp16 bits [n_out][k_in], row-major, read only.  Outputs
+ * (device, caller-owned): codes [n_out][k_in*bits/32], lut [n_out][2^bits],
+ * rowptr [n_out+1], col and val [nnz_capacity] (NULL allowed when no
+ * outliers are asked for), iters_out [n_out] (may be NULL: the iterations
+ * each row ran).  *nnz_out (host) receives the number of outliers, which is
+ * sqz_encode_outliers(n_out * k_in, outlier_fraction) -- size col/val with it.
+ * The call is ordered on `stream`, allocates a device workspace of about
+ * n_out*k_in bytes, and synchronises the stream before returning.
+ *
+ * Errors: SQZ_ERR_INVALID_ARG for NULL w/codes/lut/rowptr/nnz_out, bits not
+ * in {3,4}, n_out or k_in < 1, k_in not a multiple of 32 (3-bit) or 8 (4-bit),
+ * outlier_fraction outside [0,1], max_iters outside [0,100000], nnz_capacity
+ * below the outlier count, NULL col/val with outliers, or weights that are
+ * inf or NaN; SQZ_ERR_UNSUPPORTED when k_in * max|w| reaches 2^29 (row sums of
+ * fp16 values are then no longer exact in fp64) or the outliers exceed the
+ * int32 range; SQZ_ERR_OOM; SQZ_ERR_CUDA.
+ */
+SQZ_API sqz_status sqz_encode(const uint16_t* w, int32_t n_out, int32_t k_in, int32_t bits, double outlier_fraction,
+                              int32_t max_iters, uint32_t* codes, uint16_t* lut, int32_t* rowptr, int32_t* col,
+                              uint16_t* val, int64_t nnz_capacity, int64_t* nnz_out, int32_t* iters_out,
+                              void* stream);
+
+/* Outliers sqz_encode selects for n_weights weights at outlier_fraction
+ * (2*m above; 0 for n_weights <= 0 or a negative or NaN fraction). */
+SQZ_API int64_t sqz_encode_outliers(int64_t n_weights, double outlier_fraction);
+
 /* Message for the calling thread's last non-OK status ("" if none). */
 SQZ_API const char* sqz_last_error(void);
 

@@ -37,7 +37,8 @@ STATUS_NAMES = {0: "SQZ_OK", 1: "SQZ_ERR_INVALID_ARG", 2: "SQZ_ERR_UNSUPPORTED",
 # Every entry point include/sqz.h declares.
 EXPORTED = ("sqz_create_layer", "sqz_gemv", "sqz_gemv_host", "sqz_debug_dequant", "sqz_layer_info",
             "sqz_destroy", "sqz_fp16_gemv", "sqz_last_error", "sqz_version", "sqz_check_csr_static",
-            "sqz_layer_set_mac", "sqz_layer_set_csr_mode", "sqz_layer_status")
+            "sqz_layer_set_mac", "sqz_layer_set_csr_mode", "sqz_layer_status", "sqz_encode",
+            "sqz_encode_outliers")
 
 
 class SqzError(RuntimeError):
@@ -90,6 +91,11 @@ def lib() -> ctypes.CDLL:
         L.sqz_layer_status.restype = ctypes.c_int
         L.sqz_check_csr_static.argtypes = [P, P, i32, i32, i64, P, ctypes.POINTER(i32)]
         L.sqz_check_csr_static.restype = ctypes.c_int
+        L.sqz_encode.argtypes = [P, i32, i32, i32, ctypes.c_double, i32, P, P, P, P, P, i64,
+                                 ctypes.POINTER(i64), P, P]
+        L.sqz_encode.restype = ctypes.c_int
+        L.sqz_encode_outliers.argtypes = [i64, ctypes.c_double]
+        L.sqz_encode_outliers.restype = i64
         L.sqz_last_error.argtypes = []
         L.sqz_last_error.restype = ctypes.c_char_p
         L.sqz_version.argtypes = []
@@ -289,6 +295,36 @@ def sqz_check_csr_static(rowptr: Optional[torch.Tensor], col: Optional[torch.Ten
                                       n_out, k_in, nnz, _stream(stream), ctypes.byref(flags)),
            "sqz_check_csr_static")
     return int(flags.value)
+
+
+def sqz_encode_outliers(n_weights: int, outlier_fraction: float) -> int:
+    return int(lib().sqz_encode_outliers(int(n_weights), float(outlier_fraction)))
+
+
+def sqz_encode(w: torch.Tensor, bits: int, outlier_fraction: float, max_iters: int, stream=None,
+               want_iters: bool = False):
+    """Quantize fp16 weights [n_out, k_in] (CUDA) into (codes, lut, rowptr, col,
+    val[, iters]) device tensors in the layout sqz_create_layer takes."""
+    if w.dim() != 2 or not w.is_contiguous():
+        raise ValueError("w must be a contiguous [n_out, k_in] tensor")
+    n_out, k_in = (int(d) for d in w.shape)
+    dev = w.device
+    nnz = sqz_encode_outliers(n_out * k_in, outlier_fraction)
+    wpr = k_in * bits // 32 if bits in (3, 4) else 0
+    codes = torch.empty((n_out, max(wpr, 1)), dtype=torch.int32, device=dev)
+    lut = torch.empty((n_out, 1 << bits if bits in (3, 4) else 1), dtype=torch.int16, device=dev)
+    rowptr = torch.empty(n_out + 1, dtype=torch.int32, device=dev)
+    col = torch.empty(max(nnz, 1), dtype=torch.int32, device=dev)
+    val = torch.empty(max(nnz, 1), dtype=torch.int16, device=dev)
+    iters = torch.empty(n_out, dtype=torch.int32, device=dev) if want_iters else None
+    got = ctypes.c_int64(0)
+    _check(lib().sqz_encode(_dptr_any(w, "w"), n_out, k_in, int(bits), float(outlier_fraction), int(max_iters),
+                            codes.data_ptr(), lut.data_ptr(), rowptr.data_ptr(), col.data_ptr(), val.data_ptr(),
+                            max(nnz, 1), ctypes.byref(got), None if iters is None else iters.data_ptr(),
+                            _stream(stream)), "sqz_encode")
+    n = int(got.value)
+    out = (codes[:, :wpr], lut, rowptr, col[:n], val[:n])
+    return out + (iters,) if want_iters else out
 
 
 def sqz_layer_set_mac(layer: Layer, mac: int) -> None:

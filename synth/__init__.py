@@ -42,7 +42,7 @@ import numpy as np
 
 FP16_MAX = 65504.0
 
-_TENSOR_IDS = {"lut": 1, "codes": 2, "pos": 3, "sign": 4, "mag": 5, "x": 6, "rows": 7}
+_TENSOR_IDS = {"lut": 1, "codes": 2, "pos": 3, "sign": 4, "mag": 5, "x": 6, "rows": 7, "w": 8}
 
 
 def _rng(seed: int, key: str, instance: int, tensor: str) -> np.random.Generator:
@@ -144,6 +144,15 @@ def make_layer(n_out: int, k_in: int, bits: int, density: float, *, seed: int = 
     codes = draw_codes(_rng(seed, key, instance, "codes"), n_out, k_in, bits)
     rowptr, col, val = draw_outliers(seed, key, instance, n_out, k_in, density, dist)
     return Layer(n_out, k_in, bits, codes, lut, rowptr, col, val)
+
+
+def make_weights(n_out: int, k_in: int, *, seed: int = 0, key: str = "weights", instance: int = 0,
+                 scale: float = 0.02, df: float = 4.0) -> np.ndarray:
+    """Dense fp16 weights for the encoder: scale * Student-t(df) per entry,
+    rounded to fp16 (bits as uint16).  Heavy tails give the few extreme
+    values per layer that the Dense-and-Sparse split is for."""
+    w = scale * _rng(seed, key, instance, "w").standard_t(df, size=(n_out, k_in))
+    return w.astype(np.float16).view(np.uint16)
 
 
 def make_x(batch: int, k_in: int, *, seed: int = 0, key: str = "layer", instance: int = 0) -> np.ndarray:

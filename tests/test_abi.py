@@ -98,3 +98,37 @@ def test_layer_options_reject_null_handles_and_unknown_values(lib):
     assert lib.sqz_layer_set_mac(None, 0) == B.SQZ_ERR_INVALID_ARG
     assert lib.sqz_layer_set_csr_mode(None, B.SQZ_CSR_ROWWISE) == B.SQZ_ERR_INVALID_ARG
     assert "NULL" in B.sqz_last_error()
+
+
+def test_encode_outlier_count_matches_the_oracle(lib, orc):
+    # the count the caller sizes col/val with: 2 * floor(f * n / 2 + 1/2), at most n
+    for n in (0, 1, 7, 1000, 4096 * 4096, 11008 * 4096):
+        for f in (0.0, 0.004, 0.0045, 0.005, 0.5, 1.0):
+            assert B.sqz_encode_outliers(n, f) == 2 * orc.outliers_per_tail(n, f), (n, f)
+    assert B.sqz_encode_outliers(100, -0.1) == 0
+    assert B.sqz_encode_outliers(100, float("nan")) == 0
+
+
+@pytest.mark.parametrize("kw,msg", [
+    (dict(w=None), "non-NULL"),
+    (dict(bits=5), "bits"),
+    (dict(n_out=0), "positive"),
+    (dict(k_in=48), "multiple of 32"),
+    (dict(fraction=1.5), "outlier_fraction"),
+    (dict(fraction=float("nan")), "outlier_fraction"),
+    (dict(iters=-1), "max_iters"),
+    (dict(cap=3), "capacity"),
+    (dict(col=None), "col and val"),
+])
+def test_encode_rejects_bad_arguments_before_touching_the_device(lib, kw, msg):
+    import ctypes
+
+    a = dict(w=0x1000, n_out=64, k_in=64, bits=3, fraction=0.01, iters=10, codes=0x2000, lut=0x3000,
+             rowptr=0x4000, col=0x5000, val=0x6000, cap=1024)
+    a.update(kw)
+    nnz = ctypes.c_int64(-1)
+    st = lib.sqz_encode(a["w"], a["n_out"], a["k_in"], a["bits"], a["fraction"], a["iters"], a["codes"], a["lut"],
+                        a["rowptr"], a["col"], a["val"], a["cap"], ctypes.byref(nnz), None, None)
+    assert st == B.SQZ_ERR_INVALID_ARG
+    assert msg in B.sqz_last_error()
+    assert nnz.value == 0
