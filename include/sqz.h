@@ -281,8 +281,9 @@ SQZ_API sqz_status sqz_check_csr_static(const int32_t* rowptr, const int32_t* co
  * outlier_fraction outside [0,1], max_iters outside [0,100000], nnz_capacity
  * below the outlier count, NULL col/val with outliers, or weights that are
  * inf or NaN; SQZ_ERR_UNSUPPORTED when k_in * max|w| reaches 2^29 (row sums of
- * fp16 values are then no longer exact in fp64) or the outliers exceed the
- * int32 range; SQZ_ERR_OOM; SQZ_ERR_CUDA.
+ * fp16 values are then no longer exact in fp64), k_in exceeds 102400 (a row
+ * is staged in 200 KB of shared memory) or the outliers exceed the int32
+ * range; SQZ_ERR_OOM; SQZ_ERR_CUDA.
  */
 SQZ_API sqz_status sqz_encode(const uint16_t* w, int32_t n_out, int32_t k_in, int32_t bits, double outlier_fraction,
                               int32_t max_iters, uint32_t* codes, uint16_t* lut, int32_t* rowptr, int32_t* col,

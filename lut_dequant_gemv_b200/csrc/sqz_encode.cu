@@ -229,25 +229,37 @@ __device__ __forceinline__ uint16_t d2h_rne(double v) {
     return (uint16_t)(sign | (uint16_t)q);  // subnormal (q == 1024 is the smallest normal)
 }
 
-// One warp per row: Lloyd k-means on the row of D, then the LUT and the codes.
+// One CTA of kThreads threads per row: Lloyd k-means on the row of D, then
+// the LUT and the codes.  The row of D is first copied into shared memory
+// (fp16, +0 at the outliers and for -0); each iteration every thread
+// assigns its values (columns tid, tid + kThreads, ...) and sums them per
+// centroid as integers in units of 2^-24, the warps' sums are added in
+// shared memory (integer sums: exact in any order), and the new centroids
+// are formed once and broadcast.
 template <int BITS>
 __global__ void __launch_bounds__(kThreads) kmeans_kernel(const uint16_t* __restrict__ w,
                                                           const uint8_t* __restrict__ flags, int32_t n_out,
                                                           int32_t k_in, int max_iters, uint32_t* __restrict__ codes,
                                                           uint16_t* __restrict__ lut, int32_t* __restrict__ iters_out) {
     constexpr int L = 1 << BITS;
-    const int lane = threadIdx.x & 31;
+    constexpr int NW = kThreads / 32;
+    extern __shared__ __align__(16) uint16_t dr[];  // [k_in]
+    __shared__ long long s_sum[NW][L];
+    __shared__ int s_cnt[NW][L];
+    __shared__ double s_c[L], s_lo[NW], s_hi[NW];
+    __shared__ int s_moved;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const int64_t wpr = (int64_t)k_in * BITS / 32;
-    for (int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; i < n_out;
-         i += ((int64_t)gridDim.x * blockDim.x) >> 5) {
+    for (int64_t i = blockIdx.x; i < n_out; i += gridDim.x) {
         const uint16_t* wr = w + i * k_in;
         const uint8_t* fr = flags + i * k_in;
-        auto value = [&](int64_t k) -> double {  // d(i, k): +0 at outliers, -0 read as +0
-            return fr[k] ? 0.0 : (double)__half2float(__ushort_as_half(wr[k])) + 0.0;
-        };
+        __syncthreads();
         double lo = INFINITY, hi = -INFINITY;
-        for (int64_t k = lane; k < k_in; k += 32) {
-            const double d = value(k);
+        for (int64_t k = tid; k < k_in; k += kThreads) {
+            const uint16_t h = wr[k];
+            const uint16_t v = (fr[k] || h == 0x8000u) ? (uint16_t)0 : h;
+            dr[k] = v;
+            const double d = (double)__half2float(__ushort_as_half(v));
             lo = fmin(lo, d);
             hi = fmax(hi, d);
         }
@@ -255,18 +267,30 @@ __global__ void __launch_bounds__(kThreads) kmeans_kernel(const uint16_t* __rest
             lo = fmin(lo, __shfl_xor_sync(0xffffffffu, lo, o));
             hi = fmax(hi, __shfl_xor_sync(0xffffffffu, hi, o));
         }
+        if (lane == 0) {
+            s_lo[wid] = lo;
+            s_hi[wid] = hi;
+        }
+        __syncthreads();
+        lo = s_lo[0];
+        hi = s_hi[0];
+#pragma unroll
+        for (int v = 1; v < NW; ++v) {
+            lo = fmin(lo, s_lo[v]);
+            hi = fmax(hi, s_hi[v]);
+        }
         double c[L];
         const double step = __ddiv_rn(__dsub_rn(hi, lo), (double)(L - 1));
 #pragma unroll
         for (int j = 0; j < L; ++j) c[j] = __dadd_rn(lo, __dmul_rn((double)j, step));
         int it = 0;
         for (; it < max_iters; ++it) {
-            long long s[L];
+            long long sm[L];
             int cnt[L];
 #pragma unroll
-            for (int j = 0; j < L; ++j) s[j] = 0, cnt[j] = 0;
-            for (int64_t k = lane; k < k_in; k += 32) {
-                const double d = value(k);
+            for (int j = 0; j < L; ++j) sm[j] = 0, cnt[j] = 0;
+            for (int64_t k = tid; k < k_in; k += kThreads) {
+                const double d = (double)__half2float(__ushort_as_half(dr[k]));
                 const long long di = __double2ll_rn(__dmul_rn(d, 16777216.0));  // exact: d is a multiple of 2^-24
                 int best = 0;
                 double bd = fabs(__dsub_rn(d, c[0]));
@@ -281,43 +305,67 @@ __global__ void __launch_bounds__(kThreads) kmeans_kernel(const uint16_t* __rest
 #pragma unroll
                 for (int j = 0; j < L; ++j)
                     if (best == j) {
-                        s[j] += di;
+                        sm[j] += di;
                         cnt[j] += 1;
                     }
             }
-            bool moved = false;
 #pragma unroll
             for (int j = 0; j < L; ++j) {
-                long long sj = s[j];
-                int cj = cnt[j];
                 for (int o = 16; o; o >>= 1) {
-                    sj += __shfl_xor_sync(0xffffffffu, sj, o);
-                    cj += __shfl_xor_sync(0xffffffffu, cj, o);
+                    sm[j] += __shfl_xor_sync(0xffffffffu, sm[j], o);
+                    cnt[j] += __shfl_xor_sync(0xffffffffu, cnt[j], o);
                 }
-                const double nc = cj ? __ddiv_rn(__dmul_rn((double)sj, 0x1p-24), (double)cj) : c[j];
-                moved |= nc != c[j];
-                c[j] = nc;
             }
+            if (lane == 0) {
+#pragma unroll
+                for (int j = 0; j < L; ++j) {
+                    s_sum[wid][j] = sm[j];
+                    s_cnt[wid][j] = cnt[j];
+                }
+            }
+            if (tid == 0) s_moved = 0;
+            __syncthreads();
+            if (tid < L) {
+                long long tot = 0;
+                int n = 0;
+#pragma unroll
+                for (int v = 0; v < NW; ++v) {
+                    tot += s_sum[v][tid];
+                    n += s_cnt[v][tid];
+                }
+                double cj = 0.0;
+#pragma unroll
+                for (int j = 0; j < L; ++j)
+                    if (j == tid) cj = c[j];
+                const double nc = n ? __ddiv_rn(__dmul_rn((double)tot, 0x1p-24), (double)n) : cj;
+                if (nc != cj) s_moved = 1;
+                s_c[tid] = nc;
+            }
+            __syncthreads();
+#pragma unroll
+            for (int j = 0; j < L; ++j) c[j] = s_c[j];
+            const bool moved = s_moved != 0;
+            __syncthreads();  // s_moved and the sums are rewritten next iteration
             if (!moved) {
                 ++it;
                 break;
             }
         }
-        if (iters_out && lane == 0) iters_out[i] = it;
+        if (iters_out && tid == 0) iters_out[i] = it;
         // the LUT and each weight's nearest entry
         double lv[L];
 #pragma unroll
         for (int j = 0; j < L; ++j) {
             const uint16_t hb = d2h_rne(c[j]);
             lv[j] = (double)__half2float(__ushort_as_half(hb));
-            if (lane == j) lut[i * L + j] = hb;
+            if (tid == j) lut[i * L + j] = hb;
         }
         uint32_t* cw = codes + i * wpr;
-        for (int64_t k0 = 0; k0 < k_in; k0 += 32) {
+        for (int64_t k0 = (int64_t)wid * 32; k0 < k_in; k0 += kThreads) {
             const int64_t k = k0 + lane;
             uint32_t code = 0;
             if (k < k_in) {
-                const double d = value(k);
+                const double d = (double)__half2float(__ushort_as_half(dr[k]));
                 double bd = fabs(__dsub_rn(d, lv[0]));
 #pragma unroll
                 for (int j = 1; j < L; ++j) {
@@ -537,11 +585,21 @@ SQZ_API sqz_status sqz_encode(const uint16_t* w, int32_t n_out, int32_t k_in, in
         ENC_TRY(cudaGetLastError(), "encode CSR");
     }
 
-    // ---- k-means per row, LUT and codes
-    if (bits == 3)
-        kmeans_kernel<3><<<warp_blocks, kThreads, 0, s>>>(w, d_flags, n_out, k_in, max_iters, codes, lut, iters_out);
-    else
-        kmeans_kernel<4><<<warp_blocks, kThreads, 0, s>>>(w, d_flags, n_out, k_in, max_iters, codes, lut, iters_out);
+    // ---- k-means per row, LUT and codes (one CTA per row, the row in shared memory)
+    const size_t smem = (size_t)k_in * 2;
+    if (smem > 200u * 1024u)
+        return enc_fail(SQZ_ERR_UNSUPPORTED, "sqz_encode: k_in = %d exceeds the %u columns a row stage holds", k_in,
+                        (200u * 1024u) / 2u);
+    const int kblocks = (int)std::min<int64_t>(n_out, 1 << 20);
+    if (bits == 3) {
+        ENC_TRY(cudaFuncSetAttribute(kmeans_kernel<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem),
+                "encode attributes");
+        kmeans_kernel<3><<<kblocks, kThreads, smem, s>>>(w, d_flags, n_out, k_in, max_iters, codes, lut, iters_out);
+    } else {
+        ENC_TRY(cudaFuncSetAttribute(kmeans_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem),
+                "encode attributes");
+        kmeans_kernel<4><<<kblocks, kThreads, smem, s>>>(w, d_flags, n_out, k_in, max_iters, codes, lut, iters_out);
+    }
     ENC_TRY(cudaGetLastError(), "encode k-means");
     ENC_TRY(cudaStreamSynchronize(s), "encode k-means");
     *nnz_out = 2 * m;
