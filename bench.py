@@ -57,6 +57,9 @@ def parse():
     p.add_argument("--seed", type=int, default=0)
     p.add_argument("--csr", choices=("balanced", "rowwise"), default="balanced",
                    help="sparse scheme of the fused kernel (rowwise: the plain CSR comparison)")
+    p.add_argument("--encode", action="store_true",
+                   help="time the encoder (sqz_encode) on synthetic weights of the workload's shape instead")
+    p.add_argument("--encode-iters", type=int, default=30, help="k-means iterations of --encode")
     p.add_argument("--profile-launches", type=int, default=0,
                    help="for profiler captures: one layer instance of the shape, this many plain launches, "
                         "no timing and no JSON line")
@@ -484,8 +487,64 @@ def run_profile_launches(args):
     return 0
 
 
+def run_encode(args):
+    """The encoder on one layer of the workload's shape: synthetic Student-t
+    fp16 weights, the shape's bits and outlier fraction; ms per layer on the
+    device (CUDA events, K timed calls after W warm-up calls) and the fp64
+    oracle on a bounded sample (the whole outlier split plus the k-means of
+    a few rows, scaled to the layer)."""
+    import torch
+
+    from lut_dequant_gemv_b200 import binding as B
+
+    B.lib()
+    shape = shape_for(args)
+    w_np = synth.make_weights(shape.n_out, shape.k_in, seed=args.seed, key=shape.key)
+    w = torch.from_numpy(w_np.view(np.int16).copy()).cuda()
+    frac = shape.density if shape.density > 0 else 0.0045
+    steps, warmup = max(1, min(args.steps, 20)), max(3, min(args.warmup, 5))
+    for _ in range(warmup):
+        out = B.sqz_encode(w, shape.bits, frac, args.encode_iters, want_iters=True)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        out = B.sqz_encode(w, shape.bits, frac, args.encode_iters, want_iters=True)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    iters = out[5].cpu().numpy()
+    n_w = shape.n_out * shape.k_in
+    line = {"metric": "encoder weights per second (Dense-and-Sparse split + per-row k-means)",
+            "value": n_w / (ms * 1e-3), "unit": "weights/s", "n_gpus": 1, "steps": steps, "warmup": warmup,
+            "ms_per_layer": ms, "higher_is_better": True, "dtype": "fp16 in, fp64 k-means, exact integer sums",
+            "data": "synthetic (0.02 x Student-t(4) weights)",
+            "config": {"workload": f"{shape.n_out}x{shape.k_in}, {shape.bits}-bit, outlier fraction {frac}",
+                       "kmeans_iters": args.encode_iters, "iters_mean": float(iters.mean()),
+                       "rows_at_iteration_limit": float((iters == args.encode_iters).mean())}}
+    if not args.no_cpu_baseline:
+        import oracle
+
+        orc = oracle.default()
+        rows = np.arange(8, dtype=np.int32)
+        t0 = time.perf_counter()
+        orc.encode(w_np.reshape(shape.n_out, shape.k_in), shape.bits, frac, args.encode_iters, rows=rows[:1])
+        t_split = time.perf_counter() - t0
+        t0 = time.perf_counter()
+        orc.encode(w_np.reshape(shape.n_out, shape.k_in), shape.bits, frac, args.encode_iters, rows=rows)
+        t_rows = max(time.perf_counter() - t0 - t_split, 1e-9) / (len(rows) - 1)
+        t_layer = t_split + t_rows * shape.n_out
+        line["cpu_baseline"] = {"value": n_w / t_layer, "unit": "weights/s", "cores": 1, "kind": "oracle",
+                                "sample": f"outlier split of the whole layer ({t_split:.1f} s) plus the k-means "
+                                          f"of 8 rows, scaled to {shape.n_out} rows ({t_layer:.0f} s per layer)"}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse()
+    if args.encode:
+        return run_encode(args)
     if args.profile_launches:
         return run_profile_launches(args)
     if args.impl == "reference":
