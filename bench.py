@@ -526,13 +526,17 @@ def run_encode(args):
         import oracle
 
         orc = oracle.default()
-        rows = np.arange(8, dtype=np.int32)
+        w2 = w_np.reshape(shape.n_out, shape.k_in)
+        m = orc.outliers_per_tail(w2.size, frac)
         t0 = time.perf_counter()
-        orc.encode(w_np.reshape(shape.n_out, shape.k_in), shape.bits, frac, args.encode_iters, rows=rows[:1])
+        marks = orc.select_outliers(w2, m)
         t_split = time.perf_counter() - t0
+        n_rows = 8
+        dense = np.where(marks[:n_rows] != 0, 0.0, w2[:n_rows].view(np.float16).astype(np.float64))
         t0 = time.perf_counter()
-        orc.encode(w_np.reshape(shape.n_out, shape.k_in), shape.bits, frac, args.encode_iters, rows=rows)
-        t_rows = max(time.perf_counter() - t0 - t_split, 1e-9) / (len(rows) - 1)
+        for r in range(n_rows):
+            orc.kmeans_row(dense[r], 1 << shape.bits, args.encode_iters)
+        t_rows = (time.perf_counter() - t0) / n_rows
         t_layer = t_split + t_rows * shape.n_out
         line["cpu_baseline"] = {"value": n_w / t_layer, "unit": "weights/s", "cores": 1, "kind": "oracle",
                                 "sample": f"outlier split of the whole layer ({t_split:.1f} s) plus the k-means "

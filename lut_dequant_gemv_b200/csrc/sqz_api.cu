@@ -287,10 +287,21 @@ sqz_status gemv_impl(const sqz_layer* L, const uint16_t* x, int32_t batch, int64
                      cudaStream_t s) {
     if (L->n_out == 0) return SQZ_OK;
     sqz::tc::Plan P;
-    // Columns per launch: the whole batch when its x fits in shared memory,
-    // else chunks of 8, 4, 2 or 1 columns (each launch reads the weights).
+    // Columns per launch: the whole batch when a plan exists for it, else
+    // chunks of 8, 4, 2 or 1 columns (each launch reads the weights).  A batch
+    // above 8 whose x fits only in several passes runs as launches of 8
+    // columns in one pass each when those fit: a pass gives each warp about
+    // one unit per tile, and the passes' barriers then cost more than
+    // decoding the weights twice.
     int chunk = batch;
     bool fits = L->fused_ok && fused_plan(L, chunk, &P);
+    if (fits && batch > 8 && P.passes > 1) {
+        sqz::tc::Plan P8;
+        if (fused_plan(L, 8, &P8) && P8.passes == 1) {
+            chunk = 8;
+            P = P8;
+        }
+    }
     while (L->fused_ok && !fits && chunk > 1) {
         chunk = chunk > 8 ? 8 : chunk / 2;
         fits = fused_plan(L, chunk, &P);
