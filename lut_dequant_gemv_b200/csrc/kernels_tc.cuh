@@ -89,8 +89,8 @@ constexpr int kMaxCtas = 512;     // CTAs per launch (one per SM)
 constexpr int kMinStages = 2;     // shared-memory stages per warp (units in flight + 1)
 constexpr int kMaxStages = 16;
 constexpr int kRingStages = 4;    // ring depth reserved before the CSR staging area
-constexpr int kSbStages = 4;      // batch 1: the ring depth, 4 stages (3 when 4 do not fit), so
-                                  // that the wait for a unit's copies is one of two fixed forms
+constexpr int kSbStages = 4;      // one pass over K: the ring depth, 4 stages (3 when 4 do not fit),
+                                  // so that the wait for a unit's copies is one of two fixed forms
 constexpr int kPreWait = 2;       // code units per warp requested before waiting for the previous kernel;
                                   // the rest of the first ring follows once x has landed
 constexpr int kCsrCap = 4096;     // CSR entries per CTA staged in shared memory, at most (more: read from global)
@@ -223,9 +223,10 @@ __host__ __device__ inline Plan make_plan(int bits, int n_out, int k_in, int bat
     // (up to kCsrCap entries; entries beyond it are read from global memory)
     // batch 1: a ring of kSbStages stages when it fits beside at least a
     // small CSR stage, else one stage less
+    const bool fixed = P.passes == 1;  // one pass: a ring of fixed depth (compile-time waits)
     int sb_stages = kSbStages;
-    if (single && budget - off - kSbStages * kWarps * sg_bytes - 512 < 6 * 256) sb_stages = kSbStages - 1;
-    const int ring_min = (single ? sb_stages : kRingStages) * kWarps * sg_bytes;
+    if (fixed && budget - off - kSbStages * kWarps * sg_bytes - 512 < 6 * 256) sb_stages = kSbStages - 1;
+    const int ring_min = (fixed ? sb_stages : kRingStages) * kWarps * sg_bytes;
     int cap = (budget - off - ring_min - 512) / 6;  // 4-byte column + 2-byte value per entry
     cap = cap > kCsrCap ? kCsrCap : cap;
     P.csr_cap = cap < 0 ? 0 : cap & ~7;
@@ -237,7 +238,7 @@ __host__ __device__ inline Plan make_plan(int bits, int n_out, int k_in, int bat
     int stages = (budget - off) / (kWarps * sg_bytes);
     if (stages > kMaxStages) stages = kMaxStages;
     if (stages < kMinStages) stages = kMinStages;
-    if (single) stages = sb_stages;
+    if (fixed) stages = sb_stages;
     P.stages = stages;
     off += stages * kWarps * sg_bytes;
     P.total = off;
@@ -1160,14 +1161,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_fused_kernel(const 
     int s_read = 0, s_fill = D;
 #pragma unroll 1
     for (int i = 0; i < nwu; ++i) {
-        if constexpr (SB) {
-            if (S == kSbStages)
-                cp_async_wait<kSbStages - 2>();
-            else
-                cp_async_wait<kSbStages - 3>();
-        } else {
-            cp_async_wait_newest(D - 1);
-        }
+        if (S == kSbStages)  // single-pass plans: 4 stages, or 3
+            cp_async_wait<kSbStages - 2>();
+        else
+            cp_async_wait<kSbStages - 3>();
         uint4 v[V];
         const uint8_t* src = ring + s_read * F::kSgBytes;
 #pragma unroll
