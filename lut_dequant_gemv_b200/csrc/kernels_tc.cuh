@@ -262,9 +262,11 @@ struct Params {
     uint16_t* y;
     int64_t ldy;
     int* status;             // error bits (bounded waits that gave up)
-    // CSR entries of the rows of CTA c: [csr_cta[c], csr_cta[c+1]); all zero
-    // when the layer has no outliers.
-    int32_t csr_cta[kMaxCtas + 1];
+    // CSR entries of the rows of CTA c: [csr_cta[c], csr_cta[c+1]) (device
+    // array of grid + 1 values; all zero when the layer has no outliers).  Kept
+    // out of the parameters: a small parameter block stays in the constant
+    // cache, whose misses cost hundreds of cycles wherever a field is reread.
+    const int32_t* csr_cta;
 };
 
 // ------------------------------------------------------------- PTX helpers
@@ -637,7 +639,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_fused_kernel(const 
         mbar_expect_tx(lbar, lut_bytes + rp_bytes);
         bulk_g2s(luts, p.lutp + (int64_t)t_first * kTileRows * F::kLutBytes, lut_bytes, lbar);
         if (rp_bytes) bulk_g2s(smem + P.off_rp, p.rowptr + (ra - rp_off), rp_bytes, lbar);
-        const int q0 = p.csr_cta[c], nz = p.csr_cta[c + 1] - q0;
+        const int q0 = __ldg(p.csr_cta + c), nz = __ldg(p.csr_cta + c + 1) - q0;
         const bool csr_in_smem = nz > 0 && nz <= P.csr_cap;
         const uint32_t col_bytes = csr_in_smem ? (uint32_t)round_up(nz + (q0 & 3), 4) * 4 : 0u;
         const uint32_t val_bytes = csr_in_smem ? (uint32_t)round_up(nz + (q0 & 7), 8) * 2 : 0u;
@@ -727,7 +729,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_fused_kernel(const 
     __syncthreads();
 
     // ---- the CTA's CSR entries [q0, q1), a fixed share e_per per thread
-    const int q0 = p.csr_cta[c], q1 = p.csr_cta[c + 1];
+    const int q0 = __ldg(p.csr_cta + c), q1 = __ldg(p.csr_cta + c + 1);
     const int nz = q1 - q0;
     const bool has_csr = nz > 0;
     const bool csr_in_smem = has_csr && nz <= P.csr_cap;
@@ -763,7 +765,18 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_fused_kernel(const 
         }
     }
 
-    // ---- x may be written by the previous kernel of the stream: wait for it
+    // ---- x may be written by the previous kernel of the stream: wait for it.
+    // Before that, warp 1 asks L2 for x's lines (a hint that returns nothing:
+    // a line the previous kernel writes later is updated in L2, so the copy
+    // after the wait reads the new values either way), which hides the DRAM
+    // latency when x was written earlier.
+    if (warp == 1) {
+        const int lines = (p.k_in * 2 + 127) / 128;
+        for (int b = 0; b < B; ++b) {
+            const char* xr = reinterpret_cast<const char*>(p.x + b * p.ldx);
+            for (int l = lane; l < lines; l += 32) asm volatile("prefetch.global.L2 [%0];" ::"l"(xr + l * 128));
+        }
+    }
     pdl_wait_previous();
     // x chunk q into buffer q % 2: bulk copies issued by thread 0 (x rows
     // 16-byte aligned), or copied by all threads (then a barrier follows)

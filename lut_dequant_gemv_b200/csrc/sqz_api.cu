@@ -91,7 +91,7 @@ struct sqz_layer {
     int ntiles = 0, nsteps = 0, nsg = 0;
     int64_t units = 0;
     int grid = 0;                     // CTAs of a fused launch (one per SM)
-    std::vector<int32_t> csr_cta;     // [grid + 1]: CSR entry range of each CTA's rows
+    int32_t* csr_cta = nullptr;       // [grid + 1] (device): CSR entry range of each CTA's rows
     uint8_t* codes_native = nullptr;  // [ntiles][nsg][sg_bytes]
     uint8_t* lut_native = nullptr;    // [ntiles*16][2 << bits] byte planes
     int* status = nullptr;            // [1]
@@ -112,6 +112,7 @@ void free_layer(sqz_layer* L) {
     cudaFree(L->codes_native);
     cudaFree(L->lut_native);
     cudaFree(L->status);
+    cudaFree(L->csr_cta);
     cudaFree(L->x_stage);
     cudaFree(L->y_stage);
     delete L;
@@ -330,7 +331,7 @@ sqz_status gemv_impl(const sqz_layer* L, const uint16_t* x, int32_t batch, int64
             prm.has_csr = L->nnz > 0;
             prm.x_bulk = (reinterpret_cast<uintptr_t>(xc) % 16 == 0) && (ldx % 8 == 0) && (L->k_in % 8 == 0);
             prm.plan = P;
-            std::memcpy(prm.csr_cta, L->csr_cta.data(), sizeof(int32_t) * L->csr_cta.size());
+            prm.csr_cta = L->csr_cta;
             const cudaError_t e = L->bits == 3 ? launch_fused_bits<3>(prm, nb, L->mac, L->csr_mode, s)
                                                : launch_fused_bits<4>(prm, nb, L->mac, L->csr_mode, s);
             SQZ_CUDA_TRY(e, "fused gemv launch");
@@ -380,19 +381,14 @@ sqz_status build_native(sqz_layer* L, cudaStream_t s) {
             sqz::tc::repack_lut_kernel<4><<<blocks, 256, 0, s>>>(L->lut, L->n_out, rows, L->lut_native);
         SQZ_CUDA_TRY(cudaGetLastError(), "repack lut");
     }
-    // CSR entry range of every CTA's rows, passed with each launch
-    L->csr_cta.assign((size_t)L->grid + 1, 0);
+    // CSR entry range of every CTA's rows (device array read by each launch)
+    if ((st = alloc(&L->csr_cta, (size_t)L->grid + 1, L, "CTA bounds")) != SQZ_OK) return st;
     if (L->nnz > 0) {
         if (L->grid > kMaxCtas) return fail(SQZ_ERR_UNSUPPORTED, "%d CTAs exceed the fused kernel's %d", L->grid, kMaxCtas);
-        int32_t* d_b = nullptr;
-        SQZ_CUDA_TRY(cudaMalloc(&d_b, sizeof(int32_t) * (L->grid + 1)), "CTA bounds allocation");
-        csr_cta_bounds_kernel<<<(L->grid + 256) / 256, 256, 0, s>>>(L->rowptr, L->n_out, L->ntiles, L->grid, d_b);
-        cudaError_t e = cudaGetLastError();
-        if (e == cudaSuccess)
-            e = cudaMemcpyAsync(L->csr_cta.data(), d_b, sizeof(int32_t) * (L->grid + 1), cudaMemcpyDeviceToHost, s);
-        if (e == cudaSuccess) e = cudaStreamSynchronize(s);
-        cudaFree(d_b);
-        SQZ_CUDA_TRY(e, "CTA bounds");
+        csr_cta_bounds_kernel<<<(L->grid + 256) / 256, 256, 0, s>>>(L->rowptr, L->n_out, L->ntiles, L->grid, L->csr_cta);
+        SQZ_CUDA_TRY(cudaGetLastError(), "CTA bounds");
+    } else {
+        SQZ_CUDA_TRY(cudaMemsetAsync(L->csr_cta, 0, sizeof(int32_t) * ((size_t)L->grid + 1), s), "memset");
     }
     return SQZ_OK;
 }
