@@ -1199,6 +1199,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_fused_kernel(const 
     // warps' parts are added in warp order (the same order for every batch
     // size) and the rows get their sparse sums.
     __syncthreads();
+    csr_ready = true;  // every sparse share was written before this barrier
     for (int idx = tid; idx < ctiles * TE; idx += kThreads) {
         const int tl = idx / TE, e = idx - tl * TE;
         const int mask = s_tinfo[tl];
