@@ -517,16 +517,25 @@ sqz_status sqz_gemv_host(sqz_layer_t layer, const uint16_t* x_host, int32_t batc
     if (st != SQZ_OK) return st;
     cudaStream_t s = as_stream(stream);
     const sqz_layer* L = layer;
-    if (L->k_in > 0)
-        SQZ_CUDA_TRY(cudaMemcpy2DAsync(L->x_stage, (size_t)L->k_in * 2, x_host, (size_t)ldx * 2, (size_t)L->k_in * 2,
-                                       (size_t)batch, cudaMemcpyHostToDevice, s),
-                     "x host-to-device copy");
+    // one flat copy each way when the rows are packed (a 2-D copy otherwise)
+    if (L->k_in > 0) {
+        const size_t row = (size_t)L->k_in * 2;
+        const cudaError_t e = (ldx == L->k_in || batch == 1)
+                                  ? cudaMemcpyAsync(L->x_stage, x_host, row * batch, cudaMemcpyHostToDevice, s)
+                                  : cudaMemcpy2DAsync(L->x_stage, row, x_host, (size_t)ldx * 2, row, (size_t)batch,
+                                                      cudaMemcpyHostToDevice, s);
+        SQZ_CUDA_TRY(e, "x host-to-device copy");
+    }
     st = gemv_impl(L, L->x_stage, batch, L->k_in, L->y_stage, L->n_out, s);
     if (st != SQZ_OK) return st;
-    if (L->n_out > 0)
-        SQZ_CUDA_TRY(cudaMemcpy2DAsync(y_host, (size_t)ldy * 2, L->y_stage, (size_t)L->n_out * 2, (size_t)L->n_out * 2,
-                                       (size_t)batch, cudaMemcpyDeviceToHost, s),
-                     "y device-to-host copy");
+    if (L->n_out > 0) {
+        const size_t row = (size_t)L->n_out * 2;
+        const cudaError_t e = (ldy == L->n_out || batch == 1)
+                                  ? cudaMemcpyAsync(y_host, L->y_stage, row * batch, cudaMemcpyDeviceToHost, s)
+                                  : cudaMemcpy2DAsync(y_host, (size_t)ldy * 2, L->y_stage, row, row, (size_t)batch,
+                                                      cudaMemcpyDeviceToHost, s);
+        SQZ_CUDA_TRY(e, "y device-to-host copy");
+    }
     SQZ_CUDA_TRY(cudaStreamSynchronize(s), "stream synchronize");
     return SQZ_OK;
 }
