@@ -75,6 +75,31 @@ def dist_env():
     return world, rank, local
 
 
+def instance_id(rank: int, i: int) -> int:
+    """Layer instance i of a rank: every rank owns its own layers (replicas
+    of the workload, no shared data and no data-path collective)."""
+    return rank * 1000 + i
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """The slowest rank's time: an all-reduce MAX of one float (NCCL on the
+    GPU run, gloo on CPU); the value itself when there is one rank."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_gbs(world: int, bytes_per_step: int, steps: int, ms: float) -> float:
+    """Whole-job throughput: every rank processes bytes_per_step per step,
+    and the job takes the slowest rank's ms."""
+    return world * bytes_per_step * steps / (ms / 1e3) / 1e9
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -278,17 +303,18 @@ def run_ours(args):
 
     shape = shape_for(args)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    L0 = synth.layer_for(shape, seed=args.seed, instance=rank * 1000)
+    L0 = synth.layer_for(shape, seed=args.seed, instance=instance_id(rank, 0))
     inst_bytes = L0.nbytes()
     instances = max(2, math.ceil(4 * l2 / inst_bytes))
     layers, xs, ys = [], [], []
     for i in range(instances):
-        L = L0 if i == 0 else synth.layer_for(shape, seed=args.seed, instance=rank * 1000 + i)
+        L = L0 if i == 0 else synth.layer_for(shape, seed=args.seed, instance=instance_id(rank, i))
         layers.append(B.create_layer_from_numpy(L.n_out, L.k_in, L.bits, L.codes, L.lut, L.rowptr, L.col, L.val,
                                                 device=dev))
         if args.csr == "rowwise":
             B.sqz_layer_set_csr_mode(layers[-1], B.SQZ_CSR_ROWWISE)
-        xs.append(torch.from_numpy(synth.x_for(shape, seed=args.seed, instance=rank * 1000 + i).view(np.int16)).to(dev))
+        xs.append(torch.from_numpy(synth.x_for(shape, seed=args.seed, instance=instance_id(rank, i)).view(np.int16))
+                  .to(dev))
         ys.append(torch.empty((shape.batch, shape.n_out), dtype=torch.int16, device=dev))
     nnz = L0.nnz
     bytes_per_step = acc.gemv_bytes(shape.n_out, shape.k_in, shape.bits, nnz, shape.batch)
@@ -341,17 +367,13 @@ def run_ours(args):
         torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
-    ms = ev0.elapsed_time(ev1)
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
     ms_per_step = ms / args.steps
-    value = world * bytes_per_step * args.steps / (ms / 1e3) / 1e9
+    value = whole_job_gbs(world, bytes_per_step, args.steps, ms)
     per_launch_gbs = bytes_per_step / (ms_per_step / 1e3) / 1e9
 
     # ---- end to end through the host entry point (pinned buffers)
-    xh = [torch.from_numpy(synth.x_for(shape, seed=args.seed, instance=rank * 1000 + i).view(np.int16).copy())
+    xh = [torch.from_numpy(synth.x_for(shape, seed=args.seed, instance=instance_id(rank, i)).view(np.int16).copy())
           .pin_memory() for i in range(instances)]
     yh = torch.empty((shape.batch, shape.n_out), dtype=torch.int16).pin_memory()
     e2e_steps = min(args.steps, 20000)
@@ -367,12 +389,8 @@ def run_ours(args):
             B.sqz_gemv_host(layers[j % instances], xh[j % instances], yh, stream=stream)
         e1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * bytes_per_step * e2e_steps / (e2e_ms / 1e3) / 1e9
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    e2e_value = whole_job_gbs(world, bytes_per_step, e2e_steps, e2e_ms)
 
     # ---- fp16 dense yardstick (same shape, uncompressed weights)
     yard = None
