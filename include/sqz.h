@@ -191,6 +191,28 @@ SQZ_API sqz_status sqz_layer_status(sqz_layer_t layer, void* stream, int32_t* st
 SQZ_API sqz_status sqz_layer_info(sqz_layer_t layer, int32_t* n_out, int32_t* k_in, int32_t* bits, int64_t* nnz,
                           int64_t* device_bytes);
 
+/*
+ * The launch plan sqz_gemv would use for a layer shape and batch on a device
+ * with the given SM count and shared memory (per SM, and the opt-in maximum
+ * of one CTA) -- computed on the host, no device needed.  fused = 0 means the
+ * row-per-warp kernel serves the call (all other fields 0).  Otherwise the
+ * batch runs as `launches` launches of up to columns_per_launch columns,
+ * each a grid of `grid` CTAs of `threads` threads with smem_bytes of dynamic
+ * shared memory (ctas_per_sm = 2 when two CTAs share an SM), x staged in
+ * `passes` chunks of K, a code ring of ring_stages stages per warp and up to
+ * csr_stage_entries outliers per CTA staged in shared memory (the first
+ * launch's plan; a shorter last launch may differ).  No counterpart in the
+ * paper: it exposes this library's own scheduling.
+ * Errors: SQZ_ERR_INVALID_ARG for a NULL out, bits not in {3,4}, n_out or k_in
+ * < 1, batch outside [1,16], or a non-positive device figure.
+ */
+typedef struct {
+    int32_t fused, columns_per_launch, launches, grid, threads, ctas_per_sm, smem_bytes, passes, ring_stages,
+        csr_stage_entries;
+} sqz_plan_info;
+SQZ_API sqz_status sqz_plan_query(int32_t n_out, int32_t k_in, int32_t bits, int32_t batch, int32_t sm_count,
+                                  int32_t smem_per_sm, int32_t smem_optin, sqz_plan_info* out);
+
 /* Release a handle and its device memory.  NULL is accepted.  The caller
  * must make sure no work that uses the handle is still in flight. */
 SQZ_API sqz_status sqz_destroy(sqz_layer_t layer);

@@ -38,13 +38,19 @@ STATUS_NAMES = {0: "SQZ_OK", 1: "SQZ_ERR_INVALID_ARG", 2: "SQZ_ERR_UNSUPPORTED",
 EXPORTED = ("sqz_create_layer", "sqz_gemv", "sqz_gemv_host", "sqz_debug_dequant", "sqz_layer_info",
             "sqz_destroy", "sqz_fp16_gemv", "sqz_last_error", "sqz_version", "sqz_check_csr_static",
             "sqz_layer_set_mac", "sqz_layer_set_csr_mode", "sqz_layer_status", "sqz_encode",
-            "sqz_encode_outliers")
+            "sqz_encode_outliers", "sqz_plan_query")
 
 
 class SqzError(RuntimeError):
     def __init__(self, status: int, where: str, message: str):
         super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}: {message}")
         self.status = status
+
+
+class sqz_plan_info(ctypes.Structure):
+    _fields_ = [(name, ctypes.c_int32) for name in (
+        "fused", "columns_per_launch", "launches", "grid", "threads", "ctas_per_sm", "smem_bytes", "passes",
+        "ring_stages", "csr_stage_entries")]
 
 
 class sqz_layer_desc(ctypes.Structure):
@@ -94,6 +100,8 @@ def lib() -> ctypes.CDLL:
         L.sqz_encode.argtypes = [P, i32, i32, i32, ctypes.c_double, i32, P, P, P, P, P, i64,
                                  ctypes.POINTER(i64), P, P]
         L.sqz_encode.restype = ctypes.c_int
+        L.sqz_plan_query.argtypes = [i32, i32, i32, i32, i32, i32, i32, ctypes.POINTER(sqz_plan_info)]
+        L.sqz_plan_query.restype = ctypes.c_int
         L.sqz_encode_outliers.argtypes = [i64, ctypes.c_double]
         L.sqz_encode_outliers.restype = i64
         L.sqz_last_error.argtypes = []
@@ -295,6 +303,18 @@ def sqz_check_csr_static(rowptr: Optional[torch.Tensor], col: Optional[torch.Ten
                                       n_out, k_in, nnz, _stream(stream), ctypes.byref(flags)),
            "sqz_check_csr_static")
     return int(flags.value)
+
+
+B200_DEVICE = {"sm_count": 148, "smem_per_sm": 233472, "smem_optin": 232448}
+
+
+def sqz_plan_query(n_out: int, k_in: int, bits: int, batch: int, sm_count: int = 148, smem_per_sm: int = 233472,
+                   smem_optin: int = 232448) -> dict:
+    """The launch plan sqz_gemv would use (host computation; defaults: B200)."""
+    info = sqz_plan_info()
+    _check(lib().sqz_plan_query(n_out, k_in, bits, batch, sm_count, smem_per_sm, smem_optin, ctypes.byref(info)),
+           "sqz_plan_query")
+    return {name: int(getattr(info, name)) for name, _ in sqz_plan_info._fields_}
 
 
 def sqz_encode_outliers(n_weights: int, outlier_fraction: float) -> int:

@@ -217,11 +217,19 @@ sqz_status prepare_fused_kernels(int optin) {
 // stream its weights while this one computes); one whose x does not fit
 // there gets a whole SM; a batch whose x does not fit at all is staged in K
 // chunks (several passes, fewest first).
-bool fused_plan(const sqz_layer* L, int batch, sqz::tc::Plan* out) {
+// The device's side of a plan: SMs, the shared memory of one CTA when two
+// share an SM, and the opt-in maximum of one CTA.
+struct DeviceShape {
+    int sm_count, smem_half, smem_optin;
+};
+
+bool plan_for(int bits, int n_out, int k_in, const DeviceShape& d, int batch, sqz::tc::Plan* out) {
     const int nt = batch > 8 ? 2 : 1;
-    for (int budget : {L->smem_budget, L->smem_optin}) {
-        sqz::tc::Plan P = sqz::tc::make_plan(L->bits, L->n_out, L->k_in, batch, nt, batch == 1, L->sm_count, budget);
-        if (P.total <= budget && P.grid == L->grid) {
+    const int grid = sqz::tc::grid_size(n_out, d.sm_count);
+    const int nsg = ((k_in + 15) / 16 + sqz::tc::kSgSteps - 1) / sqz::tc::kSgSteps;
+    for (int budget : {d.smem_half, d.smem_optin}) {
+        sqz::tc::Plan P = sqz::tc::make_plan(bits, n_out, k_in, batch, nt, batch == 1, d.sm_count, budget);
+        if (P.total <= budget && P.grid == grid) {
             *out = P;
             return true;
         }
@@ -230,10 +238,10 @@ bool fused_plan(const sqz_layer* L, int batch, sqz::tc::Plan* out) {
         // fewest passes that still leave a ring of 4 stages per warp, else the
         // fewest passes that fit at all
         bool have = false;
-        for (int passes = 2; passes <= L->nsg; ++passes) {
+        for (int passes = 2; passes <= nsg; ++passes) {
             sqz::tc::Plan P =
-                sqz::tc::make_plan(L->bits, L->n_out, L->k_in, batch, nt, false, L->sm_count, L->smem_optin, passes);
-            if (P.passes != passes || P.total > L->smem_optin || P.grid != L->grid) continue;
+                sqz::tc::make_plan(bits, n_out, k_in, batch, nt, false, d.sm_count, d.smem_optin, passes);
+            if (P.passes != passes || P.total > d.smem_optin || P.grid != grid) continue;
             if (!have) {
                 *out = P;
                 have = true;
@@ -246,6 +254,34 @@ bool fused_plan(const sqz_layer* L, int batch, sqz::tc::Plan* out) {
         return have;
     }
     return false;
+}
+
+bool fused_plan(const sqz_layer* L, int batch, sqz::tc::Plan* out) {
+    return plan_for(L->bits, L->n_out, L->k_in, DeviceShape{L->sm_count, L->smem_budget, L->smem_optin}, batch, out);
+}
+
+// Columns per launch and the plan of the first launch: the whole batch when
+// a plan exists for it, else chunks of 8, 4, 2 or 1 columns (each launch
+// reads the weights).  A batch above 8 whose x fits only in several passes
+// runs as launches of 8 columns in one pass each when those fit: a pass
+// gives each warp about one unit per tile, and the passes' barriers then
+// cost more than decoding the weights twice.  Returns 0 when no fused plan
+// exists (the row-per-warp kernel serves the call).
+int launch_columns(int bits, int n_out, int k_in, const DeviceShape& d, int batch, sqz::tc::Plan* P) {
+    int chunk = batch;
+    bool fits = plan_for(bits, n_out, k_in, d, chunk, P);
+    if (fits && batch > 8 && P->passes > 1) {
+        sqz::tc::Plan P8;
+        if (plan_for(bits, n_out, k_in, d, 8, &P8) && P8.passes == 1) {
+            chunk = 8;
+            *P = P8;
+        }
+    }
+    while (!fits && chunk > 1) {
+        chunk = chunk > 8 ? 8 : chunk / 2;
+        fits = plan_for(bits, n_out, k_in, d, chunk, P);
+    }
+    return fits ? chunk : 0;
 }
 
 // Launch with programmatic stream serialization: the kernel may start while
@@ -288,25 +324,10 @@ sqz_status gemv_impl(const sqz_layer* L, const uint16_t* x, int32_t batch, int64
                      cudaStream_t s) {
     if (L->n_out == 0) return SQZ_OK;
     sqz::tc::Plan P;
-    // Columns per launch: the whole batch when a plan exists for it, else
-    // chunks of 8, 4, 2 or 1 columns (each launch reads the weights).  A batch
-    // above 8 whose x fits only in several passes runs as launches of 8
-    // columns in one pass each when those fit: a pass gives each warp about
-    // one unit per tile, and the passes' barriers then cost more than
-    // decoding the weights twice.
-    int chunk = batch;
-    bool fits = L->fused_ok && fused_plan(L, chunk, &P);
-    if (fits && batch > 8 && P.passes > 1) {
-        sqz::tc::Plan P8;
-        if (fused_plan(L, 8, &P8) && P8.passes == 1) {
-            chunk = 8;
-            P = P8;
-        }
-    }
-    while (L->fused_ok && !fits && chunk > 1) {
-        chunk = chunk > 8 ? 8 : chunk / 2;
-        fits = fused_plan(L, chunk, &P);
-    }
+    const int chunk = L->fused_ok ? launch_columns(L->bits, L->n_out, L->k_in,
+                                                   DeviceShape{L->sm_count, L->smem_budget, L->smem_optin}, batch, &P)
+                                  : 0;
+    const bool fits = chunk > 0;
     if (fits) {
         for (int b0 = 0; b0 < batch; b0 += chunk) {
             const int nb = batch - b0 < chunk ? batch - b0 : chunk;
@@ -537,6 +558,34 @@ sqz_status sqz_gemv_host(sqz_layer_t layer, const uint16_t* x_host, int32_t batc
         SQZ_CUDA_TRY(e, "y device-to-host copy");
     }
     SQZ_CUDA_TRY(cudaStreamSynchronize(s), "stream synchronize");
+    return SQZ_OK;
+}
+
+sqz_status sqz_plan_query(int32_t n_out, int32_t k_in, int32_t bits, int32_t batch, int32_t sm_count,
+                          int32_t smem_per_sm, int32_t smem_optin, sqz_plan_info* out) {
+    if (!out) return fail(SQZ_ERR_INVALID_ARG, "out is NULL");
+    *out = sqz_plan_info{};
+    if (bits != 3 && bits != 4) return fail(SQZ_ERR_INVALID_ARG, "bits must be 3 or 4 (got %d)", bits);
+    if (n_out < 1 || k_in < 1) return fail(SQZ_ERR_INVALID_ARG, "n_out and k_in must be positive");
+    if (batch < 1 || batch > SQZ_MAX_BATCH) return fail(SQZ_ERR_INVALID_ARG, "batch must lie in [1, %d]", SQZ_MAX_BATCH);
+    if (sm_count < 1 || smem_per_sm < 1 || smem_optin < 1)
+        return fail(SQZ_ERR_INVALID_ARG, "sm_count, smem_per_sm and smem_optin must be positive");
+    const int share = smem_per_sm / sqz::tc::kCtasPerSm - 1024;
+    const DeviceShape d{sm_count, share < smem_optin ? share : smem_optin, smem_optin};
+    const int grid = sqz::tc::grid_size(n_out, sm_count);
+    sqz::tc::Plan P{};
+    const int chunk = grid <= sqz::tc::kMaxCtas ? launch_columns(bits, n_out, k_in, d, batch, &P) : 0;
+    if (chunk == 0) return SQZ_OK;  // fused = 0: the row-per-warp kernel
+    out->fused = 1;
+    out->columns_per_launch = chunk;
+    out->launches = (batch + chunk - 1) / chunk;
+    out->grid = P.grid;
+    out->threads = sqz::tc::kThreads;
+    out->smem_bytes = P.total;
+    out->ctas_per_sm = P.total <= d.smem_half ? sqz::tc::kCtasPerSm : 1;
+    out->passes = P.passes;
+    out->ring_stages = P.stages;
+    out->csr_stage_entries = P.csr_cap;
     return SQZ_OK;
 }
 

@@ -1,0 +1,68 @@
+"""The launch plan (host logic, no GPU): for every workload shape and every
+batch size the fused kernel serves the call with a plan that fits the
+shared memory it claims, single-pass launches use the fixed 3- or 4-stage
+code ring (the kernel's compile-time waits depend on it), and batches above
+8 run as one-pass launches of 8 columns when those fit while the whole
+batch would need several passes."""
+import pytest
+
+import synth
+from lut_dequant_gemv_b200 import binding as B
+
+DEV = B.B200_DEVICE
+HALF = DEV["smem_per_sm"] // 2 - 1024
+
+
+def shapes():
+    seen = set()
+    for name, ss in synth.workloads().items():
+        for s in ss:
+            if (s.n_out, s.k_in, s.bits) not in seen:
+                seen.add((s.n_out, s.k_in, s.bits))
+                yield s
+
+
+@pytest.mark.parametrize("shape", list(shapes()), ids=lambda s: f"{s.n_out}x{s.k_in}b{s.bits}")
+def test_every_batch_gets_a_fitting_fused_plan(shape):
+    for batch in range(1, 17):
+        p = B.sqz_plan_query(shape.n_out, shape.k_in, shape.bits, batch, **DEV)
+        assert p["fused"] == 1, (shape.key, batch)
+        assert p["grid"] == min(DEV["sm_count"], (shape.n_out + 15) // 16)
+        assert p["threads"] == 384
+        budget = HALF if p["ctas_per_sm"] == 2 else DEV["smem_optin"]
+        assert 0 < p["smem_bytes"] <= budget
+        assert p["launches"] * p["columns_per_launch"] >= batch
+        assert (p["launches"] - 1) * p["columns_per_launch"] < batch
+        if p["passes"] == 1:
+            assert p["ring_stages"] in (3, 4)
+        else:
+            assert p["ring_stages"] >= 2
+        if batch == 1:
+            assert p["passes"] == 1 and p["launches"] == 1
+            assert p["ctas_per_sm"] == 2, "batch 1 must leave room for the next call's CTA"
+        assert p["csr_stage_entries"] >= 0 and p["csr_stage_entries"] % 8 == 0
+
+
+def test_large_batches_split_into_single_pass_launches_of_eight():
+    # whole batch of 16 would need passes, 8 columns fit one pass: two launches
+    for n, k in ((5120, 5120), (13824, 5120), (4096, 4096)):
+        p = B.sqz_plan_query(n, k, 3, 16, **DEV)
+        assert (p["launches"], p["columns_per_launch"], p["passes"]) == (2, 8, 1), (n, k, p)
+    # 8 columns of K = 13824 do not fit one pass: one launch of 16 in several passes
+    p = B.sqz_plan_query(5120, 13824, 3, 16, **DEV)
+    assert p["launches"] == 1 and p["passes"] > 1
+
+
+def test_plan_query_rejects_bad_arguments():
+    for args in ((0, 64, 3, 1), (64, 64, 5, 1), (64, 64, 3, 0), (64, 64, 3, 17)):
+        with pytest.raises(B.SqzError) as e:
+            B.sqz_plan_query(*args, **DEV)
+        assert e.value.status == B.SQZ_ERR_INVALID_ARG
+    with pytest.raises(B.SqzError):
+        B.sqz_plan_query(64, 64, 3, 1, sm_count=0)
+
+
+def test_very_long_rows_fall_back_to_the_row_kernel():
+    # one batch column of x beyond the shared memory of a CTA
+    p = B.sqz_plan_query(64, 1 << 17, 4, 1, **DEV)
+    assert p["fused"] == 0 and p["launches"] == 0
