@@ -888,10 +888,37 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_fused_kernel(const 
             for (int b = 0; b < CM; ++b) s_rowsum[i * CM + b] = acc[b];
         }
     }
+    // Balanced mode: once every share is written (a barrier of the CT sparse
+    // threads), each row's interior sum and the pieces of the threads whose
+    // shares cut it are added, in thread order, into s_rowsum -- so a row's
+    // sparse sum is one shared-memory read wherever y is written.
+    if (!RW && has_csr && tid < CT) {
+        asm volatile("bar.sync 1, %0;" ::"n"(CT) : "memory");
+        for (int i = tid; i < nrows; i += CT) {
+            const int rs = s_rp[i], re = s_rp[i + 1];
+            if (re <= rs) continue;
+            float cs[CM];
+#pragma unroll
+            for (int b = 0; b < CM; ++b) cs[b] = s_rowsum[i * CM + b];
+            const int tau_a = (rs - q0) / e_per, tau_b = min(CT - 1, (re - 1 - q0) / e_per);
+            for (int tau = tau_a; tau <= tau_b; ++tau) {
+                if (s_headrow[tau] == i) {
+#pragma unroll
+                    for (int b = 0; b < CM; ++b) cs[b] += s_head[tau * CM + b];
+                }
+                if (s_tailrow[tau] == i) {
+#pragma unroll
+                    for (int b = 0; b < CM; ++b) cs[b] += s_tail[tau * CM + b];
+                }
+            }
+#pragma unroll
+            for (int b = 0; b < CM; ++b) s_rowsum[i * CM + b] = cs[b];
+        }
+    }
     if (has_csr && tid < CT) mbar_arrive(rbar);
 
-    // The sparse sum of row ra+i, batch column col: the interior sum, then
-    // the pieces of the threads whose shares cut the row, in thread order.
+    // The sparse sum of row ra+i, batch column col (complete once rbar's
+    // first phase has completed).
     bool csr_ready = !has_csr;
     auto csr_row_sum = [&](int i, int col) -> float {
         if (!has_csr) return 0.f;
@@ -899,16 +926,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_fused_kernel(const 
             if (!mbar_wait(rbar, 0)) atomicOr(p.status, kStatusWaitTimeout);
             csr_ready = true;
         }
-        const int rs = s_rp[i], re = s_rp[i + 1];
-        float cs = s_rowsum[i * CM + col];
-        if (re > rs) {
-            const int tau_a = (rs - q0) / e_per, tau_b = min(CT - 1, (re - 1 - q0) / e_per);
-            for (int tau = tau_a; tau <= tau_b; ++tau) {
-                if (s_headrow[tau] == i) cs += s_head[tau * CM + col];
-                if (s_tailrow[tau] == i) cs += s_tail[tau * CM + col];
-            }
-        }
-        return cs;
+        return s_rowsum[i * CM + col];
     };
 
     // ---- dense part
