@@ -128,8 +128,13 @@ SQZ_API sqz_status sqz_gemv(sqz_layer_t layer, const uint16_t* x, int32_t batch,
  * copies x (host, [batch][ldx]) to the handle's device staging buffer,
  * runs sqz_gemv, copies y back to host memory ([batch][ldy]) and
  * synchronises `stream` before returning.  Pinned host buffers give
- * asynchronous copies; pageable ones work but copy synchronously.
- * Errors as sqz_gemv.
+ * asynchronous copies; pageable ones work but copy synchronously.  With
+ * pinned buffers on a created (non-default) stream, the copy-in, product
+ * and copy-out are captured as a CUDA graph on first use and replayed by
+ * later calls with the same buffers, shape and stream (up to 64 per handle,
+ * least recently used dropped; released by sqz_destroy and by a change of
+ * the handle's MAC unit or CSR mode).  Not thread-safe against other calls
+ * on the same handle.  Errors as sqz_gemv.
  */
 SQZ_API sqz_status sqz_gemv_host(sqz_layer_t layer, const uint16_t* x_host, int32_t batch, int64_t ldx,
                          uint16_t* y_host, int64_t ldy, void* stream);

@@ -97,13 +97,32 @@ struct sqz_layer {
     int* status = nullptr;            // [1]
     uint16_t* x_stage = nullptr;      // [SQZ_MAX_BATCH][k_in] for sqz_gemv_host
     uint16_t* y_stage = nullptr;      // [SQZ_MAX_BATCH][n_out]
+    // sqz_gemv_host: copy-in, product and copy-out captured once per (host
+    // buffers, shape, stream) and replayed as one graph launch
+    struct HostGraph {
+        const void* x;
+        void* y;
+        int32_t batch;
+        int64_t ldx, ldy;
+        cudaStream_t stream;
+        cudaGraphExec_t exec;
+        uint64_t used;
+    };
+    std::vector<HostGraph> host_graphs;
+    uint64_t host_clock = 0;
     int64_t device_bytes = 0;
 };
 
 namespace {
 
+void drop_host_graphs(sqz_layer* L) {
+    for (auto& g : L->host_graphs) cudaGraphExecDestroy(g.exec);
+    L->host_graphs.clear();
+}
+
 void free_layer(sqz_layer* L) {
     if (!L) return;
+    drop_host_graphs(L);
     cudaFree(L->codes);
     cudaFree(L->lut);
     cudaFree(L->rowptr);
@@ -532,12 +551,14 @@ sqz_status sqz_gemv(sqz_layer_t layer, const uint16_t* x, int32_t batch, int64_t
     return gemv_impl(layer, x, batch, ldx, y, ldy, as_stream(stream));
 }
 
-sqz_status sqz_gemv_host(sqz_layer_t layer, const uint16_t* x_host, int32_t batch, int64_t ldx, uint16_t* y_host,
-                         int64_t ldy, void* stream) {
-    sqz_status st = check_gemv_args(layer, x_host, batch, ldx, y_host, ldy);
-    if (st != SQZ_OK) return st;
-    cudaStream_t s = as_stream(stream);
-    const sqz_layer* L = layer;
+}  // extern "C"
+
+namespace {
+
+// Copy x in, run the product, copy y out, all on stream s.
+sqz_status enqueue_host_call(const sqz_layer* L, const uint16_t* x_host, int32_t batch, int64_t ldx, uint16_t* y_host,
+                             int64_t ldy, cudaStream_t s) {
+    sqz_status st;
     // one flat copy each way when the rows are packed (a 2-D copy otherwise)
     if (L->k_in > 0) {
         const size_t row = (size_t)L->k_in * 2;
@@ -556,6 +577,68 @@ sqz_status sqz_gemv_host(sqz_layer_t layer, const uint16_t* x_host, int32_t batc
                                   : cudaMemcpy2DAsync(y_host, (size_t)ldy * 2, L->y_stage, row, row, (size_t)batch,
                                                       cudaMemcpyDeviceToHost, s);
         SQZ_CUDA_TRY(e, "y device-to-host copy");
+    }
+    return SQZ_OK;
+}
+
+constexpr size_t kHostGraphsPerLayer = 64;
+
+// The cached graph of this call, captured on first use; nullptr when the
+// call cannot be captured (the legacy default stream, or a stream that is
+// already being captured), in which case the caller enqueues it directly.
+cudaGraphExec_t host_graph(sqz_layer* L, const uint16_t* x_host, int32_t batch, int64_t ldx, uint16_t* y_host,
+                           int64_t ldy, cudaStream_t s) {
+    if (s == nullptr || s == cudaStreamLegacy || s == cudaStreamPerThread) return nullptr;
+    for (const void* p : {static_cast<const void*>(x_host), static_cast<const void*>(y_host)}) {
+        cudaPointerAttributes a{};
+        if (cudaPointerGetAttributes(&a, p) != cudaSuccess || a.type != cudaMemoryTypeHost) {
+            (void)cudaGetLastError();
+            return nullptr;  // pageable memory: copied directly, not captured
+        }
+    }
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) return nullptr;
+    for (auto& g : L->host_graphs)
+        if (g.x == x_host && g.y == y_host && g.batch == batch && g.ldx == ldx && g.ldy == ldy && g.stream == s) {
+            g.used = ++L->host_clock;
+            return g.exec;
+        }
+    if (cudaStreamBeginCapture(s, cudaStreamCaptureModeThreadLocal) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return nullptr;
+    }
+    const sqz_status st = enqueue_host_call(L, x_host, batch, ldx, y_host, ldy, s);
+    cudaGraph_t graph = nullptr;
+    const cudaError_t e = cudaStreamEndCapture(s, &graph);
+    cudaGraphExec_t exec = nullptr;
+    if (st == SQZ_OK && e == cudaSuccess && graph && cudaGraphInstantiate(&exec, graph, 0) != cudaSuccess) exec = nullptr;
+    if (graph) cudaGraphDestroy(graph);
+    (void)cudaGetLastError();
+    if (!exec) return nullptr;
+    if (L->host_graphs.size() >= kHostGraphsPerLayer) {  // drop the least recently used
+        size_t old = 0;
+        for (size_t i = 1; i < L->host_graphs.size(); ++i)
+            if (L->host_graphs[i].used < L->host_graphs[old].used) old = i;
+        cudaGraphExecDestroy(L->host_graphs[old].exec);
+        L->host_graphs.erase(L->host_graphs.begin() + (ptrdiff_t)old);
+    }
+    L->host_graphs.push_back({x_host, y_host, batch, ldx, ldy, s, exec, ++L->host_clock});
+    return exec;
+}
+
+}  // namespace
+
+extern "C" {
+
+sqz_status sqz_gemv_host(sqz_layer_t layer, const uint16_t* x_host, int32_t batch, int64_t ldx, uint16_t* y_host,
+                         int64_t ldy, void* stream) {
+    sqz_status st = check_gemv_args(layer, x_host, batch, ldx, y_host, ldy);
+    if (st != SQZ_OK) return st;
+    cudaStream_t s = as_stream(stream);
+    if (cudaGraphExec_t exec = host_graph(layer, x_host, batch, ldx, y_host, ldy, s)) {
+        SQZ_CUDA_TRY(cudaGraphLaunch(exec, s), "graph launch");
+    } else if ((st = enqueue_host_call(layer, x_host, batch, ldx, y_host, ldy, s)) != SQZ_OK) {
+        return st;
     }
     SQZ_CUDA_TRY(cudaStreamSynchronize(s), "stream synchronize");
     return SQZ_OK;
@@ -627,6 +710,7 @@ sqz_status sqz_layer_set_mac(sqz_layer_t layer, int32_t mac) {
     if (mac != SQZ_MAC_TENSOR_CORES && mac != SQZ_MAC_CUDA_CORES && mac != SQZ_MAC_MIXED)
         return fail(SQZ_ERR_INVALID_ARG, "unknown MAC unit %d", mac);
     layer->mac = mac;
+    drop_host_graphs(layer);  // captured launches used the previous kernel
     return SQZ_OK;
 }
 
@@ -634,6 +718,7 @@ sqz_status sqz_layer_set_csr_mode(sqz_layer_t layer, int32_t mode) {
     if (!layer) return fail(SQZ_ERR_INVALID_ARG, "layer is NULL");
     if (mode != SQZ_CSR_BALANCED && mode != SQZ_CSR_ROWWISE) return fail(SQZ_ERR_INVALID_ARG, "unknown CSR mode %d", mode);
     layer->csr_mode = mode;
+    drop_host_graphs(layer);
     return SQZ_OK;
 }
 

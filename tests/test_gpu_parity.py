@@ -202,6 +202,31 @@ def test_host_entry_point_matches_device(B):
     assert np.array_equal(yh.numpy().view(np.uint16), yd)
 
 
+def test_host_entry_point_replays_read_new_inputs(B, orc):
+    """Repeated host calls on the same pinned buffers (served by one captured
+    graph) read each call's x and write each call's y; changing the MAC unit
+    drops the captured launches; pageable buffers take the direct path."""
+    L = make_small(33, 300, 1024, 3, 600)
+    layer = upload(B, L)
+    s = torch.cuda.Stream()
+    xh = torch.empty((2, 1024), dtype=torch.int16).pin_memory()
+    yh = torch.empty((2, 300), dtype=torch.int16).pin_memory()
+    for trial in range(4):
+        if trial == 2:
+            B.sqz_layer_set_mac(layer, B.SQZ_MAC_CUDA_CORES)
+        x = synth.make_x(2, 1024, seed=40 + trial)
+        xh.copy_(torch.from_numpy(x.view(np.int16)))
+        B.sqz_gemv_host(layer, xh, yh, stream=s, batch=2 if trial < 2 else 1)
+        b = 2 if trial < 2 else 1
+        y_ref, bound = orc.gemv_layer(L, x[:b])
+        assert_close(yh.numpy()[:b].view(np.uint16), y_ref, bound, f"host replay {trial}")
+    xp = torch.from_numpy(synth.make_x(1, 1024, seed=50).view(np.int16).copy())  # pageable
+    yp = torch.zeros((1, 300), dtype=torch.int16)
+    B.sqz_gemv_host(layer, xp, yp, stream=s)
+    y_ref, bound = orc.gemv_layer(L, xp.numpy().view(np.uint16))
+    assert_close(yp.numpy().view(np.uint16), y_ref, bound, "host pageable")
+
+
 def test_non_default_stream(B, orc):
     L = make_small(21, 500, 2048, 3, 400)
     x = synth.make_x(2, 2048, seed=9)
