@@ -420,8 +420,11 @@ def pin_enc_double_to_half_matches_numpy(orc):
 
 
 def pin_enc_outlier_tails_page_example(orc):
-    # 0.2th / 99.8th percentiles: 0.4 % of the weights, 0.2 % in each tail
-    assert orc.outliers_per_tail(100000, 0.004) == 200
+    # the page's 0.2th / 99.8th percentiles: 0.4 % of the weights, 0.2 % in each tail
+    lo, hi, frac, tail = (float(v) for v in read_golden("outlier_percentiles.txt")[0])
+    assert abs((lo + (100.0 - hi)) / 100.0 - frac) < 1e-12 and abs(lo / 100.0 - tail) < 1e-12
+    n = 100000
+    assert orc.outliers_per_tail(n, frac) == round(tail * n) == 200
     assert orc.outliers_per_tail(1000, 0.0045) == 2  # 2.25 rounds to 2
     assert orc.outliers_per_tail(1000, 0.005) == 3   # 2.5 rounds up (the reading taken)
     assert orc.outliers_per_tail(10, 1.0) == 5        # at most half the weights per tail
