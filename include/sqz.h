@@ -31,8 +31,10 @@
  *
  * Arithmetic: products of fp16 operands are exact in fp32; accumulation is
  * in fp32; y(i,b) is rounded once to fp16 (round to nearest even).  The
- * result agrees with the exact value within 1e-3 * sum_k |w x| + 1e-6 and is
- * bitwise reproducible from run to run (no floating-point atomics).
+ * result agrees with the exact value within
+ * 1e-3 * (sum_k |w(i,k) x(b,k)| + sum_j |val(j) x(b,col(j))|) + 1e-6 (j over
+ * row i's outliers) and is bitwise reproducible from run to run (no
+ * floating-point atomics).
  *
  * Layouts: x is [batch][ldx] and y is [batch][ldy], row-major (the
  * torch `x @ W.T` convention).  y is overwritten, never accumulated into.
