@@ -1,18 +1,22 @@
 #!/usr/bin/env python3
 """Benchmark of the fused Dense-and-Sparse LUT GEMV, y = (Q + S) x.
 
-One step = one call of the fused kernel on one layer instance with one batch
-of activations.  Steps rotate over enough distinct layer instances that their
-total size is at least 4x the L2 cache, so every step streams its layer from
-HBM.  The K timed steps are CUDA-graph replays (one kernel node per step),
-bracketed by a barrier and a device synchronise, timed with CUDA events on
-the launching stream; the reported time is the maximum over ranks.
+One step = one batch-1 token through a stack of R distinct layers of the
+workload's shape: R fused-kernel calls, each on its own layer instance with
+its own activations.  R is at least 32 (LLaMA-7B's decoder depth) and large
+enough that the stack is at least 4x the L2 cache, so every call streams its
+layer from HBM.  The K timed steps are CUDA-graph replays (several steps per
+graph, one kernel node per call), bracketed by a barrier and a device
+synchronise, timed with CUDA events on the launching stream; the reported
+time is the maximum over ranks.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
-Prints one JSON line on rank 0.  ``--impl reference`` times the CPU oracle
-(plain fp64 C, single thread) on a bounded sample of the same workload.
-``--sweep`` prints one line per workload shape instead (for the notes).
+Prints one JSON line on rank 0.  ``--gpus N`` without a torchrun
+environment starts N ranks itself (one GPU each, independent replicas).
+``--impl reference`` times the CPU oracle (plain fp64 C) on a bounded
+sample of the same workload.  ``--sweep`` prints one line per workload
+shape instead (for the notes).
 """
 from __future__ import annotations
 
@@ -47,8 +51,8 @@ WORKLOAD_DESC = {
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=50000)
-    p.add_argument("--warmup", type=int, default=5000)
+    p.add_argument("--steps", type=int, default=2000)
+    p.add_argument("--warmup", type=int, default=200)
     p.add_argument("--workload", default=DEFAULT_WORKLOAD)
     p.add_argument("--shape-index", type=int, default=0)
     p.add_argument("--impl", choices=("ours", "reference"), default="ours")
@@ -60,6 +64,8 @@ def parse():
     p.add_argument("--encode", action="store_true",
                    help="time the encoder (sqz_encode) on synthetic weights of the workload's shape instead")
     p.add_argument("--encode-iters", type=int, default=30, help="k-means iterations of --encode")
+    p.add_argument("--selftest-ranks", action="store_true",
+                   help="(tests) the rank plumbing alone on CPU: gloo ranks report fixed times, no GPU work")
     p.add_argument("--profile-launches", type=int, default=0,
                    help="for profiler captures: one layer instance of the shape, this many plain launches, "
                         "no timing and no JSON line")
@@ -148,7 +154,7 @@ class ClockSampler:
                0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
                0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
 
-    def __init__(self, device_index: int, period_s: float = 0.005):
+    def __init__(self, device_index: int, period_s: float = 0.001):
         self.ok = False
         self.samples, self.reasons = [], 0
         self.period = period_s
@@ -214,32 +220,70 @@ def config_for(args, shape, instances, inst_bytes):
             args.workload, f"{shape.n_out}x{shape.k_in}, {shape.bits}-bit, {shape.density:.2%} CSR, batch {shape.batch}"),
         "n_out": shape.n_out, "k_in": shape.k_in, "bits": shape.bits, "density": shape.density,
         "batch": shape.batch, "outliers": shape.dist, "csr_scheme": args.csr,
-        "l2": f"inputs larger than L2: {instances} rotating layer instances, {instances * inst_bytes / 1e6:.0f} MB",
+        "step": f"one token through a stack of {instances} distinct layers of this shape ({instances} calls)",
+        "l2": f"inputs larger than L2: the stack holds {instances * inst_bytes / 1e6:.0f} MB",
         "parallelism": "replicas (independent layers per GPU)",
     }
 
 
 # ------------------------------------------------------------- CPU oracle
 
-def cpu_oracle_rate(shape, seconds: float, rows_per_call: int, instance: int = 0):
-    """Time the oracle on rows of one layer instance; returns (GB/s, rows done, s)."""
+def _oracle_rows_rate(orc, L, x, rows_per_call, seconds, start_row, per_row_bytes):
+    """One thread: oracle calls over consecutive row blocks for `seconds`;
+    returns (rows, elapsed s)."""
+    done, t0, start = 0, time.perf_counter(), start_row
+    while True:
+        rows = (np.arange(start, start + rows_per_call) % L.n_out).astype(np.int32)
+        orc.gemv_layer(L, x, rows=rows)
+        done += rows_per_call
+        start += rows_per_call
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            return done, el
+
+
+def cpu_oracle_rate(shape, seconds: float, rows_per_call: int, threads: int = 1, instance: int = 0):
+    """The oracle as it stands on `threads` host threads (ctypes releases the
+    GIL, so the C oracle runs in parallel on disjoint row blocks), for about
+    `seconds`; returns (GB/s, rows done, elapsed s)."""
     import oracle
 
     orc = oracle.default()
     L = synth.layer_for(shape, instance=instance)
     x = synth.x_for(shape, instance=instance)
     per_row_bytes = acc.gemv_bytes(shape.n_out, shape.k_in, shape.bits, L.nnz, shape.batch) / shape.n_out
-    done, t0 = 0, time.perf_counter()
-    start = 0
-    while True:
-        rows = (np.arange(start, start + rows_per_call) % shape.n_out).astype(np.int32)
-        orc.gemv_layer(L, x, rows=rows)
-        done += rows_per_call
-        start += rows_per_call
-        el = time.perf_counter() - t0
-        if el >= seconds:
-            break
-    return done * per_row_bytes / el / 1e9, done, el
+    out = [None] * threads
+
+    def work(t):
+        out[t] = _oracle_rows_rate(orc, L, x, rows_per_call, seconds, t * (shape.n_out // threads), per_row_bytes)
+
+    t0 = time.perf_counter()
+    ts = [threading.Thread(target=work, args=(t,)) for t in range(threads)]
+    for t in ts:
+        t.start()
+    for t in ts:
+        t.join()
+    el = time.perf_counter() - t0
+    rows = sum(r for r, _ in out)
+    return rows * per_row_bytes / el / 1e9, rows, el
+
+
+def cpu_baseline(shape, seconds_per_rep: float = 2.5, reps: int = 3):
+    """Median of `reps` timings at one thread and at every host core."""
+    cores = os.cpu_count() or 1
+    res = {}
+    for threads in sorted({1, cores}):
+        runs = [cpu_oracle_rate(shape, seconds_per_rep, 64, threads) for _ in range(reps)]
+        gbs = statistics.median(r[0] for r in runs)
+        res[threads] = (gbs, sum(r[1] for r in runs), sum(r[2] for r in runs))
+    gbs, rows, secs = res[cores]
+    line = {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"{rows} rows of one {shape.n_out}x{shape.k_in} layer in {secs:.1f} s on {cores} host threads "
+                      f"(fp64 C oracle, disjoint row blocks per thread), median of {reps}"}
+    g1, r1, s1 = res[1]
+    line["one_thread"] = {"value": g1, "unit": "GB/s", "cores": 1,
+                          "sample": f"{r1} rows in {s1:.1f} s on one thread, median of {reps}"}
+    return line
 
 
 def run_reference(args):
@@ -285,6 +329,20 @@ def run_reference(args):
 
 # ------------------------------------------------------------ GPU arm
 
+MIN_STACK = 32          # layers per step: at least LLaMA-7B's decoder depth
+CALLS_PER_GRAPH = 512   # about this many kernel nodes per captured graph
+
+
+def stack_depth(l2_bytes: int, layer_bytes: int) -> int:
+    """Layers per step: at least MIN_STACK and at least 4x L2 in total."""
+    return max(MIN_STACK, math.ceil(4 * l2_bytes / layer_bytes))
+
+
+def graph_plan(steps: int, per_graph: int):
+    """Replays of the full graph and the step count of the tail graph."""
+    return divmod(steps, per_graph)
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -292,12 +350,10 @@ def run_ours(args):
     from lut_dequant_gemv_b200 import binding as B
 
     world, rank, local = dist_env()
+    torch.cuda.set_device(local)
     if world > 1:
-        torch.cuda.set_device(local)
         dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
-    else:
-        torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     B.lib()
 
@@ -305,9 +361,9 @@ def run_ours(args):
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     L0 = synth.layer_for(shape, seed=args.seed, instance=instance_id(rank, 0))
     inst_bytes = L0.nbytes()
-    instances = max(2, math.ceil(4 * l2 / inst_bytes))
+    R = stack_depth(l2, inst_bytes)
     layers, xs, ys = [], [], []
-    for i in range(instances):
+    for i in range(R):
         L = L0 if i == 0 else synth.layer_for(shape, seed=args.seed, instance=instance_id(rank, i))
         layers.append(B.create_layer_from_numpy(L.n_out, L.k_in, L.bits, L.codes, L.lut, L.rowptr, L.col, L.val,
                                                 device=dev))
@@ -317,42 +373,41 @@ def run_ours(args):
                   .to(dev))
         ys.append(torch.empty((shape.batch, shape.n_out), dtype=torch.int16, device=dev))
     nnz = L0.nnz
-    bytes_per_step = acc.gemv_bytes(shape.n_out, shape.k_in, shape.bits, nnz, shape.batch)
+    bytes_per_call = acc.gemv_bytes(shape.n_out, shape.k_in, shape.bits, nnz, shape.batch)
+    bytes_per_step = R * bytes_per_call
 
     stream = torch.cuda.Stream(device=dev)
     torch.cuda.synchronize(dev)
     with torch.cuda.stream(stream):
-        for i in range(instances):
+        for i in range(R):
             B.sqz_gemv(layers[i], xs[i], ys[i], stream=stream)
     stream.synchronize()
 
-    def capture(n, offset):
+    def capture(nsteps):
         g = torch.cuda.CUDAGraph()
-        if n == 0:
-            return None
         with torch.cuda.graph(g, stream=stream):
-            for j in range(n):
-                i = (offset + j) % instances
-                B.sqz_gemv(layers[i], xs[i], ys[i], stream=stream)
+            for _ in range(nsteps):
+                for i in range(R):
+                    B.sqz_gemv(layers[i], xs[i], ys[i], stream=stream)
         return g
 
-    per_graph = instances * max(1, 512 // instances)
+    per_graph = max(1, CALLS_PER_GRAPH // R)  # steps per full graph
+    graphs = {per_graph: capture(per_graph)}
+    for k in (args.warmup % per_graph, args.steps % per_graph):
+        if k and k not in graphs:
+            graphs[k] = capture(k)
 
-    def run_steps(k, graphs):
-        full, tail = divmod(k, per_graph)
+    def run_steps(k):
+        full, tail = graph_plan(k, per_graph)
         for _ in range(full):
-            graphs[0].replay()
+            graphs[per_graph].replay()
         if tail:
-            graphs[1][tail].replay()
-
-    main_graph = capture(per_graph, 0)
-    tails = {}
-    for k in {args.warmup % per_graph, args.steps % per_graph} - {0}:
-        tails[k] = capture(k, 0)
-    graphs = (main_graph, tails)
+            graphs[tail].replay()
 
     with torch.cuda.stream(stream):
-        run_steps(args.warmup, graphs)
+        for g in graphs.values():  # first replays upload the graphs
+            g.replay()
+        run_steps(args.warmup)
     stream.synchronize()
 
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -362,35 +417,19 @@ def run_ours(args):
     with ClockSampler(local) as clk:
         with torch.cuda.stream(stream):
             ev0.record(stream)
-            run_steps(args.steps, graphs)
+            run_steps(args.steps)
             ev1.record(stream)
         torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
     ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
     ms_per_step = ms / args.steps
+    us_per_call = ms_per_step * 1e3 / R
     value = whole_job_gbs(world, bytes_per_step, args.steps, ms)
-    per_launch_gbs = bytes_per_step / (ms_per_step / 1e3) / 1e9
+    per_launch_gbs = bytes_per_call / (us_per_call * 1e-6) / 1e9
 
-    # ---- end to end through the host entry point (pinned buffers)
-    xh = [torch.from_numpy(synth.x_for(shape, seed=args.seed, instance=instance_id(rank, i)).view(np.int16).copy())
-          .pin_memory() for i in range(instances)]
-    yh = torch.empty((shape.batch, shape.n_out), dtype=torch.int16).pin_memory()
-    e2e_steps = min(args.steps, 20000)
-    with torch.cuda.stream(stream):
-        for j in range(min(args.warmup, 200)):
-            B.sqz_gemv_host(layers[j % instances], xh[j % instances], yh, stream=stream)
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize(dev)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for j in range(e2e_steps):
-            B.sqz_gemv_host(layers[j % instances], xh[j % instances], yh, stream=stream)
-        e1.record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
-    e2e_value = whole_job_gbs(world, bytes_per_step, e2e_steps, e2e_ms)
+    e2e = e2e_measure(B, torch, dist, shape, layers, R, args, world, rank, dev, stream, bytes_per_step,
+                      us_per_call)
 
     # ---- fp16 dense yardstick (same shape, uncompressed weights)
     yard = None
@@ -404,26 +443,21 @@ def run_ours(args):
     line = {
         "metric": METRIC if args.workload == DEFAULT_WORKLOAD else f"dense+sparse GEMV achieved HBM GB/s ({args.workload})",
         "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": ms_per_step, "us_per_call": ms_per_step * 1e3,
+        "ms_per_step": ms_per_step, "us_per_call": us_per_call, "calls_per_step": R,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f16 storage, f32 accumulate", "data": "synthetic",
-        "config": config_for(args, shape, instances, inst_bytes),
+        "config": config_for(args, shape, R, inst_bytes),
         "roofline": {"bound": "hbm", "achieved": per_launch_gbs, "peak": peak, "unit": "GB/s",
                      "frac": per_launch_gbs / peak, "traffic": traffic,
-                     "peak_kind": f"{peak_kind} copy bandwidth", "algorithmic_bytes_per_launch": bytes_per_step,
+                     "peak_kind": f"{peak_kind} copy bandwidth", "algorithmic_bytes_per_launch": bytes_per_call,
                      "frac_of_nominal_8000": per_launch_gbs / 8000.0},
-        "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": 2 * shape.batch * shape.k_in,
-                "d2h_bytes_per_step": 2 * shape.batch * shape.n_out, "us_per_call": e2e_ms / e2e_steps * 1e3,
-                "steps": e2e_steps, "api": "sqz_gemv_host"},
-        "gpu_launches": args.steps,
+        "e2e": e2e,
+        "gpu_launches": args.steps * R,
         "clocks": clk.summary(),
         "yardstick_fp16_dense": yard,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        gbs, rows, secs = cpu_oracle_rate(shape, 10.0, 256)
-        line["cpu_baseline"] = {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
-                                "sample": f"{rows} rows of one {shape.n_out}x{shape.k_in} layer in {secs:.1f} s "
-                                          f"(fp64 C oracle, one thread)"}
+        line["cpu_baseline"] = cpu_baseline(shape)
     if rank == 0:
         print(json.dumps(line), flush=True)
     for lay in layers:
@@ -432,6 +466,65 @@ def run_ours(args):
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def e2e_measure(B, torch, dist, shape, layers, R, args, world, rank, dev, stream, bytes_per_step, us_kernel):
+    """End to end through the host entry point: every call copies its
+    layer's x in from pinned host memory, runs the product, copies y back
+    and synchronises.  One step = R calls (the same stack as the device
+    measurement).  Every (layer, host buffers) pair is warmed first, so the
+    timed calls replay captured graphs rather than capture them."""
+    xh = [torch.from_numpy(synth.x_for(shape, seed=args.seed, instance=instance_id(rank, i)).view(np.int16).copy())
+          .pin_memory() for i in range(R)]
+    yh = torch.empty((shape.batch, shape.n_out), dtype=torch.int16).pin_memory()
+    steps = max(1, min(args.steps, 200))
+    with torch.cuda.stream(stream):
+        for _ in range(max(2, min(args.warmup, 20))):
+            for i in range(R):
+                B.sqz_gemv_host(layers[i], xh[i], yh, stream=stream)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        t0 = time.perf_counter()
+        for _ in range(steps):
+            for i in range(R):
+                B.sqz_gemv_host(layers[i], xh[i], yh, stream=stream)
+        wall = time.perf_counter() - t0
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    calls = steps * R
+    us_call = ms * 1e3 / calls
+
+    # ---- where a call's time goes: the device span of one call (copies +
+    # kernel, events on the stream around it), the ctypes round trip of a
+    # call that does nothing, and the rest (launch and synchronisation)
+    dev_spans = []
+    with torch.cuda.stream(stream):
+        for i in range(min(R, 64)):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            B.sqz_gemv_host(layers[i], xh[i], yh, stream=stream)
+            b.record(stream)
+            b.synchronize()
+            dev_spans.append(a.elapsed_time(b) * 1e3)
+    lib = B.lib()
+    n = 20000
+    t0 = time.perf_counter()
+    for _ in range(n):
+        lib.sqz_version()
+    ctypes_us = (time.perf_counter() - t0) / n * 1e6
+    span = statistics.median(dev_spans)
+    return {"value": whole_job_gbs(world, bytes_per_step, steps, ms), "unit": "GB/s",
+            "h2d_bytes_per_step": R * 2 * shape.batch * shape.k_in,
+            "d2h_bytes_per_step": R * 2 * shape.batch * shape.n_out,
+            "us_per_call": us_call, "wall_us_per_call": wall * 1e6 / calls, "steps": steps, "calls_per_step": R,
+            "api": "sqz_gemv_host (pinned host x/y)",
+            "breakdown_us": {"device_span_copies_and_kernel": span, "kernel_in_graph_loop": us_kernel,
+                             "copies_and_dependencies": span - us_kernel, "ctypes_round_trip": ctypes_us,
+                             "launch_sync_python_rest": us_call - span - ctypes_us}}
 
 
 def fp16_yardstick(B, torch, shape, dev, stream, l2):
@@ -563,8 +656,59 @@ def run_encode(args):
     return 0
 
 
+def free_port() -> int:
+    import socket
+
+    with socket.socket() as so:
+        so.bind(("127.0.0.1", 0))
+        return so.getsockname()[1]
+
+
+def spawn_ranks(args) -> int:
+    """`--gpus N` outside torchrun: start N ranks of this script (one GPU
+    each; independent replicas) through torch.distributed.run on this node
+    and return its exit status.  Refuses when fewer than N GPUs are visible."""
+    import subprocess
+
+    if not args.selftest_ranks:
+        import torch
+
+        have = torch.cuda.device_count()
+        if have < args.gpus:
+            print(f"bench.py: --gpus {args.gpus} but only {have} CUDA device(s) are visible", file=sys.stderr)
+            return 2
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={args.gpus}",
+           "--master-addr", "127.0.0.1", f"--master-port={free_port()}", os.path.abspath(__file__), *sys.argv[1:]]
+    return subprocess.call(cmd)
+
+
+def run_selftest(args):
+    """Rank plumbing without a GPU: gloo ranks, rank r reports 10*(r+1) ms;
+    rank 0 prints the slowest rank's time, the world size and the whole-job
+    value exactly as the GPU arm computes them."""
+    import datetime
+
+    import torch.distributed as dist
+
+    world, rank, _ = dist_env()
+    if world > 1:
+        dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+    ms = max_over_ranks(10.0 * (rank + 1), world)
+    if rank == 0:
+        print(json.dumps({"n_gpus": world, "ms": ms, "value": whole_job_gbs(world, 1_000_000, args.steps, ms),
+                          "steps": args.steps}), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     args = parse()
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        return spawn_ranks(args)
+    if args.selftest_ranks:
+        return run_selftest(args)
     if args.encode:
         return run_encode(args)
     if args.profile_launches:

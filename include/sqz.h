@@ -187,10 +187,12 @@ SQZ_API sqz_status sqz_layer_set_csr_mode(sqz_layer_t layer, int32_t mode);
 
 /*
  * Read and clear the handle's device status word, ordered on `stream`
- * (synchronises it).  0 means every call so far completed normally; bit 0
- * (1) means a bounded wait for a copy into shared memory gave up, in which
- * case the outputs of the affected call are not valid.
- * Errors: SQZ_ERR_INVALID_ARG, SQZ_ERR_CUDA.
+ * (synchronises it).  *status receives the word: 0 means every call so far
+ * completed normally; bit 0 (1) means a bounded wait for a copy into shared
+ * memory gave up, and then y of the affected call is undefined.  Returns
+ * SQZ_ERR_TIMEOUT (with *status set) when bit 0 was set, so that a caller
+ * checking only return codes sees it; SQZ_OK otherwise.
+ * Errors: SQZ_ERR_INVALID_ARG, SQZ_ERR_CUDA, SQZ_ERR_TIMEOUT.
  */
 SQZ_API sqz_status sqz_layer_status(sqz_layer_t layer, void* stream, int32_t* status);
 
@@ -240,33 +242,31 @@ SQZ_API sqz_status sqz_fp16_gemv(const uint16_t* w, int32_t n_out, int32_t k_in,
  * counterpart in the paper; it exists for callers that cannot allocate.)
  *
  * Who needs it: code that cannot call cudaMalloc where it wants the check --
- * code running while a CUDA graph is being captured (allocation is not
- * permitted during capture), serving loops that must not take the implicit
- * device synchronisation of cudaMalloc/cudaFree, and runtimes that reserve
- * all device memory up front and forbid later allocations.
- * sqz_create_layer allocates a flag word for its check; this call uses a
- * fixed 256-byte device array inside the library instead (held on every
- * GPU that loads the library until the process exits; the check uses one
- * 4-byte word of it whatever the matrix size).
+ * serving loops that must not take the implicit device synchronisation of
+ * cudaMalloc/cudaFree, and runtimes that reserve all device memory up front
+ * and forbid later allocations.  sqz_create_layer allocates a flag word for
+ * its check; this call uses a fixed 256-byte device array inside the library
+ * instead (held on every GPU that loads the library until the process exits;
+ * the check uses one 4-byte word of it whatever the matrix size).
  *
  * rowptr: device [n_out+1]; col: device [nnz] (both caller-owned, read
  * only).  *flags (host) receives 0 for a well-formed matrix, else the OR of
  * 1 rowptr[0] != 0, 2 rowptr[n_out] != nnz, 4 rowptr decreasing, 8 a column
  * outside [0, k_in).  nnz == 0 writes 0 without touching the device (as
  * sqz_create_layer ignores the CSR arrays then).  The call is ordered on
- * `stream` and synchronises it before returning.
+ * `stream` and synchronises it before returning, so it cannot be recorded
+ * into a CUDA graph: on a stream that is being captured it returns
+ * SQZ_ERR_UNSUPPORTED before enqueuing anything (the capture stays valid).
  *
- * The first call on a device looks up the array's device address (once per
- * device, with that device current); make that first call before any
- * stream capture.  Every call shares the one array: calls whose work
- * overlaps on the GPU (different streams, or host threads) race and may
- * report each other's flags -- serialise them.
+ * Every call looks up the array's device address in the current context
+ * (no allocation) and clears the flag word first.  Every call shares the one
+ * array: calls whose work overlaps on the GPU (different streams, or host
+ * threads) race and may report each other's flags -- serialise them.
  *
  * Errors: SQZ_ERR_INVALID_ARG for a NULL flags pointer, n_out outside
  * [0, 2^31-2], k_in < 0, nnz outside [0, 2^31-1] (the int32 limits of the
- * CSR format), or NULL rowptr/col with nnz > 0; SQZ_ERR_UNSUPPORTED for a
- * device ordinal above 127; SQZ_ERR_CUDA.  Never calls cudaMalloc or
- * cudaFree.
+ * CSR format), or NULL rowptr/col with nnz > 0; SQZ_ERR_UNSUPPORTED on a
+ * stream under capture; SQZ_ERR_CUDA.  Never calls cudaMalloc or cudaFree.
  */
 SQZ_API sqz_status sqz_check_csr_static(const int32_t* rowptr, const int32_t* col, int32_t n_out, int32_t k_in,
                                         int64_t nnz, void* stream, int32_t* flags);

@@ -7,40 +7,41 @@
 // Work decomposition
 //   * Rows are grouped in tiles of 16 (the M of an m16n8k16 MMA); columns in
 //     super-groups of 256 (16 k16-steps).  A unit = (tile, super-group).
-//   * One CTA of 16 warps per SM.  Each CTA owns a contiguous run of whole
-//     tiles (runs differ by at most one tile) and its warps split the CTA's
-//     units into contiguous ranges (equal, except that the eight warps that
-//     also sum the sparse part take one unit less each when there is one),
-//     so a tile is finished inside one CTA: no global atomics, no second
-//     pass.
-//   * A tile held by several warps is finished by the warp that flushes its
-//     part last (a shared-memory arrival counter): it adds the parts in warp
-//     order -- deterministic -- and writes y while the other warps keep
-//     decoding.  There is no CTA-wide barrier after the dense loop.
+//   * One CTA of 12 warps per SM and call; its registers and shared memory
+//     fit two CTAs on an SM, so the next call's CTA (programmatic dependent
+//     launch) is resident while this one computes.  Each CTA owns a
+//     contiguous run of whole tiles (runs differ by at most one tile) and its
+//     warps split the CTA's units into contiguous ranges (equal, except that
+//     the eight warps that also sum the sparse part give one unit each to the
+//     other warps when the layer has outliers), so a tile is finished inside
+//     one CTA: no global atomics, no second pass.
+//   * A warp that holds a whole tile writes its rows of y itself.  Tiles
+//     split between warps are finished after the dense loop: one CTA
+//     barrier, then the threads add the warps' parts of every shared tile in
+//     warp order (deterministic, the same order for every batch size), add
+//     each row's sparse sum and write y.
 //
 // Streaming: every warp streams its units through a private ring of
 // shared-memory stages with asynchronous 16-byte copies (cp.async, one
 // commit group per unit), keeping stages-1 units in flight while it
-// decodes.  The copies are asynchronous on purpose: a CTA barrier waits for
-// the outstanding ordinary loads of the threads that reach it, but not for
-// asynchronous copies, so the barriers of the prologue never wait for the
-// code stream.  Before waiting for the previous kernel of the stream
-// (programmatic dependent launch; the weights never depend on it) a CTA
-// requests its LUT planes, rowptr slice and sparse entries (bulk copies) and
-// the first code unit of every warp; x is requested right after the wait and
-// ahead of the remaining code units.  Waits on the bulk copies are bounded
-// and record a status bit instead of hanging.
+// decodes.  The copies are asynchronous on purpose: the barriers of the
+// prologue never wait for the code stream.  Before waiting for the previous
+// kernel of the stream (programmatic dependent launch; the weights never
+// depend on it) a CTA requests its LUT planes, rowptr slice and sparse
+// entries (bulk copies) and the first code units of every warp; x is
+// requested right after the wait and ahead of the remaining code units.
+// Waits on the bulk copies are bounded and record a status bit instead of
+// hanging.
 //
 // Decode (kernel-native code layout, built by repack_codes_kernel): for each
 // k16-step a lane holds 4 codes of row g and 4 of row g+8 (g = lane/4) at
 // columns 4*t4..4*t4+3 (t4 = lane%4) of the step.  A code indexes the row's
 // LUT kept in registers as byte planes (low bytes, high bytes); `prmt`
-// gathers the bytes of four weights at once and a second `prmt` interleaves
+// gathers the bytes of four weights at once and two more `prmt` interleave
 // them into fp16 pairs, which are exactly the A fragment of the MMA once
 // the MMA's k order is permuted to match (the same permutation is applied
 // to x, so the product is unchanged).  The byte permutes run on the integer
-// ALU pipe, which bounds the dense part; shifts are written as high
-// multiplies so that they run on the FMA pipe instead.
+// ALU pipe, which bounds the dense part.
 //
 // Padding instead of ragged paths: columns past K inside the last
 // super-group carry, per row, the code of a finite LUT entry, and x is zero
@@ -55,12 +56,12 @@
 // Sparse part: the CSR entries of the rows of a CTA's tiles are split evenly
 // over 256 of its threads (a fixed number of nonzeros per thread,
 // independent of how skewed the rows are) -- the balanced scheme of the
-// pages.  Each thread
-// sums its share per row before entering the dense loop, while the code
-// units are in flight, and signals an mbarrier; no CTA barrier follows.
-// The warp that finishes a tile waits on that mbarrier and adds to each row
-// the interior sum and then the pieces of the threads whose shares cut the
-// row, in thread order (deterministic).
+// pages.  Each thread sums its share per row (head piece, rows it holds
+// whole, tail piece) after x has arrived and before its dense loop; after a
+// barrier of those 256 threads, each row's interior sum and the pieces of the
+// threads whose shares cut the row are added in thread order (deterministic)
+// into the row's slot, and the threads arrive on an mbarrier that the
+// writers of y wait on.
 #pragma once
 
 #include <type_traits>
@@ -135,7 +136,7 @@ struct Plan {
     int csr_cap;     // CSR entries of a CTA that are staged in shared memory (more: read from global)
     // byte offsets
     int off_x, off_lut, off_rp, off_rowsum, off_head, off_tail, off_headrow, off_tailrow, off_slots, off_wrange,
-        off_tinfo, off_cnt, off_col, off_val, off_acc, off_ring, total;
+        off_tinfo, off_col, off_val, off_acc, off_ring, total;
 };
 
 __host__ __device__ inline int round_up(int v, int m) { return (v + m - 1) / m * m; }
@@ -212,8 +213,6 @@ __host__ __device__ inline Plan make_plan(int bits, int n_out, int k_in, int bat
     P.off_wrange = off;
     off += round_up(kWarps * 3 * 4, 16);
     P.off_tinfo = off;
-    off += round_up(P.ctiles_max * 4, 16);
-    P.off_cnt = off;
     off += round_up(P.ctiles_max * 4, 16);
     off = round_up(off, 128);
     P.off_acc = off;  // per-tile sums across passes
@@ -621,7 +620,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_fused_kernel(const 
     float* s_slots = reinterpret_cast<float*>(smem + P.off_slots);
     int* s_wrange = reinterpret_cast<int*>(smem + P.off_wrange);  // [warp] = {first unit, end unit, first tile}
     int* s_tinfo = reinterpret_cast<int*>(smem + P.off_tinfo);    // [tile] = mask of warps holding parts
-    int* s_cnt = reinterpret_cast<int*>(smem + P.off_cnt);        // [tile] = parts flushed so far
     const int rp_off = ra & 3;
     const int* s_rp = reinterpret_cast<const int*>(smem + P.off_rp) + rp_off;  // s_rp[i] = rowptr[ra + i]
 
@@ -688,8 +686,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_fused_kernel(const 
     const int pre = D < kPreWait ? D : kPreWait;
     for (int j = 0; j < pre; ++j) issue(j);
 
-    // ---- bookkeeping: warp ranges, contributors and arrival counters per
-    // tile, zeroed sparse sums, zero x past K
+    // ---- bookkeeping: warp ranges, contributors per tile, zeroed sparse
+    // sums, zero x past K
     if (lane == 0) {
         s_wrange[warp * 3] = wu0;
         s_wrange[warp * 3 + 1] = wu1;
@@ -703,7 +701,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_fused_kernel(const 
             if (max(a, ta_u) < min(b, tb_u)) mask |= 1 << wv;
         }
         s_tinfo[tl] = mask;
-        s_cnt[tl] = 0;
     }
     if (layer_csr) {
         for (int i = tid; i < nrows * CM; i += kThreads) s_rowsum[i] = 0.f;
@@ -811,8 +808,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_fused_kernel(const 
     // ---- sparse part: a fixed share of nonzeros per thread (balanced).
     // Each thread sums its entries per row: the first and last rows it
     // touches go to head/tail pieces, rows it holds entirely to s_rowsum;
-    // then it arrives on rbar.  No CTA barrier: the warp that finishes a
-    // tile waits on rbar and combines the pieces of the tile's rows.
+    // the pieces are combined per row below, then the threads arrive on
+    // rbar, which the writers of y wait on.
     if (has_csr && ca < cb) {
         bool first = true;
         float acc[CM];
@@ -960,8 +957,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_fused_kernel(const 
     };
 
     // Hand this warp's part of `tile` over: written out directly when the
-    // warp holds the whole tile, otherwise into its slot; the last warp to
-    // arrive adds the slots in warp order and writes y.
+    // warp holds the whole tile, otherwise into its slot (the slots of shared
+    // tiles are added in warp order after the loop).
     auto flush_tile = [&]() {
         float rr[NT][4];
         if constexpr (MAC != kMacCuda) {

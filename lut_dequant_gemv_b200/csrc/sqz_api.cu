@@ -78,8 +78,8 @@ struct sqz_layer {
     // The fused kernel serves every layer with N > 0 and K > 0 (columns past
     // K are padded inside the kernel-native layout).
     bool fused_ok = false;
-    // canonical copies (row-per-warp kernel for requests the fused kernel
-    // cannot stage in shared memory)
+    // canonical copies, kept only for layers whose batch-1 calls the fused
+    // kernel cannot serve (the row-per-warp kernel reads them)
     uint32_t* codes = nullptr;
     uint16_t* lut = nullptr;
     // CSR copies, padded by 8 elements so that 16-byte aligned bulk copies
@@ -376,6 +376,8 @@ sqz_status gemv_impl(const sqz_layer* L, const uint16_t* x, int32_t batch, int64
                                                : launch_fused_bits<4>(prm, nb, L->mac, L->csr_mode, s);
             SQZ_CUDA_TRY(e, "fused gemv launch");
         }
+    } else if (!L->codes) {
+        return fail(SQZ_ERR_UNSUPPORTED, "no fused plan for this call and the canonical codes were released");
     } else if (L->bits == 3) {
         dispatch_rowwarp<3>(L, x, batch, ldx, y, ldy, s);
     } else {
@@ -538,6 +540,18 @@ sqz_status sqz_create_layer(const sqz_layer_desc* desc, void* stream, sqz_layer_
     L->fused_ok = L->n_out > 0 && L->k_in > 0 && sqz::tc::grid_size(L->n_out, L->sm_count) <= sqz::tc::kMaxCtas;
     if (L->fused_ok) SQZ_STEP(build_native(L, s));
     SQZ_CUDA_STEP(cudaStreamSynchronize(s), "layer creation");
+    // When the fused kernel serves one batch column, it serves every batch
+    // (larger batches fall back to launches of fewer columns, down to one),
+    // so the canonical codes and LUT -- read only by the row-per-warp kernel
+    // -- are dropped: the handle then holds the compressed weights once.
+    sqz::tc::Plan plan1;
+    if (L->fused_ok && fused_plan(L, 1, &plan1)) {
+        cudaFree(L->codes);
+        cudaFree(L->lut);
+        L->device_bytes -= (int64_t)(code_n * 4 + lut_n * 2);
+        L->codes = nullptr;
+        L->lut = nullptr;
+    }
 #undef SQZ_STEP
 #undef SQZ_CUDA_STEP
     *out = L;
@@ -732,6 +746,9 @@ sqz_status sqz_layer_status(sqz_layer_t layer, void* stream, int32_t* status) {
     SQZ_CUDA_TRY(cudaMemsetAsync(layer->status, 0, sizeof(int), s), "status clear");
     SQZ_CUDA_TRY(cudaStreamSynchronize(s), "stream synchronize");
     *status = h;
+    if (h & sqz::tc::kStatusWaitTimeout)
+        return fail(SQZ_ERR_TIMEOUT, "a bounded device wait gave up (status 0x%x): y of the affected call is undefined",
+                    h);
     return SQZ_OK;
 }
 

@@ -2,17 +2,17 @@
 //
 // sqz_create_layer validates an outlier matrix with a kernel that reports
 // into a flag word it cudaMalloc's for the occasion.  Some callers cannot
-// allocate device memory at the point where they want that check: code that
-// runs while a CUDA graph is being captured (cudaMalloc is not permitted
-// during capture), serving loops that must never take the implicit device
-// synchronisation of cudaMalloc/cudaFree, and runtimes that reserve all of
-// their device memory up front and forbid allocations afterwards.  For them
-// sqz_check_csr_static runs the same validation kernel with its flag word in
-// a fixed, file-scope device array instead.
+// allocate device memory at the point where they want that check: serving
+// loops that must never take the implicit device synchronisation of
+// cudaMalloc/cudaFree, and runtimes that reserve all of their device memory
+// up front and forbid allocations afterwards.  For them sqz_check_csr_static
+// runs the same validation kernel with its flag word in a fixed, file-scope
+// device array instead.  It reads the verdict back and synchronises its
+// stream, so it cannot run inside a CUDA-graph capture: it refuses a stream
+// that is being captured.
 #include <cuda_runtime.h>
 
 #include <cstdio>
-#include <mutex>
 
 #include "../../include/sqz.h"
 #include "kernels_basic.cuh"
@@ -28,12 +28,10 @@ namespace {
 constexpr int kCheckScratchWords = 64;
 __device__ __align__(256) int g_check_scratch[kCheckScratchWords];
 
-// Device address of g_check_scratch, looked up once per device.  In host
-// code the symbol's name is only a host-side stand-in and must never be
-// passed to a kernel.
-constexpr int kMaxDevices = 128;
-std::mutex g_scratch_mu;
-int* g_scratch_addr[kMaxDevices] = {};
+// In host code the symbol's name is only a host-side stand-in and must never
+// be passed to a kernel; its device address is looked up on every call (the
+// address belongs to the current context, which may change between calls;
+// the lookup allocates nothing).
 
 sqz_status fail(sqz_status st, const char* msg) {
     sqz_internal_set_last_error(msg);
@@ -47,19 +45,14 @@ sqz_status cuda_fail(cudaError_t e, const char* what) {
     return fail(SQZ_ERR_CUDA, buf);
 }
 
-// Set-up: resolve the scratch's device address for the current device.
+// The scratch's device address in the current context, and the device.
 sqz_status scratch_of_current_device(int** out, int* device) {
     cudaError_t e = cudaGetDevice(device);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-    if (*device < 0 || *device >= kMaxDevices) return fail(SQZ_ERR_UNSUPPORTED, "device ordinal beyond 127");
-    std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (!g_scratch_addr[*device]) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_check_scratch);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(check scratch)");
-        g_scratch_addr[*device] = static_cast<int*>(p);
-    }
-    *out = g_scratch_addr[*device];
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_check_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(check scratch)");
+    *out = static_cast<int*>(p);
     return SQZ_OK;
 }
 
@@ -75,6 +68,17 @@ extern "C" SQZ_API sqz_status sqz_check_csr_static(const int32_t* rowptr, const 
     if (nnz == 0) return SQZ_OK;  // like sqz_create_layer: nothing to check without outliers
     if (!rowptr || !col) return fail(SQZ_ERR_INVALID_ARG, "nnz > 0 but rowptr or col is NULL");
 
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // The verdict is read back with a synchronisation, which a stream capture
+    // cannot contain: refuse before touching the stream, so the caller's
+    // capture stays intact.
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    cudaError_t e = cudaStreamIsCapturing(s, &cap);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamIsCapturing");
+    if (cap != cudaStreamCaptureStatusNone)
+        return fail(SQZ_ERR_UNSUPPORTED, "the stream is being captured into a CUDA graph; the check reads its "
+                                         "verdict back and synchronises, which a capture cannot contain");
+
     int* scratch = nullptr;
     int device = 0;
     sqz_status st = scratch_of_current_device(&scratch, &device);
@@ -82,9 +86,8 @@ extern "C" SQZ_API sqz_status sqz_check_csr_static(const int32_t* rowptr, const 
     int sms = 148;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess || sms <= 0) sms = 148;
 
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     // The array keeps the previous call's flags: clear the word first.
-    cudaError_t e = cudaMemsetAsync(scratch, 0, sizeof(int), s);
+    e = cudaMemsetAsync(scratch, 0, sizeof(int), s);
     if (e != cudaSuccess) return cuda_fail(e, "clearing the check scratch");
     const int64_t work = nnz > (int64_t)n_out + 1 ? nnz : (int64_t)n_out + 1;
     int64_t blocks = (work + 255) / 256;

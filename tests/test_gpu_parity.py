@@ -435,3 +435,31 @@ def test_status_word_clear_after_runs(B):
     assert B.sqz_layer_status(layer) == 0
     with pytest.raises(B.SqzError):
         B.sqz_layer_set_mac(layer, 7)
+
+
+@pytest.mark.parametrize("wl", ["llama7b-up-3bit", "llama7b-q-4bit"])
+def test_layer_holds_the_compressed_weights_once(B, wl):
+    """A handle's device memory is the compressed layer (codes, LUTs, CSR)
+    once, in the kernel's layout, plus the fixed staging buffers of the host
+    entry point (16 columns of x and of y): no second copy of the weights
+    (summary page §5 "Inference Latency and Memory Benchmarking", Table 3:
+    the memory footprint is the point of the method)."""
+    from lut_dequant_gemv_b200 import accounting as acc
+
+    shape = synth.workloads()[wl][0]
+    L = synth.layer_for(shape)
+    layer = upload(B, L)
+    info = B.sqz_layer_info(layer)
+    weights = (acc.code_bytes(L.n_out, L.k_in, L.bits) + acc.lut_bytes(L.n_out, L.bits)
+               + acc.csr_bytes(L.n_out, L.nnz))
+    staging = 2 * 16 * (L.k_in + L.n_out)
+    assert info["device_bytes"] <= 1.05 * (weights + staging), (info["device_bytes"], weights, staging)
+    # and it still computes the product
+    x = synth.x_for(shape)
+    y16 = gpu_gemv(B, layer, x)
+    import oracle
+
+    rows = np.arange(0, L.n_out, 97, dtype=np.int32)
+    y_ref, bound = oracle.default().gemv_layer(L, x, rows=rows)
+    assert_close(y16[:, rows], y_ref, bound, wl)
+    layer.close()

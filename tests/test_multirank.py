@@ -79,3 +79,36 @@ def test_single_rank_helpers_need_no_process_group():
     assert bench.max_over_ranks(3.5, 1) == 3.5
     assert bench.whole_job_gbs(1, 2_000_000, 4, 8.0) == pytest.approx(2_000_000 * 4 / 0.008 / 1e9)
     assert bench.instance_id(0, 3) != bench.instance_id(1, 3)
+
+
+def test_gpus_flag_spawns_that_many_ranks():
+    """`bench.py --gpus 2` outside torchrun starts two ranks itself (here in
+    the CPU self-test mode: gloo, fixed per-rank times): rank 0 alone prints,
+    n_gpus is the real world size and the time is the slowest rank's."""
+    import json
+    import subprocess
+
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--steps", "10",
+                          "--selftest-ranks"], capture_output=True, text=True, timeout=180, env=env, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, out.stdout
+    rec = json.loads(lines[0])
+    assert rec["n_gpus"] == 2
+    assert rec["ms"] == 20.0
+    assert rec["value"] == pytest.approx(2 * 1_000_000 * 10 / 0.020 / 1e9)
+
+
+def test_bench_step_is_a_stack_of_layers_larger_than_l2():
+    sys.path.insert(0, ROOT)
+    import bench
+
+    l2 = 126 * 1024 * 1024
+    # the 18.4 MB bench layer: 32 layers (590 MB) already exceed 4x L2
+    assert bench.stack_depth(l2, 18_376_054) == 32
+    # the 9 MB 4096x4096 4-bit layer needs more than 32 to reach 4x L2
+    r = bench.stack_depth(l2, 9_004_678)
+    assert r > 32 and r * 9_004_678 >= 4 * l2
+    assert bench.graph_plan(20, 16) == (1, 4)
+    assert bench.graph_plan(32, 16) == (2, 0)

@@ -1,7 +1,6 @@
 """sqz_check_csr_static: the CSR check for callers that cannot allocate
-device memory (code running during CUDA-graph capture, serving loops that
-must avoid cudaMalloc's implicit synchronisation, runtimes with all device
-memory reserved up front).
+device memory (serving loops that must avoid cudaMalloc's implicit
+synchronisation, runtimes with all device memory reserved up front).
 
 Its verdict must equal the one sqz_create_layer reaches with its own,
 allocating, check on the same arrays -- on consecutive calls, since every
@@ -110,3 +109,29 @@ def test_static_check_on_a_side_stream(B):
     with torch.cuda.stream(s):
         assert B.sqz_check_csr_static(rp, bad, L.n_out, L.k_in, stream=s) == 8
         assert B.sqz_check_csr_static(rp, col, L.n_out, L.k_in, stream=s) == 0
+
+
+def test_static_check_refuses_a_capturing_stream(B):
+    """The check reads its verdict back and synchronises, which a graph
+    capture cannot contain: on a capturing stream it must return
+    SQZ_ERR_UNSUPPORTED without enqueuing anything, and the capture must
+    still end cleanly and replay."""
+    L = synth.make_layer(64, 256, 3, 0.02, seed=9, key="noalloc-capture")
+    rp, col = torch.from_numpy(L.rowptr).cuda(), torch.from_numpy(L.col).cuda()
+    out = torch.zeros(4, device="cuda")
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            out.add_(1.0)
+            with pytest.raises(B.SqzError) as ei:
+                B.sqz_check_csr_static(rp, col, L.n_out, L.k_in, stream=s)
+            assert ei.value.status == B.SQZ_ERR_UNSUPPORTED
+            assert "captured" in str(ei.value)
+            out.add_(1.0)
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.all(out == 2.0)
+    # outside the capture the same call works and clears what it finds
+    assert B.sqz_check_csr_static(rp, col, L.n_out, L.k_in) == 0
