@@ -186,6 +186,19 @@ SQZ_API sqz_status sqz_layer_set_mac(sqz_layer_t layer, int32_t mac);
 SQZ_API sqz_status sqz_layer_set_csr_mode(sqz_layer_t layer, int32_t mode);
 
 /*
+ * Batches of 1..8 columns take, by default (enable = 1), the kernel that
+ * decodes the first code units of every warp into tensor memory while it
+ * waits for the previous kernel of the stream and for x, and multiplies them
+ * once x has arrived (the dependency wait is dead time otherwise).  enable = 0
+ * selects the kernel without that step, for comparison; both give results
+ * within the same bound (only the order of additions differs).  The choice
+ * applies with the default MAC unit and CSR mode.  Not thread-safe against
+ * concurrent sqz_gemv calls on the same handle.
+ * Errors: SQZ_ERR_INVALID_ARG.
+ */
+SQZ_API sqz_status sqz_layer_set_predecode(sqz_layer_t layer, int32_t enable);
+
+/*
  * Read and clear the handle's device status word, ordered on `stream`
  * (synchronises it).  *status receives the word: 0 means every call so far
  * completed normally; bit 0 (1) means a bounded wait for a copy into shared
@@ -210,14 +223,16 @@ SQZ_API sqz_status sqz_layer_info(sqz_layer_t layer, int32_t* n_out, int32_t* k_
  * shared memory (ctas_per_sm = 2 when two CTAs share an SM), x staged in
  * `passes` chunks of K, a code ring of ring_stages stages per warp and up to
  * csr_stage_entries outliers per CTA staged in shared memory (the first
- * launch's plan; a shorter last launch may differ).  No counterpart in the
- * paper: it exposes this library's own scheduling.
+ * launch's plan; a shorter last launch may differ).  predecode = 1 when the
+ * call takes the decode-ahead kernel (sqz_layer_set_predecode; this query
+ * assumes the handle's default options).  No counterpart in the paper: it
+ * exposes this library's own scheduling.
  * Errors: SQZ_ERR_INVALID_ARG for a NULL out, bits not in {3,4}, n_out or k_in
  * < 1, batch outside [1,16], or a non-positive device figure.
  */
 typedef struct {
     int32_t fused, columns_per_launch, launches, grid, threads, ctas_per_sm, smem_bytes, passes, ring_stages,
-        csr_stage_entries;
+        csr_stage_entries, predecode;
 } sqz_plan_info;
 SQZ_API sqz_status sqz_plan_query(int32_t n_out, int32_t k_in, int32_t bits, int32_t batch, int32_t sm_count,
                                   int32_t smem_per_sm, int32_t smem_optin, sqz_plan_info* out);

@@ -38,7 +38,7 @@ STATUS_NAMES = {0: "SQZ_OK", 1: "SQZ_ERR_INVALID_ARG", 2: "SQZ_ERR_UNSUPPORTED",
 EXPORTED = ("sqz_create_layer", "sqz_gemv", "sqz_gemv_host", "sqz_debug_dequant", "sqz_layer_info",
             "sqz_destroy", "sqz_fp16_gemv", "sqz_last_error", "sqz_version", "sqz_check_csr_static",
             "sqz_layer_set_mac", "sqz_layer_set_csr_mode", "sqz_layer_status", "sqz_encode",
-            "sqz_encode_outliers", "sqz_plan_query")
+            "sqz_encode_outliers", "sqz_plan_query", "sqz_layer_set_predecode")
 
 
 class SqzError(RuntimeError):
@@ -50,7 +50,7 @@ class SqzError(RuntimeError):
 class sqz_plan_info(ctypes.Structure):
     _fields_ = [(name, ctypes.c_int32) for name in (
         "fused", "columns_per_launch", "launches", "grid", "threads", "ctas_per_sm", "smem_bytes", "passes",
-        "ring_stages", "csr_stage_entries")]
+        "ring_stages", "csr_stage_entries", "predecode")]
 
 
 class sqz_layer_desc(ctypes.Structure):
@@ -93,6 +93,8 @@ def lib() -> ctypes.CDLL:
         L.sqz_layer_set_mac.restype = ctypes.c_int
         L.sqz_layer_set_csr_mode.argtypes = [P, i32]
         L.sqz_layer_set_csr_mode.restype = ctypes.c_int
+        L.sqz_layer_set_predecode.argtypes = [P, i32]
+        L.sqz_layer_set_predecode.restype = ctypes.c_int
         L.sqz_layer_status.argtypes = [P, P, ctypes.POINTER(i32)]
         L.sqz_layer_status.restype = ctypes.c_int
         L.sqz_check_csr_static.argtypes = [P, P, i32, i32, i64, P, ctypes.POINTER(i32)]
@@ -353,6 +355,10 @@ def sqz_layer_set_mac(layer: Layer, mac: int) -> None:
 
 def sqz_layer_set_csr_mode(layer: Layer, mode: int) -> None:
     _check(lib().sqz_layer_set_csr_mode(layer, int(mode)), "sqz_layer_set_csr_mode")
+
+
+def sqz_layer_set_predecode(layer: Layer, enable: bool) -> None:
+    _check(lib().sqz_layer_set_predecode(layer, int(bool(enable))), "sqz_layer_set_predecode")
 
 
 def sqz_layer_status(layer: Layer, stream=None) -> int:

@@ -1,0 +1,643 @@
+// kernels_pd.cuh -- the fused Dense-and-Sparse GEMV with weights decoded into
+// tensor memory ahead of the activations (batches of 1..8 columns).
+//
+// y = (Q + S) x ("SqueezeLLM: Dense-and-Sparse Quantization", summary page,
+// §3.4 "Kernel Implementation": LUT-based dense kernel, balanced sparse
+// kernel, both fused into one launch).
+//
+// Why: a call cannot use x before the previous kernel of the stream has
+// finished (programmatic dependent launch, griddepcontrol.wait), and on B200
+// that wait returns about a microsecond after the previous grid's last CTA
+// exits; x then takes a few hundred nanoseconds more to arrive.  The dense
+// part's cost is the LUT decode (byte permutes on the integer pipe), and the
+// decode needs only the codes and the LUTs -- never x.  So every warp decodes
+// its first code units while it waits, and parks their MMA A fragments in
+// tensor memory (TMEM: 256 KB per SM that this path would otherwise leave
+// unused; a tcgen05.st of a quad of k16-steps is nearly free next to the
+// decode).  When x lands the warp stops decoding ahead (it checks the x
+// barrier before every quad, without blocking), runs the MMAs of the
+// fragments it parked (tcgen05.ld + mma.sync, about a third of the cost of
+// decoding), and then decodes the rest of its units as usual.
+//
+// Work decomposition
+//   * Rows in tiles of 16 (the M of an m16n8k16 MMA), columns in
+//     super-groups of 256 (16 k16-steps); a unit = (tile, super-group).  The
+//     code layout and decoder are those of kernels_tc.cuh.
+//   * One CTA per SM (the whole register file): 16 dense warps and one
+//     control warp.  A CTA owns a contiguous run of whole tiles; its dense
+//     warps split the CTA's units into 16 contiguous, equal ranges.
+//   * The control warp requests the LUT planes, the rowptr slice and the
+//     CSR entries of the CTA (bulk copies), asks L2 for the CTA's whole code
+//     range (the HBM streams it while the SMs wait for the previous kernel),
+//     allocates TMEM, waits for the previous kernel, copies x in and sums the
+//     sparse part: the CTA's nonzeros split evenly over its 32 lanes (the
+//     balanced scheme), the pieces of rows cut between lanes added in lane
+//     order.
+//   * Tiles held whole by a warp are written by it; tiles split between
+//     warps are finished after one CTA barrier, the warps' parts added in
+//     warp order.  Every summation order is fixed: results are bitwise
+//     reproducible, and a column of a batch equals the batch-1 call on it.
+//
+// TMEM: warp w reaches the 32 lanes of quarter w % 4 (lane = the warp's
+// lane); its columns are [(w / 4) * 128, +128): two units of 64 columns (a
+// quad of 4 k16-steps = 16 columns of A fragments).  The control warp
+// allocates all 512 columns at the start and frees them after the last
+// tcgen05.ld, on every path.  A CTA takes the whole register file and more
+// than half of the shared memory, so no second CTA of this kernel can be
+// resident on the SM and wait for its TMEM.
+//
+// Every wait on a copy or mbarrier is bounded and records a status bit
+// instead of hanging.
+#pragma once
+
+#include "kernels_tc.cuh"
+
+namespace sqz {
+namespace pd {
+
+using tc::Fmt;
+using tc::kSgCols;
+using tc::kSgSteps;
+using tc::kTileRows;
+using tc::round_up;
+using tc::tile_begin;
+
+constexpr int kDenseWarps = 16;
+constexpr int kCtrlWarp = kDenseWarps;       // warp 16
+constexpr int kThreads = (kDenseWarps + 1) * 32;
+constexpr int kStages = 4;                   // code ring stages per dense warp
+constexpr int kPreUnits = 2;                 // units per warp that can be parked in TMEM
+constexpr int kTmemCols = 512;
+constexpr int kCsrCap = 4096;                // CSR entries per CTA staged in shared memory
+constexpr int kMinSmem = 120 * 1024;         // more than half an SM: one CTA per SM
+
+struct Plan {
+    int grid, ctiles_max, x_stride, cm, csr_cap;
+    int off_taddr, off_x, off_lut, off_rp, off_rowsum, off_head, off_tail, off_headrow, off_tailrow, off_slots,
+        off_tinfo, off_col, off_val, off_ring, total;
+};
+
+// Shared-memory plan of a launch; total > budget when it does not fit.
+__host__ __device__ inline Plan make_plan(int bits, int n_out, int k_in, int batch, int sms, int budget) {
+    Plan P{};
+    const int ntiles = (n_out + kTileRows - 1) / kTileRows;
+    const int nsg = ((k_in + 15) / 16 + kSgSteps - 1) / kSgSteps;
+    const int lut_bytes = bits == 3 ? 16 : 32;
+    const int sg_bytes = bits == 3 ? 1536 : 2048;
+    P.grid = tc::grid_size(n_out, sms);
+    P.ctiles_max = (ntiles + P.grid - 1) / P.grid;
+    P.cm = batch == 1 ? 1 : 8;
+    // x rows: stride = 32 (mod 128) bytes keeps the batch rows of one
+    // fragment load in different banks
+    const int xs_bytes = round_up(nsg * kSgCols * 2, 128) + 32;
+    P.x_stride = xs_bytes / 2;
+    const int rows = P.ctiles_max * kTileRows;
+    int off = 128;  // mbarriers
+    P.off_taddr = 64;
+    P.off_x = off;
+    off += round_up(batch * xs_bytes, 128);
+    P.off_lut = off;
+    off += round_up(rows * lut_bytes, 128);
+    P.off_rp = off;
+    off += round_up((rows + 8) * 4, 128);
+    P.off_rowsum = off;
+    off += round_up(rows * P.cm * 4, 128);
+    P.off_head = off;
+    P.off_tail = off + 32 * P.cm * 4;
+    P.off_headrow = P.off_tail + 32 * P.cm * 4;
+    P.off_tailrow = P.off_headrow + 32 * 4;
+    off += round_up(2 * 32 * P.cm * 4 + 2 * 32 * 4, 128);
+    P.off_slots = off;
+    off += round_up(kDenseWarps * 2 * kTileRows * P.cm * 4, 128);
+    P.off_tinfo = off;
+    off += round_up(P.ctiles_max * 4, 128);
+    const int ring = kStages * kDenseWarps * sg_bytes;
+    int cap = (budget - off - ring - 512) / 6;
+    cap = cap > kCsrCap ? kCsrCap : cap;
+    P.csr_cap = cap < 0 ? 0 : cap & ~7;
+    P.off_col = off;  // a slice starts up to 3 entries early and is rounded up to 4
+    off += round_up((P.csr_cap + 8) * 4, 128);
+    P.off_val = off;  // up to 7 entries early, rounded up to 8
+    off += round_up((P.csr_cap + 16) * 2, 128);
+    P.off_ring = off;
+    off += ring;
+    P.total = off < kMinSmem ? kMinSmem : off;
+    return P;
+}
+
+struct Params {
+    const uint8_t* codes;    // [ntiles][nsg][sg_bytes], kernel-native layout
+    int n_out, k_in, nsg, ntiles, batch;
+    int has_csr;
+    int x_bulk;              // 1: every x row is 16-byte aligned -> bulk copies
+    Plan plan;
+    const uint8_t* lutp;     // [ntiles*16][lut_bytes] byte planes
+    const int32_t* rowptr;
+    const int32_t* col;
+    const uint16_t* val;
+    const uint16_t* x;
+    int64_t ldx;
+    uint16_t* y;
+    int64_t ldy;
+    int* status;
+    const int32_t* csr_cta;  // [grid + 1]: CSR entry range of each CTA's rows
+};
+
+// ---------------------------------------------------------------- helpers
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(ok)
+        : "r"(tc::smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t cols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(tc::smem_u32(dst)),
+                 "r"(cols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t cols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(cols) : "memory");
+}
+__device__ __forceinline__ void tmem_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tmem_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+// 16 consecutive 32-bit columns of the warp's 32 lanes (one value per lane each)
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+        "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+          "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// The A fragments of quad q (k16-steps 4q..4q+3) of a unit: a[4j..4j+3] =
+// (a0, a1, a2, a3) of step 4q+j.
+template <int BITS, class TAB>
+__device__ __forceinline__ void decode_quad(const TAB& tg, const TAB& tg8, const uint32_t (&w)[4 * Fmt<BITS>::kVecs],
+                                            int q, uint32_t (&a)[16]) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        tc::decode_step<BITS>(tg, tg8, w, 4 * q + j, a[4 * j], a[4 * j + 1], a[4 * j + 2], a[4 * j + 3]);
+}
+
+// ------------------------------------------------------------ main kernel
+// SB: batch 1 (one column carried through the sparse part and the combine).
+template <int BITS, bool SB>
+__global__ void __launch_bounds__(kThreads, 1) gemv_pd_kernel(const __grid_constant__ Params p) {
+    using F = Fmt<BITS>;
+    using TAB = typename std::conditional<BITS == 3, tc::Tab3, tc::Tab4>::type;
+    constexpr int CM = SB ? 1 : 8;           // batch columns carried after the dense loop
+    constexpr int TE = kTileRows * CM;       // elements of one tile's result
+    constexpr int V = F::kVecs;
+    constexpr int S = kStages, D = kStages - 1;
+    extern __shared__ __align__(128) uint8_t smem[];
+    const Plan& P = p.plan;
+
+    tc::pdl_launch_dependents();
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t4 = lane & 3;
+    const bool ctrl = warp == kCtrlWarp;
+    const int G = gridDim.x, c = blockIdx.x;
+    const int nsg = p.nsg;
+    const int t_first = tile_begin(p.ntiles, G, c), t_end = tile_begin(p.ntiles, G, c + 1);
+    const int ctiles = t_end - t_first;
+    const int u0 = t_first * nsg, cn = ctiles * nsg;
+    // dense warp w: units [wu0, wu1) of the CTA, contiguous and equal
+    const int wsel = ctrl ? 0 : warp;
+    const int wu0 = u0 + cn * wsel / kDenseWarps, wu1 = u0 + cn * (wsel + 1) / kDenseWarps;
+    const int nwu = ctrl ? 0 : wu1 - wu0;
+    const int wfirst = nwu > 0 ? wu0 / nsg : -1;
+    const int ra = min(p.n_out, t_first * kTileRows);
+    const int nrows = min(p.n_out, t_end * kTileRows) - ra;
+    const bool layer_csr = p.has_csr != 0;
+
+    uint64_t* lbar = reinterpret_cast<uint64_t*>(smem);      // LUT planes + rowptr slice
+    uint64_t* xbar = reinterpret_cast<uint64_t*>(smem) + 1;  // x
+    uint64_t* cbar = reinterpret_cast<uint64_t*>(smem) + 2;  // CSR slices
+    uint64_t* rbar = reinterpret_cast<uint64_t*>(smem) + 3;  // sparse sums complete (32 arrivals)
+    uint32_t* s_taddr = reinterpret_cast<uint32_t*>(smem + P.off_taddr);
+    uint16_t* xs = reinterpret_cast<uint16_t*>(smem + P.off_x);
+    uint8_t* luts = smem + P.off_lut;
+    float* s_rowsum = reinterpret_cast<float*>(smem + P.off_rowsum);
+    float* s_head = reinterpret_cast<float*>(smem + P.off_head);
+    float* s_tail = reinterpret_cast<float*>(smem + P.off_tail);
+    int* s_headrow = reinterpret_cast<int*>(smem + P.off_headrow);
+    int* s_tailrow = reinterpret_cast<int*>(smem + P.off_tailrow);
+    float* s_slots = reinterpret_cast<float*>(smem + P.off_slots);
+    int* s_tinfo = reinterpret_cast<int*>(smem + P.off_tinfo);  // [tile] = mask of dense warps holding parts
+    const int rp_off = ra & 3;
+    const int* s_rp = reinterpret_cast<const int*>(smem + P.off_rp) + rp_off;  // s_rp[i] = rowptr[ra + i]
+    const int B = p.batch;
+
+    // ---- control warp: barriers, copies of the weights (independent of the
+    // previous kernel), the L2 prefetch of the CTA's codes, TMEM
+    if (ctrl) {
+        if (lane == 0) {
+            tc::mbar_init(lbar, 1);
+            tc::mbar_init(xbar, p.x_bulk ? 1 : 32);  // bulk: one expect_tx; else every lane after its stores
+            tc::mbar_init(cbar, 1);
+            tc::mbar_init(rbar, 32);
+            tc::fence_mbar_init();
+            const uint32_t lut_bytes = (uint32_t)ctiles * kTileRows * F::kLutBytes;
+            const uint32_t rp_bytes = layer_csr ? (uint32_t)round_up(nrows + 1 + rp_off, 4) * 4 : 0u;
+            tc::mbar_expect_tx(lbar, lut_bytes + rp_bytes);
+            tc::bulk_g2s(luts, p.lutp + (int64_t)t_first * kTileRows * F::kLutBytes, lut_bytes, lbar);
+            if (rp_bytes) tc::bulk_g2s(smem + P.off_rp, p.rowptr + (ra - rp_off), rp_bytes, lbar);
+            const int q0 = __ldg(p.csr_cta + c), nz = __ldg(p.csr_cta + c + 1) - q0;
+            const bool csr_in_smem = nz > 0 && nz <= P.csr_cap;
+            const uint32_t col_bytes = csr_in_smem ? (uint32_t)round_up(nz + (q0 & 3), 4) * 4 : 0u;
+            const uint32_t val_bytes = csr_in_smem ? (uint32_t)round_up(nz + (q0 & 7), 8) * 2 : 0u;
+            tc::mbar_expect_tx(cbar, col_bytes + val_bytes);
+            if (col_bytes) tc::bulk_g2s(smem + P.off_col, p.col + (q0 - (q0 & 3)), col_bytes, cbar);
+            if (val_bytes) tc::bulk_g2s(smem + P.off_val, p.val + (q0 - (q0 & 7)), val_bytes, cbar);
+        }
+        // every code unit of the CTA into L2 (one unit per lane and request)
+        for (int u = lane; u < cn; u += 32) prefetch_l2(p.codes + (int64_t)(u0 + u) * F::kSgBytes, F::kSgBytes);
+        __syncwarp();
+        tmem_alloc(s_taddr, kTmemCols);
+    }
+
+    // ---- dense warps: the first D units of the warp's code ring
+    uint8_t* ring = smem + P.off_ring + (ctrl ? 0 : warp) * S * F::kSgBytes + lane * 16;
+    int pj = wu0;  // next unit to request
+    auto issue = [&](int stage) {
+        if (pj < wu1) {
+            const uint8_t* src = p.codes + (int64_t)pj * F::kSgBytes + lane * 16;
+            uint8_t* dst = ring + stage * F::kSgBytes;
+#pragma unroll
+            for (int m = 0; m < V; ++m) tc::cp_async16(dst + m * 512, src + m * 512);
+            ++pj;
+        }
+        tc::cp_async_commit();
+    };
+    if (!ctrl)
+        for (int j = 0; j < D; ++j) issue(j);
+
+    // ---- bookkeeping: contributors per tile, zeroed sparse sums, zero x past K
+    for (int tl = tid; tl < ctiles; tl += kThreads) {
+        const int ta_u = (t_first + tl) * nsg, tb_u = ta_u + nsg;
+        int mask = 0;
+        for (int wv = 0; wv < kDenseWarps; ++wv) {
+            const int a = u0 + cn * wv / kDenseWarps, b = u0 + cn * (wv + 1) / kDenseWarps;
+            if (max(a, ta_u) < min(b, tb_u)) mask |= 1 << wv;
+        }
+        s_tinfo[tl] = mask;
+    }
+    if (layer_csr)
+        for (int i = tid; i < nrows * CM; i += kThreads) s_rowsum[i] = 0.f;
+    {
+        const int len = p.k_in, pad = nsg * kSgCols - len;
+        for (int i = tid; i < B * pad; i += kThreads) {
+            const int b = i / pad;
+            xs[b * P.x_stride + len + (i - b * pad)] = 0;
+        }
+    }
+    tmem_fence_before();
+    __syncthreads();
+    tmem_fence_after();
+    const uint32_t taddr = *s_taddr;
+
+    bool csr_ready = !layer_csr;
+    if (ctrl) {
+        // ---- x may be written by the previous kernel of the stream: wait
+        // for it (its lines were requested into L2 first: a hint only)
+        {
+            const int lines = (p.k_in * 2 + 127) / 128;
+            for (int b = 0; b < B; ++b) {
+                const char* xr = reinterpret_cast<const char*>(p.x + b * p.ldx);
+                for (int l = lane; l < lines; l += 32) asm volatile("prefetch.global.L2 [%0];" ::"l"(xr + l * 128));
+            }
+        }
+        tc::pdl_wait_previous();
+        if (p.x_bulk) {
+            if (lane == 0) {
+                tc::mbar_expect_tx(xbar, (uint32_t)B * p.k_in * 2);
+                for (int b = 0; b < B; ++b) tc::bulk_g2s(xs + b * P.x_stride, p.x + b * p.ldx, p.k_in * 2, xbar);
+            }
+        } else {
+            for (int i = lane; i < B * p.k_in; i += 32) {
+                const int b = i / p.k_in, k = i - b * p.k_in;
+                xs[b * P.x_stride + k] = p.x[b * p.ldx + k];
+            }
+            tc::mbar_arrive(xbar);  // release: this lane's x stores before the phase completes
+        }
+        const bool got = tc::mbar_wait(lbar, 0) && tc::mbar_wait(xbar, 0) && tc::mbar_wait(cbar, 0);
+        if (!got) atomicOr(p.status, tc::kStatusWaitTimeout);
+
+        // ---- sparse part: the CTA's entries [q0, q1) split evenly over the
+        // 32 lanes; a lane's first and last rows go to its head/tail pieces,
+        // rows it holds whole straight to s_rowsum
+        const int q0 = __ldg(p.csr_cta + c), q1 = __ldg(p.csr_cta + c + 1);
+        const int nz = q1 - q0;
+        if (nz > 0) {
+            const bool in_smem = nz <= P.csr_cap;
+            const int* csr_col = in_smem ? reinterpret_cast<const int*>(smem + P.off_col) + (q0 & 3) - q0 : p.col;
+            const uint16_t* csr_val =
+                in_smem ? reinterpret_cast<const uint16_t*>(smem + P.off_val) + (q0 & 7) - q0 : p.val;
+            const int e_per = (nz + 31) / 32;
+            const int ca = (int)min((int64_t)q1, (int64_t)q0 + (int64_t)lane * e_per);
+            const int cb = (int)min((int64_t)q1, (int64_t)ca + e_per);
+            s_headrow[lane] = -1;
+            s_tailrow[lane] = -1;
+            if (ca < cb) {
+                int lo = 0, hi = nrows - 1;  // row (relative to ra) of entry ca
+                while (lo < hi) {
+                    const int mid = (lo + hi + 1) >> 1;
+                    if (s_rp[mid] <= ca) lo = mid; else hi = mid - 1;
+                }
+                int cur = lo, nxt = s_rp[cur + 1];
+                bool first = true;
+                float acc[CM];
+#pragma unroll
+                for (int b = 0; b < CM; ++b) acc[b] = 0.f;
+                auto emit = [&](bool last) {
+                    float* dstp;
+                    if (first) {
+                        s_headrow[lane] = cur;
+                        dstp = s_head + lane * CM;
+                    } else if (last) {
+                        s_tailrow[lane] = cur;
+                        dstp = s_tail + lane * CM;
+                    } else {
+                        dstp = s_rowsum + cur * CM;
+                    }
+#pragma unroll
+                    for (int b = 0; b < CM; ++b) dstp[b] = acc[b];
+                };
+                for (int base = ca; base < cb; base += 8) {
+                    int cc[8];
+                    uint32_t vh[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int q = base + j;
+                        const bool in = q < cb;
+                        cc[j] = in ? csr_col[q] : 0;
+                        vh[j] = in ? (uint32_t)csr_val[q] : 0u;
+                    }
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int q = base + j;
+                        if (q >= cb) break;
+                        while (q >= nxt) {
+                            emit(false);
+                            first = false;
+#pragma unroll
+                            for (int b = 0; b < CM; ++b) acc[b] = 0.f;
+                            ++cur;
+                            nxt = s_rp[cur + 1];
+                        }
+                        const float v = h2f((uint16_t)vh[j]);
+#pragma unroll
+                        for (int b = 0; b < CM; ++b)
+                            if (SB || b < B) acc[b] = fmaf(v, h2f(xs[b * P.x_stride + cc[j]]), acc[b]);
+                    }
+                }
+                emit(true);
+            }
+            __syncwarp();
+            // rows cut between lanes: the interior sum plus the pieces of the
+            // lanes whose shares cut the row, in lane order
+            for (int i = lane; i < nrows; i += 32) {
+                const int rs = s_rp[i], re = s_rp[i + 1];
+                if (re <= rs) continue;
+                float cs[CM];
+#pragma unroll
+                for (int b = 0; b < CM; ++b) cs[b] = s_rowsum[i * CM + b];
+                const int tau_a = (rs - q0) / e_per, tau_b = min(31, (re - 1 - q0) / e_per);
+                for (int tau = tau_a; tau <= tau_b; ++tau) {
+                    if (s_headrow[tau] == i) {
+#pragma unroll
+                        for (int b = 0; b < CM; ++b) cs[b] += s_head[tau * CM + b];
+                    }
+                    if (s_tailrow[tau] == i) {
+#pragma unroll
+                        for (int b = 0; b < CM; ++b) cs[b] += s_tail[tau * CM + b];
+                    }
+                }
+#pragma unroll
+                for (int b = 0; b < CM; ++b) s_rowsum[i * CM + b] = cs[b];
+            }
+        }
+        tc::mbar_arrive(rbar);  // release: this lane's sparse sums before the phase completes
+    }
+
+    // The sparse sum of row ra+i, batch column col.
+    auto csr_row_sum = [&](int i, int col) -> float {
+        if (!layer_csr) return 0.f;
+        if (!csr_ready) {
+            if (!tc::mbar_wait(rbar, 0)) atomicOr(p.status, tc::kStatusWaitTimeout);
+            csr_ready = true;
+        }
+        return s_rowsum[i * CM + col];
+    };
+
+    // ---- dense warps
+    if (!ctrl && nwu > 0) {
+        // this warp's TMEM: lanes of quarter warp % 4, columns (warp / 4) * 128 ...
+        const uint32_t tw = taddr + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)((warp >> 2) * 128);
+        TAB tg, tg8;
+        auto load_tabs = [&](int tile) {
+            const uint8_t* lt = luts + (tile - t_first) * kTileRows * F::kLutBytes;
+            if constexpr (BITS == 3) {
+                tg = tc::load_tab3(lt + g * F::kLutBytes);
+                tg8 = tc::load_tab3(lt + (g + 8) * F::kLutBytes);
+            } else {
+                tg = tc::load_tab4(lt + g * F::kLutBytes);
+                tg8 = tc::load_tab4(lt + (g + 8) * F::kLutBytes);
+            }
+        };
+        auto read_stage = [&](int s, uint32_t (&w)[4 * V]) {
+            const uint8_t* src = ring + s * F::kSgBytes;
+#pragma unroll
+            for (int m = 0; m < V; ++m) {
+                const uint4 v = *reinterpret_cast<const uint4*>(src + m * 512);
+                w[4 * m] = v.x, w[4 * m + 1] = v.y, w[4 * m + 2] = v.z, w[4 * m + 3] = v.w;
+            }
+        };
+        auto x_arrived = [&]() -> bool {
+            const bool t = lane == 0 ? mbar_test(xbar, 0) : false;
+            return __shfl_sync(0xffffffffu, t, 0);
+        };
+        if (!tc::mbar_wait(lbar, 0)) atomicOr(p.status, tc::kStatusWaitTimeout);
+        __syncwarp();
+
+        // ---- ahead of x: decode the first units' quads into TMEM until x
+        // is in shared memory (checked before every quad)
+        int qp = 0;  // quads parked
+        int s_read = 0, s_fill = D;
+        {
+            const int pre = min(nwu, kPreUnits);
+            int tab_tile = -1;
+            bool stop = false;
+            for (int u = 0; u < pre && !stop; ++u) {
+                if (x_arrived()) break;
+                tc::cp_async_wait<S - 2>();
+                uint32_t w[4 * V];
+                read_stage(s_read, w);
+                const int tile = (wu0 + u) / nsg;
+                if (tile != tab_tile) {
+                    load_tabs(tile);
+                    tab_tile = tile;
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    if (q > 0 && x_arrived()) {
+                        stop = true;
+                        break;
+                    }
+                    uint32_t a[16];
+                    decode_quad<BITS>(tg, tg8, w, q, a);
+                    tmem_st16(tw + (uint32_t)(64 * u + 16 * q), a);
+                    ++qp;
+                }
+                if (!stop) {  // the unit is parked whole: its stage is free
+                    issue(s_fill);
+                    s_read = s_read + 1 == S ? 0 : s_read + 1;
+                    s_fill = s_fill + 1 == S ? 0 : s_fill + 1;
+                }
+            }
+            tmem_wait_st();
+        }
+        if (!tc::mbar_wait(xbar, 0)) atomicOr(p.status, tc::kStatusWaitTimeout);
+        __syncwarp();
+
+        // ---- every unit in order: parked quads from TMEM, the rest decoded
+        const int xrow = g < B ? g : 0;  // batch column of this lane's B fragment (n = g)
+        float d0[4], d1[4];
+        int tile = wfirst, sg = wu0 - wfirst * nsg;
+        auto start_tile = [&]() {
+            load_tabs(tile);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) d0[q] = d1[q] = 0.f;
+        };
+        auto out = [&](int row, int col, float v) {
+            if (row < p.n_out && col < B) p.y[col * p.ldy + row] = f2h_rn(v + csr_row_sum(row - ra, col));
+        };
+        auto flush_tile = [&]() {
+            float rr[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) rr[q] = d0[q] + d1[q];
+            const int tl = tile - t_first;
+            const int row0 = tile * kTileRows;
+            const int mask = s_tinfo[tl];
+            if ((mask & (mask - 1)) == 0) {
+                if constexpr (SB) {
+                    if (t4 == 0) {
+                        out(row0 + g, 0, rr[0]);
+                        out(row0 + g + 8, 0, rr[2]);
+                    }
+                } else {
+                    const int col = 2 * t4;
+                    out(row0 + g, col, rr[0]);
+                    out(row0 + g, col + 1, rr[1]);
+                    out(row0 + g + 8, col, rr[2]);
+                    out(row0 + g + 8, col + 1, rr[3]);
+                }
+                return;
+            }
+            float* dst = s_slots + (warp * 2 + (tile == wfirst ? 0 : 1)) * TE;
+            if constexpr (SB) {
+                if (t4 == 0) {
+                    dst[g] = rr[0];
+                    dst[g + 8] = rr[2];
+                }
+            } else {
+                const int col = 2 * t4;
+                dst[g * CM + col] = rr[0];
+                dst[g * CM + col + 1] = rr[1];
+                dst[(g + 8) * CM + col] = rr[2];
+                dst[(g + 8) * CM + col + 1] = rr[3];
+            }
+        };
+        start_tile();
+#pragma unroll 1
+        for (int u = 0; u < nwu; ++u) {
+            const int tq = min(4, max(0, qp - 4 * u));  // quads of this unit parked in TMEM
+            uint32_t w[4 * V];
+            if (tq < 4) {
+                tc::cp_async_wait<S - 2>();
+                read_stage(s_read, w);
+                issue(s_fill);
+                s_read = s_read + 1 == S ? 0 : s_read + 1;
+                s_fill = s_fill + 1 == S ? 0 : s_fill + 1;
+            } else {
+#pragma unroll
+                for (int i = 0; i < 4 * V; ++i) w[i] = 0u;
+            }
+            const uint16_t* xb = xs + xrow * P.x_stride + sg * kSgCols + 4 * t4;
+            const uint32_t tcol = tw + (uint32_t)(64 * u);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                uint32_t a[16];
+                if (q < tq) {
+                    tmem_ld16(tcol + 16 * q, a);
+                    tmem_wait_ld();
+                } else {
+                    decode_quad<BITS>(tg, tg8, w, q, a);
+                }
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint2 xv = *reinterpret_cast<const uint2*>(xb + (4 * q + j) * 16);
+                    if (j & 1)
+                        tc::mma16816(d1, a[4 * j], a[4 * j + 1], a[4 * j + 2], a[4 * j + 3], xv.x, xv.y);
+                    else
+                        tc::mma16816(d0, a[4 * j], a[4 * j + 1], a[4 * j + 2], a[4 * j + 3], xv.x, xv.y);
+                }
+            }
+            if (++sg == nsg || u + 1 == nwu) {
+                flush_tile();
+                __syncwarp();  // the tcgen05 loads that follow need the whole warp
+                if (u + 1 < nwu) {
+                    ++tile;
+                    sg = 0;
+                    start_tile();
+                }
+            }
+        }
+    }
+
+    // ---- tiles shared by several warps: once every warp has left its loop,
+    // the warps' parts are added in warp order and the rows get their sparse
+    // sums; the control warp frees TMEM (every tcgen05.ld has completed)
+    tmem_fence_before();
+    __syncthreads();
+    tmem_fence_after();
+    if (ctrl) tmem_dealloc(taddr, kTmemCols);
+    csr_ready = true;  // the control warp wrote the sparse sums before the barrier
+    for (int idx = tid; idx < ctiles * TE; idx += kThreads) {
+        const int tl = idx / TE, e = idx - tl * TE;
+        const int mask = s_tinfo[tl];
+        if ((mask & (mask - 1)) == 0) continue;  // one warp: already written
+        const int row_l = e / CM, col = e - row_l * CM;
+        const int tile = t_first + tl;
+        float sum = 0.f;
+        for (int mm = mask; mm; mm &= mm - 1) {
+            const int wv = __ffs(mm) - 1;
+            const int wfirst_v = (u0 + cn * wv / kDenseWarps) / nsg;
+            sum += s_slots[(wv * 2 + (tile == wfirst_v ? 0 : 1)) * TE + e];
+        }
+        const int row = tile * kTileRows + row_l;
+        if (row < p.n_out && col < B) p.y[col * p.ldy + row] = f2h_rn(sum + csr_row_sum(row - ra, col));
+    }
+}
+
+}  // namespace pd
+}  // namespace sqz

@@ -15,6 +15,7 @@
 
 #include "../../include/sqz.h"
 #include "kernels_basic.cuh"
+#include "kernels_pd.cuh"
 #include "kernels_tc.cuh"
 
 namespace {
@@ -75,6 +76,7 @@ struct sqz_layer {
     int smem_budget = 232448;  // shared memory of one fused CTA (kCtasPerSm of them share an SM)
     int mac = SQZ_MAC_TENSOR_CORES;
     int csr_mode = SQZ_CSR_BALANCED;
+    int predecode = 1;  // batches of 1..8: the kernel that decodes ahead of x into TMEM
     // The fused kernel serves every layer with N > 0 and K > 0 (columns past
     // K are padded inside the kernel-native layout).
     bool fused_ok = false;
@@ -82,6 +84,7 @@ struct sqz_layer {
     // kernel cannot serve (the row-per-warp kernel reads them)
     uint32_t* codes = nullptr;
     uint16_t* lut = nullptr;
+    bool canonical_released = false;
     // CSR copies, padded by 8 elements so that 16-byte aligned bulk copies
     // of any slice stay inside the allocation
     int32_t* rowptr = nullptr;
@@ -228,7 +231,28 @@ sqz_status prepare_fused_bits(int optin) {
 
 sqz_status prepare_fused_kernels(int optin) {
     sqz_status st = prepare_fused_bits<3>(optin);
-    return st != SQZ_OK ? st : prepare_fused_bits<4>(optin);
+    if (st != SQZ_OK) return st;
+    if ((st = prepare_fused_bits<4>(optin)) != SQZ_OK) return st;
+    SQZ_CUDA_TRY(cudaFuncSetAttribute(sqz::pd::gemv_pd_kernel<3, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      optin), "cudaFuncSetAttribute");
+    SQZ_CUDA_TRY(cudaFuncSetAttribute(sqz::pd::gemv_pd_kernel<3, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      optin), "cudaFuncSetAttribute");
+    SQZ_CUDA_TRY(cudaFuncSetAttribute(sqz::pd::gemv_pd_kernel<4, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      optin), "cudaFuncSetAttribute");
+    SQZ_CUDA_TRY(cudaFuncSetAttribute(sqz::pd::gemv_pd_kernel<4, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      optin), "cudaFuncSetAttribute");
+    return SQZ_OK;
+}
+
+// The decode-ahead kernel's plan for a call, or false when it does not serve
+// it (batch above 8, or x and the rings do not fit in one CTA's shared
+// memory).
+bool pd_plan_for(int bits, int n_out, int k_in, int sm_count, int smem_optin, int batch, sqz::pd::Plan* out) {
+    if (batch < 1 || batch > 8 || n_out < 1 || k_in < 1) return false;
+    const sqz::pd::Plan P = sqz::pd::make_plan(bits, n_out, k_in, batch, sm_count, smem_optin);
+    if (P.total > smem_optin || P.grid > sqz::tc::kMaxCtas) return false;
+    *out = P;
+    return true;
 }
 
 // Plan for a call, or false when the fused kernel cannot stage x.  A call
@@ -339,9 +363,58 @@ cudaError_t launch_fused_bits(const sqz::tc::Params& prm, int batch, int mac, in
     return launch_fused<BITS, 1, kMacTensor, true>(prm, s);
 }
 
+template <int BITS>
+cudaError_t launch_pd(const sqz::pd::Params& prm, bool single, cudaStream_t s) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)prm.plan.grid);
+    cfg.blockDim = dim3(sqz::pd::kThreads);
+    cfg.dynamicSmemBytes = (size_t)prm.plan.total;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return single ? cudaLaunchKernelEx(&cfg, sqz::pd::gemv_pd_kernel<BITS, true>, prm)
+                  : cudaLaunchKernelEx(&cfg, sqz::pd::gemv_pd_kernel<BITS, false>, prm);
+}
+
+// Whether a call takes the decode-ahead kernel: the handle's default options
+// (tensor cores, balanced outliers), batch 1..8 and a plan that fits.
+bool pd_serves(const sqz_layer* L, int32_t batch, sqz::pd::Plan* P) {
+    return L->fused_ok && L->predecode && L->mac == SQZ_MAC_TENSOR_CORES && L->csr_mode == SQZ_CSR_BALANCED &&
+           pd_plan_for(L->bits, L->n_out, L->k_in, L->sm_count, L->smem_optin, batch, P) && P->grid == L->grid;
+}
+
 sqz_status gemv_impl(const sqz_layer* L, const uint16_t* x, int32_t batch, int64_t ldx, uint16_t* y, int64_t ldy,
                      cudaStream_t s) {
     if (L->n_out == 0) return SQZ_OK;
+    sqz::pd::Plan PP;
+    if (pd_serves(L, batch, &PP)) {
+        sqz::pd::Params prm{};
+        prm.codes = L->codes_native;
+        prm.lutp = L->lut_native;
+        prm.rowptr = L->rowptr;
+        prm.col = L->col;
+        prm.val = L->val;
+        prm.x = x;
+        prm.ldx = ldx;
+        prm.y = y;
+        prm.ldy = ldy;
+        prm.status = L->status;
+        prm.n_out = L->n_out;
+        prm.k_in = L->k_in;
+        prm.nsg = L->nsg;
+        prm.ntiles = L->ntiles;
+        prm.batch = batch;
+        prm.has_csr = L->nnz > 0;
+        prm.x_bulk = (reinterpret_cast<uintptr_t>(x) % 16 == 0) && (ldx % 8 == 0) && (L->k_in % 8 == 0);
+        prm.plan = PP;
+        prm.csr_cta = L->csr_cta;
+        const cudaError_t e = L->bits == 3 ? launch_pd<3>(prm, batch == 1, s) : launch_pd<4>(prm, batch == 1, s);
+        SQZ_CUDA_TRY(e, "fused gemv launch");
+        return SQZ_OK;
+    }
     sqz::tc::Plan P;
     const int chunk = L->fused_ok ? launch_columns(L->bits, L->n_out, L->k_in,
                                                    DeviceShape{L->sm_count, L->smem_budget, L->smem_optin}, batch, &P)
@@ -376,7 +449,7 @@ sqz_status gemv_impl(const sqz_layer* L, const uint16_t* x, int32_t batch, int64
                                                : launch_fused_bits<4>(prm, nb, L->mac, L->csr_mode, s);
             SQZ_CUDA_TRY(e, "fused gemv launch");
         }
-    } else if (!L->codes) {
+    } else if (L->canonical_released) {
         return fail(SQZ_ERR_UNSUPPORTED, "no fused plan for this call and the canonical codes were released");
     } else if (L->bits == 3) {
         dispatch_rowwarp<3>(L, x, batch, ldx, y, ldy, s);
@@ -551,6 +624,7 @@ sqz_status sqz_create_layer(const sqz_layer_desc* desc, void* stream, sqz_layer_
         L->device_bytes -= (int64_t)(code_n * 4 + lut_n * 2);
         L->codes = nullptr;
         L->lut = nullptr;
+        L->canonical_released = true;
     }
 #undef SQZ_STEP
 #undef SQZ_CUDA_STEP
@@ -670,6 +744,21 @@ sqz_status sqz_plan_query(int32_t n_out, int32_t k_in, int32_t bits, int32_t bat
     const int share = smem_per_sm / sqz::tc::kCtasPerSm - 1024;
     const DeviceShape d{sm_count, share < smem_optin ? share : smem_optin, smem_optin};
     const int grid = sqz::tc::grid_size(n_out, sm_count);
+    sqz::pd::Plan PP;
+    if (grid <= sqz::tc::kMaxCtas && pd_plan_for(bits, n_out, k_in, sm_count, smem_optin, batch, &PP)) {
+        out->fused = 1;
+        out->predecode = 1;
+        out->columns_per_launch = batch;
+        out->launches = 1;
+        out->grid = PP.grid;
+        out->threads = sqz::pd::kThreads;
+        out->smem_bytes = PP.total;
+        out->ctas_per_sm = 1;
+        out->passes = 1;
+        out->ring_stages = sqz::pd::kStages;
+        out->csr_stage_entries = PP.csr_cap;
+        return SQZ_OK;
+    }
     sqz::tc::Plan P{};
     const int chunk = grid <= sqz::tc::kMaxCtas ? launch_columns(bits, n_out, k_in, d, batch, &P) : 0;
     if (chunk == 0) return SQZ_OK;  // fused = 0: the row-per-warp kernel
@@ -736,6 +825,14 @@ sqz_status sqz_layer_set_csr_mode(sqz_layer_t layer, int32_t mode) {
     return SQZ_OK;
 }
 
+sqz_status sqz_layer_set_predecode(sqz_layer_t layer, int32_t enable) {
+    if (!layer) return fail(SQZ_ERR_INVALID_ARG, "layer is NULL");
+    if (enable != 0 && enable != 1) return fail(SQZ_ERR_INVALID_ARG, "enable must be 0 or 1 (got %d)", enable);
+    layer->predecode = enable;
+    drop_host_graphs(layer);
+    return SQZ_OK;
+}
+
 sqz_status sqz_layer_status(sqz_layer_t layer, void* stream, int32_t* status) {
     if (!layer || !status) return fail(SQZ_ERR_INVALID_ARG, "layer and status must be non-NULL");
     *status = 0;
@@ -793,6 +890,6 @@ void sqz_internal_set_last_error(const char* msg) { g_last_error = msg ? msg : "
 
 extern "C" {
 
-int32_t sqz_version(void) { return 200; }
+int32_t sqz_version(void) { return 300; }
 
 }  // extern "C"

@@ -463,3 +463,31 @@ def test_layer_holds_the_compressed_weights_once(B, wl):
     y_ref, bound = oracle.default().gemv_layer(L, x, rows=rows)
     assert_close(y16[:, rows], y_ref, bound, wl)
     layer.close()
+
+
+@pytest.mark.parametrize("n_out,k_in,bits,nnz,batch", [
+    (300, 4096, 3, 5000, 1), (257, 1032, 4, 1000, 3), (2000, 3072, 3, 30000, 8), (5000, 512, 4, 0, 2),
+    (33, 96, 3, 10, 1), (4100, 2048, 4, 9000, 5), (150, 20000, 3, 400, 1)])
+def test_decode_ahead_and_plain_kernels_match_oracle(B, orc, n_out, k_in, bits, nnz, batch):
+    """Batches of 1..8 take by default the kernel that decodes ahead of x
+    into tensor memory; the kernel without that step must agree with the
+    oracle on the same inputs too, and the decode-ahead results must not
+    depend on how many quads a warp parked before x arrived (the same MMAs
+    run in the same order either way): repeated calls are bit-identical."""
+    L = make_small(90 + n_out % 17, n_out, k_in, bits, nnz)
+    x = synth.make_x(batch, k_in, seed=3, key="pd")
+    layer = upload(B, L)
+    y_ref, bound = orc.gemv_layer(L, x)
+    plan = B.sqz_plan_query(n_out, k_in, bits, batch)
+    assert plan["predecode"] == 1
+    y_pd = gpu_gemv(B, layer, x)
+    assert_close(y_pd, y_ref, bound, "decode-ahead")
+    for _ in range(3):
+        assert np.array_equal(gpu_gemv(B, layer, x), y_pd)
+    B.sqz_layer_set_predecode(layer, False)
+    y_plain = gpu_gemv(B, layer, x)
+    assert_close(y_plain, y_ref, bound, "plain")
+    B.sqz_layer_set_predecode(layer, True)
+    assert np.array_equal(gpu_gemv(B, layer, x), y_pd)
+    assert B.sqz_layer_status(layer) == 0
+    layer.close()

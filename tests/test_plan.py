@@ -1,9 +1,12 @@
 """The launch plan (host logic, no GPU): for every workload shape and every
-batch size the fused kernel serves the call with a plan that fits the
-shared memory it claims, single-pass launches use the fixed 3- or 4-stage
-code ring (the kernel's compile-time waits depend on it), and batches above
-8 run as one-pass launches of 8 columns when those fit while the whole
-batch would need several passes."""
+batch size a fused kernel serves the call with a plan that fits the shared
+memory it claims.  Batches of 1..8 whose x fits take the decode-ahead kernel
+(one CTA of 17 warps per SM, more than half the SM's shared memory so that
+no second CTA of it can be resident and wait for its tensor memory); the
+others take the 12-warp kernel, whose single-pass launches use the fixed 3-
+or 4-stage code ring (its compile-time waits depend on it), and whose
+batches above 8 run as one-pass launches of 8 columns when those fit while
+the whole batch would need several passes."""
 import pytest
 
 import synth
@@ -28,19 +31,34 @@ def test_every_batch_gets_a_fitting_fused_plan(shape):
         p = B.sqz_plan_query(shape.n_out, shape.k_in, shape.bits, batch, **DEV)
         assert p["fused"] == 1, (shape.key, batch)
         assert p["grid"] == min(DEV["sm_count"], (shape.n_out + 15) // 16)
+        assert p["launches"] * p["columns_per_launch"] >= batch
+        assert (p["launches"] - 1) * p["columns_per_launch"] < batch
+        assert p["csr_stage_entries"] >= 0 and p["csr_stage_entries"] % 8 == 0
+        if p["predecode"]:
+            assert batch <= 8
+            assert p["threads"] == 17 * 32 and p["ctas_per_sm"] == 1
+            assert DEV["smem_per_sm"] // 2 < p["smem_bytes"] <= DEV["smem_optin"]
+            assert (p["launches"], p["passes"], p["ring_stages"]) == (1, 1, 4)
+            continue
         assert p["threads"] == 384
         budget = HALF if p["ctas_per_sm"] == 2 else DEV["smem_optin"]
         assert 0 < p["smem_bytes"] <= budget
-        assert p["launches"] * p["columns_per_launch"] >= batch
-        assert (p["launches"] - 1) * p["columns_per_launch"] < batch
         if p["passes"] == 1:
             assert p["ring_stages"] in (3, 4)
         else:
             assert p["ring_stages"] >= 2
-        if batch == 1:
-            assert p["passes"] == 1 and p["launches"] == 1
-            assert p["ctas_per_sm"] == 2, "batch 1 must leave room for the next call's CTA"
-        assert p["csr_stage_entries"] >= 0 and p["csr_stage_entries"] % 8 == 0
+        assert batch > 1, "batch 1 of every workload shape takes the decode-ahead kernel"
+
+
+def test_decode_ahead_kernel_serves_batches_up_to_eight_whose_x_fits():
+    x_fits = lambda k, b: b * (((k + 255) // 256 * 512 + 127) // 128 * 128 + 32)
+    for n, k, bits in ((11008, 4096, 3), (4096, 4096, 4), (5120, 13824, 3), (8192, 22016, 3)):
+        for batch in range(1, 17):
+            p = B.sqz_plan_query(n, k, bits, batch, **DEV)
+            if batch > 8:
+                assert p["predecode"] == 0
+            elif x_fits(k, batch) <= 64 * 1024:
+                assert p["predecode"] == 1, (n, k, batch)
 
 
 def test_large_batches_split_into_single_pass_launches_of_eight():
