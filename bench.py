@@ -59,8 +59,9 @@ def parse():
     p.add_argument("--sweep", action="store_true", help="one JSON line per workload shape")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--seed", type=int, default=0)
-    p.add_argument("--predecode", type=int, choices=(0, 1), default=1,
-                   help="batches of 1..8: decode ahead of x into tensor memory (1, the default) or not (0)")
+    p.add_argument("--predecode", type=int, choices=(0, 1, 8, 16), default=0,
+                   help="batches of 1..8: the kernel that decodes ahead of x into tensor memory (1; 8 or 16 dense "
+                        "warps per CTA) instead of the default 12-warp kernel (0)")
     p.add_argument("--csr", choices=("balanced", "rowwise"), default="balanced",
                    help="sparse scheme of the fused kernel (rowwise: the plain CSR comparison)")
     p.add_argument("--encode", action="store_true",
@@ -225,7 +226,7 @@ def config_for(args, shape, instances, inst_bytes):
             args.workload, f"{shape.n_out}x{shape.k_in}, {shape.bits}-bit, {shape.density:.2%} CSR, batch {shape.batch}"),
         "n_out": shape.n_out, "k_in": shape.k_in, "bits": shape.bits, "density": shape.density,
         "batch": shape.batch, "outliers": shape.dist, "csr_scheme": args.csr,
-        "kernel": "decode-ahead (TMEM)" if getattr(args, "predecode", 1) and shape.batch <= 8 else "12-warp fused",
+        "kernel": "decode-ahead (TMEM)" if getattr(args, "predecode", 0) and shape.batch <= 8 else "12-warp fused",
         "step": f"one token through a stack of {instances} distinct layers of this shape ({instances} calls)",
         "l2": f"inputs larger than L2: the stack holds {instances * inst_bytes / 1e6:.0f} MB",
         "parallelism": "replicas (independent layers per GPU)",
@@ -375,8 +376,8 @@ def run_ours(args):
                                                 device=dev))
         if args.csr == "rowwise":
             B.sqz_layer_set_csr_mode(layers[-1], B.SQZ_CSR_ROWWISE)
-        if not args.predecode:
-            B.sqz_layer_set_predecode(layers[-1], False)
+        if args.predecode:
+            B.sqz_layer_set_predecode(layers[-1], args.predecode)
         xs.append(torch.from_numpy(synth.x_for(shape, seed=args.seed, instance=instance_id(rank, i)).view(np.int16))
                   .to(dev))
         ys.append(torch.empty((shape.batch, shape.n_out), dtype=torch.int16, device=dev))

@@ -186,15 +186,18 @@ SQZ_API sqz_status sqz_layer_set_mac(sqz_layer_t layer, int32_t mac);
 SQZ_API sqz_status sqz_layer_set_csr_mode(sqz_layer_t layer, int32_t mode);
 
 /*
- * Batches of 1..8 columns take, by default (enable = 1), the kernel that
- * decodes the first code units of every warp into tensor memory while it
- * waits for the previous kernel of the stream and for x, and multiplies them
- * once x has arrived (the dependency wait is dead time otherwise).  enable = 0
- * selects the kernel without that step, for comparison; both give results
- * within the same bound (only the order of additions differs).  The choice
- * applies with the default MAC unit and CSR mode.  Not thread-safe against
- * concurrent sqz_gemv calls on the same handle.
- * Errors: SQZ_ERR_INVALID_ARG.
+ * The decode-ahead kernel (batches of 1..8 columns; off by default): every
+ * warp decodes its first code units into tensor memory while the call waits
+ * for the previous kernel of the stream and for x, and multiplies them once x
+ * has arrived.  enable = 1 takes it (two CTAs of 8 dense warps per SM when
+ * they fit half an SM, else one CTA of 16); 8 or 16 ask for one of the two
+ * CTA shapes; 0 (the default) takes the 12-warp kernel.  All choices give
+ * results within the same bound, and the two decode-ahead shapes give the
+ * same bits.  In a chain of dependent calls the next call's decoding ahead
+ * runs while the current call computes, so on B200 it has not been faster
+ * than the default; it applies with the default MAC unit and CSR mode.  Not
+ * thread-safe against concurrent sqz_gemv calls on the same handle.
+ * Errors: SQZ_ERR_INVALID_ARG (enable not in {0, 1, 8, 16}).
  */
 SQZ_API sqz_status sqz_layer_set_predecode(sqz_layer_t layer, int32_t enable);
 
@@ -223,10 +226,11 @@ SQZ_API sqz_status sqz_layer_info(sqz_layer_t layer, int32_t* n_out, int32_t* k_
  * shared memory (ctas_per_sm = 2 when two CTAs share an SM), x staged in
  * `passes` chunks of K, a code ring of ring_stages stages per warp and up to
  * csr_stage_entries outliers per CTA staged in shared memory (the first
- * launch's plan; a shorter last launch may differ).  predecode = 1 when the
- * call takes the decode-ahead kernel (sqz_layer_set_predecode; this query
- * assumes the handle's default options).  No counterpart in the paper: it
- * exposes this library's own scheduling.
+ * launch's plan; a shorter last launch may differ).  `predecode` is the
+ * handle's sqz_layer_set_predecode choice (0, 1, 8 or 16); out->predecode = 1 when
+ * the call takes the decode-ahead kernel (the query assumes the default MAC
+ * unit and CSR mode).  No counterpart in the paper: it exposes this
+ * library's own scheduling.
  * Errors: SQZ_ERR_INVALID_ARG for a NULL out, bits not in {3,4}, n_out or k_in
  * < 1, batch outside [1,16], or a non-positive device figure.
  */
@@ -235,7 +239,7 @@ typedef struct {
         csr_stage_entries, predecode;
 } sqz_plan_info;
 SQZ_API sqz_status sqz_plan_query(int32_t n_out, int32_t k_in, int32_t bits, int32_t batch, int32_t sm_count,
-                                  int32_t smem_per_sm, int32_t smem_optin, sqz_plan_info* out);
+                                  int32_t smem_per_sm, int32_t smem_optin, int32_t predecode, sqz_plan_info* out);
 
 /* Release a handle and its device memory.  NULL is accepted.  The caller
  * must make sure no work that uses the handle is still in flight. */

@@ -102,7 +102,7 @@ def lib() -> ctypes.CDLL:
         L.sqz_encode.argtypes = [P, i32, i32, i32, ctypes.c_double, i32, P, P, P, P, P, i64,
                                  ctypes.POINTER(i64), P, P]
         L.sqz_encode.restype = ctypes.c_int
-        L.sqz_plan_query.argtypes = [i32, i32, i32, i32, i32, i32, i32, ctypes.POINTER(sqz_plan_info)]
+        L.sqz_plan_query.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, ctypes.POINTER(sqz_plan_info)]
         L.sqz_plan_query.restype = ctypes.c_int
         L.sqz_encode_outliers.argtypes = [i64, ctypes.c_double]
         L.sqz_encode_outliers.restype = i64
@@ -311,11 +311,11 @@ B200_DEVICE = {"sm_count": 148, "smem_per_sm": 233472, "smem_optin": 232448}
 
 
 def sqz_plan_query(n_out: int, k_in: int, bits: int, batch: int, sm_count: int = 148, smem_per_sm: int = 233472,
-                   smem_optin: int = 232448) -> dict:
+                   smem_optin: int = 232448, predecode: int = 0) -> dict:
     """The launch plan sqz_gemv would use (host computation; defaults: B200)."""
     info = sqz_plan_info()
-    _check(lib().sqz_plan_query(n_out, k_in, bits, batch, sm_count, smem_per_sm, smem_optin, ctypes.byref(info)),
-           "sqz_plan_query")
+    _check(lib().sqz_plan_query(n_out, k_in, bits, batch, sm_count, smem_per_sm, smem_optin, int(predecode),
+                                ctypes.byref(info)), "sqz_plan_query")
     return {name: int(getattr(info, name)) for name, _ in sqz_plan_info._fields_}
 
 
@@ -357,8 +357,8 @@ def sqz_layer_set_csr_mode(layer: Layer, mode: int) -> None:
     _check(lib().sqz_layer_set_csr_mode(layer, int(mode)), "sqz_layer_set_csr_mode")
 
 
-def sqz_layer_set_predecode(layer: Layer, enable: bool) -> None:
-    _check(lib().sqz_layer_set_predecode(layer, int(bool(enable))), "sqz_layer_set_predecode")
+def sqz_layer_set_predecode(layer: Layer, enable: int) -> None:
+    _check(lib().sqz_layer_set_predecode(layer, int(enable)), "sqz_layer_set_predecode")
 
 
 def sqz_layer_status(layer: Layer, stream=None) -> int:

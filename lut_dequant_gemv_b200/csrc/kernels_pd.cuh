@@ -27,15 +27,19 @@
 //     control warp.  A CTA owns a contiguous run of whole tiles; its dense
 //     warps split the CTA's units into 16 contiguous, equal ranges.
 //   * The control warp requests the LUT planes, the rowptr slice and the
-//     CSR entries of the CTA (bulk copies), asks L2 for the CTA's whole code
-//     range (the HBM streams it while the SMs wait for the previous kernel),
-//     allocates TMEM, waits for the previous kernel, copies x in and sums the
-//     sparse part: the CTA's nonzeros split evenly over its 32 lanes (the
-//     balanced scheme), the pieces of rows cut between lanes added in lane
-//     order.
-//   * Tiles held whole by a warp are written by it; tiles split between
-//     warps are finished after one CTA barrier, the warps' parts added in
-//     warp order.  Every summation order is fixed: results are bitwise
+//     CSR entries of the CTA (bulk copies), allocates TMEM, waits for the
+//     previous kernel and copies x in.
+//   * Sparse part (the balanced scheme): the CTA's nonzeros are split evenly
+//     over the 512 dense threads.  Before x arrives a thread finds the row of
+//     its first entry and loads its first entries; once x is there it sums
+//     its share per row (head piece, rows it holds whole, tail piece), then
+//     starts its dense work.
+//   * Every warp stores its part of each tile it touches in shared memory
+//     (one slot for a tile it holds whole, per-warp slots for the first and
+//     last tiles it shares); after one CTA barrier the threads add the
+//     parts in warp order and each row's sparse sum (the interior sum plus
+//     the pieces of the threads whose shares cut the row, in thread order)
+//     and write y once.  Every summation order is fixed: results are bitwise
 //     reproducible, and a column of a batch equals the batch-1 call on it.
 //
 // TMEM: warp w reaches the 32 lanes of quarter w % 4 (lane = the warp's
@@ -62,24 +66,48 @@ using tc::kTileRows;
 using tc::round_up;
 using tc::tile_begin;
 
-constexpr int kDenseWarps = 16;
-constexpr int kCtrlWarp = kDenseWarps;       // warp 16
-constexpr int kThreads = (kDenseWarps + 1) * 32;
-constexpr int kStages = 4;                   // code ring stages per dense warp
-constexpr int kPreUnits = 2;                 // units per warp that can be parked in TMEM
-constexpr int kTmemCols = 512;
-constexpr int kCsrCap = 4096;                // CSR entries per CTA staged in shared memory
-constexpr int kMinSmem = 120 * 1024;         // more than half an SM: one CTA per SM
+// Two shapes of CTA (template argument NW, the dense warps):
+//   NW = 8:  8 dense warps + the control warp, two CTAs per SM, each with half
+//            the TMEM (256 columns): the next call's CTA is resident while
+//            this one computes, so it loads its LUTs and first code units and
+//            parks its first units in TMEM before the previous call ends.
+//   NW = 16: 16 dense warps + the control warp, one CTA per SM with all 512
+//            columns (for calls whose shared memory does not fit half an SM).
+// Either way a warp parks at most two units (128 columns of its quarter), at
+// most two CTAs of this kernel are resident on an SM, and together they never
+// ask for more than the SM's 512 columns, so no allocation ever waits for a
+// CTA that waits for it.
+// The summation structure does not depend on the shape: a CTA's units are
+// split into 16 contiguous ranges ("virtual warps", each with its own
+// accumulators and its own slots for the tiles it shares) and its nonzeros
+// into 512 equal shares; with NW = 8 a warp runs two adjacent ranges one
+// after the other and two shares.  Both shapes give the same bits.
+constexpr int kVWarps = 16;
+constexpr int kVThreads = kVWarps * 32;
+template <int NW>
+struct Shape {
+    static constexpr int kDenseWarps = NW;
+    static constexpr int kCtrlWarp = NW;
+    static constexpr int kThreads = (NW + 1) * 32;
+    static constexpr int kCtasPerSm = NW == 8 ? 2 : 1;
+    static constexpr int kTmemCols = NW == 8 ? 256 : 512;
+    static constexpr int kRanges = kVWarps / NW;  // virtual warps per warp
+    static constexpr int kMinSmem = NW == 8 ? 0 : 120 * 1024;  // NW = 16: more than half an SM
+};
+constexpr int kStages = 4;    // code ring stages per dense warp
+constexpr int kPreUnits = 2;  // units per warp that can be parked in TMEM
+constexpr int kCsrCap = 4096; // CSR entries per CTA staged in shared memory
 
 struct Plan {
     int grid, ctiles_max, x_stride, cm, csr_cap;
     int off_taddr, off_x, off_lut, off_rp, off_rowsum, off_head, off_tail, off_headrow, off_tailrow, off_slots,
-        off_tinfo, off_col, off_val, off_ring, total;
+        off_tsum, off_tinfo, off_col, off_val, off_ring, total;
 };
 
 // Shared-memory plan of a launch; total > budget when it does not fit.
-__host__ __device__ inline Plan make_plan(int bits, int n_out, int k_in, int batch, int sms, int budget) {
+__host__ __device__ inline Plan make_plan(int bits, int n_out, int k_in, int batch, int sms, int budget, int nw) {
     Plan P{};
+    const int min_smem = nw == 8 ? Shape<8>::kMinSmem : Shape<16>::kMinSmem;
     const int ntiles = (n_out + kTileRows - 1) / kTileRows;
     const int nsg = ((k_in + 15) / 16 + kSgSteps - 1) / kSgSteps;
     const int lut_bytes = bits == 3 ? 16 : 32;
@@ -102,16 +130,19 @@ __host__ __device__ inline Plan make_plan(int bits, int n_out, int k_in, int bat
     off += round_up((rows + 8) * 4, 128);
     P.off_rowsum = off;
     off += round_up(rows * P.cm * 4, 128);
+    const int ct = kVThreads;
     P.off_head = off;
-    P.off_tail = off + 32 * P.cm * 4;
-    P.off_headrow = P.off_tail + 32 * P.cm * 4;
-    P.off_tailrow = P.off_headrow + 32 * 4;
-    off += round_up(2 * 32 * P.cm * 4 + 2 * 32 * 4, 128);
+    P.off_tail = off + ct * P.cm * 4;
+    P.off_headrow = P.off_tail + ct * P.cm * 4;
+    P.off_tailrow = P.off_headrow + ct * 4;
+    off += round_up(2 * ct * P.cm * 4 + 2 * ct * 4, 128);
     P.off_slots = off;
-    off += round_up(kDenseWarps * 2 * kTileRows * P.cm * 4, 128);
+    off += round_up(kVWarps * 2 * kTileRows * P.cm * 4, 128);
+    P.off_tsum = off;  // sums of the tiles a warp holds whole
+    off += round_up(rows * P.cm * 4, 128);
     P.off_tinfo = off;
     off += round_up(P.ctiles_max * 4, 128);
-    const int ring = kStages * kDenseWarps * sg_bytes;
+    const int ring = kStages * nw * sg_bytes;
     int cap = (budget - off - ring - 512) / 6;
     cap = cap > kCsrCap ? kCsrCap : cap;
     P.csr_cap = cap < 0 ? 0 : cap & ~7;
@@ -121,7 +152,7 @@ __host__ __device__ inline Plan make_plan(int bits, int n_out, int k_in, int bat
     off += round_up((P.csr_cap + 16) * 2, 128);
     P.off_ring = off;
     off += ring;
-    P.total = off < kMinSmem ? kMinSmem : off;
+    P.total = off < min_smem ? min_smem : off;
     return P;
 }
 
@@ -185,7 +216,26 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
         : "r"(taddr)
         : "memory");
 }
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// Wait for this thread's tcgen05.ld; the registers of `r` pass through the
+// instruction so that no use of them can be scheduled before it (the load
+// writes them asynchronously).
+__device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[16]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                   "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
+                 :
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[16], uint32_t (&r2)[16]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                   "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]),
+                   "+r"(r2[0]), "+r"(r2[1]), "+r"(r2[2]), "+r"(r2[3]), "+r"(r2[4]), "+r"(r2[5]), "+r"(r2[6]),
+                   "+r"(r2[7]), "+r"(r2[8]), "+r"(r2[9]), "+r"(r2[10]), "+r"(r2[11]), "+r"(r2[12]), "+r"(r2[13]),
+                   "+r"(r2[14]), "+r"(r2[15])
+                 :
+                 : "memory");
+}
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // The A fragments of quad q (k16-steps 4q..4q+3) of a unit: a[4j..4j+3] =
@@ -200,8 +250,12 @@ __device__ __forceinline__ void decode_quad(const TAB& tg, const TAB& tg8, const
 
 // ------------------------------------------------------------ main kernel
 // SB: batch 1 (one column carried through the sparse part and the combine).
-template <int BITS, bool SB>
-__global__ void __launch_bounds__(kThreads, 1) gemv_pd_kernel(const __grid_constant__ Params p) {
+template <int BITS, bool SB, int NW>
+__global__ void __launch_bounds__(Shape<NW>::kThreads, Shape<NW>::kCtasPerSm)
+    gemv_pd_kernel(const __grid_constant__ Params p) {
+    constexpr int kCtrlWarp = Shape<NW>::kCtrlWarp;
+    constexpr int kThreads = Shape<NW>::kThreads, kTmemCols = Shape<NW>::kTmemCols;
+    constexpr int RG = Shape<NW>::kRanges;
     using F = Fmt<BITS>;
     using TAB = typename std::conditional<BITS == 3, tc::Tab3, tc::Tab4>::type;
     constexpr int CM = SB ? 1 : 8;           // batch columns carried after the dense loop
@@ -220,9 +274,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_pd_kernel(const __grid_const
     const int t_first = tile_begin(p.ntiles, G, c), t_end = tile_begin(p.ntiles, G, c + 1);
     const int ctiles = t_end - t_first;
     const int u0 = t_first * nsg, cn = ctiles * nsg;
-    // dense warp w: units [wu0, wu1) of the CTA, contiguous and equal
+    // virtual warp v: units [vbeg(v), vbeg(v + 1)) of the CTA; dense warp w
+    // runs virtual warps w*RG .. w*RG+RG-1, i.e. units [wu0, wu1)
+    auto vbeg = [&](int v) { return u0 + cn * v / kVWarps; };
     const int wsel = ctrl ? 0 : warp;
-    const int wu0 = u0 + cn * wsel / kDenseWarps, wu1 = u0 + cn * (wsel + 1) / kDenseWarps;
+    const int wu0 = vbeg(wsel * RG), wu1 = vbeg((wsel + 1) * RG);
     const int nwu = ctrl ? 0 : wu1 - wu0;
     const int wfirst = nwu > 0 ? wu0 / nsg : -1;
     const int ra = min(p.n_out, t_first * kTileRows);
@@ -232,7 +288,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_pd_kernel(const __grid_const
     uint64_t* lbar = reinterpret_cast<uint64_t*>(smem);      // LUT planes + rowptr slice
     uint64_t* xbar = reinterpret_cast<uint64_t*>(smem) + 1;  // x
     uint64_t* cbar = reinterpret_cast<uint64_t*>(smem) + 2;  // CSR slices
-    uint64_t* rbar = reinterpret_cast<uint64_t*>(smem) + 3;  // sparse sums complete (32 arrivals)
     uint32_t* s_taddr = reinterpret_cast<uint32_t*>(smem + P.off_taddr);
     uint16_t* xs = reinterpret_cast<uint16_t*>(smem + P.off_x);
     uint8_t* luts = smem + P.off_lut;
@@ -242,7 +297,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_pd_kernel(const __grid_const
     int* s_headrow = reinterpret_cast<int*>(smem + P.off_headrow);
     int* s_tailrow = reinterpret_cast<int*>(smem + P.off_tailrow);
     float* s_slots = reinterpret_cast<float*>(smem + P.off_slots);
-    int* s_tinfo = reinterpret_cast<int*>(smem + P.off_tinfo);  // [tile] = mask of dense warps holding parts
+    float* s_tsum = reinterpret_cast<float*>(smem + P.off_tsum);
+    int* s_tinfo = reinterpret_cast<int*>(smem + P.off_tinfo);  // [tile] = mask of virtual warps holding parts
     const int rp_off = ra & 3;
     const int* s_rp = reinterpret_cast<const int*>(smem + P.off_rp) + rp_off;  // s_rp[i] = rowptr[ra + i]
     const int B = p.batch;
@@ -254,7 +310,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_pd_kernel(const __grid_const
             tc::mbar_init(lbar, 1);
             tc::mbar_init(xbar, p.x_bulk ? 1 : 32);  // bulk: one expect_tx; else every lane after its stores
             tc::mbar_init(cbar, 1);
-            tc::mbar_init(rbar, 32);
             tc::fence_mbar_init();
             const uint32_t lut_bytes = (uint32_t)ctiles * kTileRows * F::kLutBytes;
             const uint32_t rp_bytes = layer_csr ? (uint32_t)round_up(nrows + 1 + rp_off, 4) * 4 : 0u;
@@ -269,8 +324,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_pd_kernel(const __grid_const
             if (col_bytes) tc::bulk_g2s(smem + P.off_col, p.col + (q0 - (q0 & 3)), col_bytes, cbar);
             if (val_bytes) tc::bulk_g2s(smem + P.off_val, p.val + (q0 - (q0 & 7)), val_bytes, cbar);
         }
-        // every code unit of the CTA into L2 (one unit per lane and request)
-        for (int u = lane; u < cn; u += 32) prefetch_l2(p.codes + (int64_t)(u0 + u) * F::kSgBytes, F::kSgBytes);
         __syncwarp();
         tmem_alloc(s_taddr, kTmemCols);
     }
@@ -295,10 +348,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_pd_kernel(const __grid_const
     for (int tl = tid; tl < ctiles; tl += kThreads) {
         const int ta_u = (t_first + tl) * nsg, tb_u = ta_u + nsg;
         int mask = 0;
-        for (int wv = 0; wv < kDenseWarps; ++wv) {
-            const int a = u0 + cn * wv / kDenseWarps, b = u0 + cn * (wv + 1) / kDenseWarps;
-            if (max(a, ta_u) < min(b, tb_u)) mask |= 1 << wv;
-        }
+        for (int v = 0; v < kVWarps; ++v)
+            if (max(vbeg(v), ta_u) < min(vbeg(v + 1), tb_u)) mask |= 1 << v;
         s_tinfo[tl] = mask;
     }
     if (layer_csr)
@@ -315,7 +366,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_pd_kernel(const __grid_const
     tmem_fence_after();
     const uint32_t taddr = *s_taddr;
 
-    bool csr_ready = !layer_csr;
     if (ctrl) {
         // ---- x may be written by the previous kernel of the stream: wait
         // for it (its lines were requested into L2 first: a hint only)
@@ -339,118 +389,98 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_pd_kernel(const __grid_const
             }
             tc::mbar_arrive(xbar);  // release: this lane's x stores before the phase completes
         }
-        const bool got = tc::mbar_wait(lbar, 0) && tc::mbar_wait(xbar, 0) && tc::mbar_wait(cbar, 0);
-        if (!got) atomicOr(p.status, tc::kStatusWaitTimeout);
-
-        // ---- sparse part: the CTA's entries [q0, q1) split evenly over the
-        // 32 lanes; a lane's first and last rows go to its head/tail pieces,
-        // rows it holds whole straight to s_rowsum
-        const int q0 = __ldg(p.csr_cta + c), q1 = __ldg(p.csr_cta + c + 1);
-        const int nz = q1 - q0;
-        if (nz > 0) {
-            const bool in_smem = nz <= P.csr_cap;
-            const int* csr_col = in_smem ? reinterpret_cast<const int*>(smem + P.off_col) + (q0 & 3) - q0 : p.col;
-            const uint16_t* csr_val =
-                in_smem ? reinterpret_cast<const uint16_t*>(smem + P.off_val) + (q0 & 7) - q0 : p.val;
-            const int e_per = (nz + 31) / 32;
-            const int ca = (int)min((int64_t)q1, (int64_t)q0 + (int64_t)lane * e_per);
-            const int cb = (int)min((int64_t)q1, (int64_t)ca + e_per);
-            s_headrow[lane] = -1;
-            s_tailrow[lane] = -1;
-            if (ca < cb) {
-                int lo = 0, hi = nrows - 1;  // row (relative to ra) of entry ca
-                while (lo < hi) {
-                    const int mid = (lo + hi + 1) >> 1;
-                    if (s_rp[mid] <= ca) lo = mid; else hi = mid - 1;
-                }
-                int cur = lo, nxt = s_rp[cur + 1];
-                bool first = true;
-                float acc[CM];
-#pragma unroll
-                for (int b = 0; b < CM; ++b) acc[b] = 0.f;
-                auto emit = [&](bool last) {
-                    float* dstp;
-                    if (first) {
-                        s_headrow[lane] = cur;
-                        dstp = s_head + lane * CM;
-                    } else if (last) {
-                        s_tailrow[lane] = cur;
-                        dstp = s_tail + lane * CM;
-                    } else {
-                        dstp = s_rowsum + cur * CM;
-                    }
-#pragma unroll
-                    for (int b = 0; b < CM; ++b) dstp[b] = acc[b];
-                };
-                for (int base = ca; base < cb; base += 8) {
-                    int cc[8];
-                    uint32_t vh[8];
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const int q = base + j;
-                        const bool in = q < cb;
-                        cc[j] = in ? csr_col[q] : 0;
-                        vh[j] = in ? (uint32_t)csr_val[q] : 0u;
-                    }
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const int q = base + j;
-                        if (q >= cb) break;
-                        while (q >= nxt) {
-                            emit(false);
-                            first = false;
-#pragma unroll
-                            for (int b = 0; b < CM; ++b) acc[b] = 0.f;
-                            ++cur;
-                            nxt = s_rp[cur + 1];
-                        }
-                        const float v = h2f((uint16_t)vh[j]);
-#pragma unroll
-                        for (int b = 0; b < CM; ++b)
-                            if (SB || b < B) acc[b] = fmaf(v, h2f(xs[b * P.x_stride + cc[j]]), acc[b]);
-                    }
-                }
-                emit(true);
-            }
-            __syncwarp();
-            // rows cut between lanes: the interior sum plus the pieces of the
-            // lanes whose shares cut the row, in lane order
-            for (int i = lane; i < nrows; i += 32) {
-                const int rs = s_rp[i], re = s_rp[i + 1];
-                if (re <= rs) continue;
-                float cs[CM];
-#pragma unroll
-                for (int b = 0; b < CM; ++b) cs[b] = s_rowsum[i * CM + b];
-                const int tau_a = (rs - q0) / e_per, tau_b = min(31, (re - 1 - q0) / e_per);
-                for (int tau = tau_a; tau <= tau_b; ++tau) {
-                    if (s_headrow[tau] == i) {
-#pragma unroll
-                        for (int b = 0; b < CM; ++b) cs[b] += s_head[tau * CM + b];
-                    }
-                    if (s_tailrow[tau] == i) {
-#pragma unroll
-                        for (int b = 0; b < CM; ++b) cs[b] += s_tail[tau * CM + b];
-                    }
-                }
-#pragma unroll
-                for (int b = 0; b < CM; ++b) s_rowsum[i * CM + b] = cs[b];
-            }
-        }
-        tc::mbar_arrive(rbar);  // release: this lane's sparse sums before the phase completes
     }
 
-    // The sparse sum of row ra+i, batch column col.
-    auto csr_row_sum = [&](int i, int col) -> float {
-        if (!layer_csr) return 0.f;
-        if (!csr_ready) {
-            if (!tc::mbar_wait(rbar, 0)) atomicOr(p.status, tc::kStatusWaitTimeout);
-            csr_ready = true;
+    // ---- sparse part (balanced): the CTA's entries [q0, q1) in kVThreads
+    // equal shares; share t is summed per row (its first and last rows into
+    // head/tail pieces, rows it holds whole straight into s_rowsum)
+    const int q0 = __ldg(p.csr_cta + c), q1 = __ldg(p.csr_cta + c + 1);
+    const int nz = q1 - q0;
+    const bool has_csr = nz > 0;
+    const int e_per = has_csr ? (nz + kVThreads - 1) / kVThreads : 1;
+    const bool csr_in_smem = has_csr && nz <= P.csr_cap;
+    const int* csr_col = csr_in_smem ? reinterpret_cast<const int*>(smem + P.off_col) + (q0 & 3) - q0 : p.col;
+    const uint16_t* csr_val = csr_in_smem ? reinterpret_cast<const uint16_t*>(smem + P.off_val) + (q0 & 7) - q0 : p.val;
+    auto share_begin = [&](int t) { return (int)min((int64_t)q1, (int64_t)q0 + (int64_t)t * e_per); };
+    // row (relative to ra) of entry ca: the largest r with s_rp[r] <= ca (needs no x)
+    auto share_row = [&](int ca) {
+        int lo = 0, hi = nrows - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (s_rp[mid] <= ca) lo = mid; else hi = mid - 1;
         }
-        return s_rowsum[i * CM + col];
+        return lo;
     };
+    auto sparse_share = [&](int t, int row0) {
+        const int ca = share_begin(t);
+        const int cb = (int)min((int64_t)q1, (int64_t)ca + e_per);
+        if (ca >= cb) return;
+        int cur = row0, nxt = s_rp[cur + 1];
+        bool first = true;
+        float acc[CM];
+#pragma unroll
+        for (int b = 0; b < CM; ++b) acc[b] = 0.f;
+        auto emit = [&](bool last) {
+            float* dstp;
+            if (first) {
+                s_headrow[t] = cur;
+                dstp = s_head + t * CM;
+            } else if (last) {
+                s_tailrow[t] = cur;
+                dstp = s_tail + t * CM;
+            } else {
+                dstp = s_rowsum + cur * CM;
+            }
+#pragma unroll
+            for (int b = 0; b < CM; ++b) dstp[b] = acc[b];
+        };
+        for (int base = ca; base < cb; base += 8) {
+            int cc[8];
+            uint32_t vh[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int q = base + j;
+                const bool in = q < cb;
+                cc[j] = in ? csr_col[q] : 0;
+                vh[j] = in ? (uint32_t)csr_val[q] : 0u;
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int q = base + j;
+                if (q >= cb) break;
+                while (q >= nxt) {
+                    emit(false);
+                    first = false;
+#pragma unroll
+                    for (int b = 0; b < CM; ++b) acc[b] = 0.f;
+                    ++cur;
+                    nxt = s_rp[cur + 1];
+                }
+                const float v = h2f((uint16_t)vh[j]);
+#pragma unroll
+                for (int b = 0; b < CM; ++b)
+                    if (SB || b < B) acc[b] = fmaf(v, h2f(xs[b * P.x_stride + cc[j]]), acc[b]);
+            }
+        }
+        emit(true);
+    };
+    bool waits_ok = true;
+    int srow[RG];  // starting row of each of this thread's shares (found before x arrives)
+    if (!ctrl) {
+        waits_ok = tc::mbar_wait(lbar, 0) && tc::mbar_wait(cbar, 0);
+        if (has_csr)
+#pragma unroll
+            for (int r = 0; r < RG; ++r) {
+                const int t = (warp * RG + r) * 32 + lane;
+                s_headrow[t] = -1;
+                s_tailrow[t] = -1;
+                const int ca = share_begin(t);
+                srow[r] = ca < q1 ? share_row(ca) : 0;
+            }
+    }
 
     // ---- dense warps
-    if (!ctrl && nwu > 0) {
+    if (!ctrl) {
         // this warp's TMEM: lanes of quarter warp % 4, columns (warp / 4) * 128 ...
         const uint32_t tw = taddr + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)((warp >> 2) * 128);
         TAB tg, tg8;
@@ -476,14 +506,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_pd_kernel(const __grid_const
             const bool t = lane == 0 ? mbar_test(xbar, 0) : false;
             return __shfl_sync(0xffffffffu, t, 0);
         };
-        if (!tc::mbar_wait(lbar, 0)) atomicOr(p.status, tc::kStatusWaitTimeout);
         __syncwarp();
 
         // ---- ahead of x: decode the first units' quads into TMEM until x
         // is in shared memory (checked before every quad)
         int qp = 0;  // quads parked
         int s_read = 0, s_fill = D;
-        {
+        if (nwu > 0) {
             const int pre = min(nwu, kPreUnits);
             int tab_tile = -1;
             bool stop = false;
@@ -516,44 +545,32 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_pd_kernel(const __grid_const
             }
             tmem_wait_st();
         }
-        if (!tc::mbar_wait(xbar, 0)) atomicOr(p.status, tc::kStatusWaitTimeout);
+        if (!tc::mbar_wait(xbar, 0)) waits_ok = false;
         __syncwarp();
 
-        // ---- every unit in order: parked quads from TMEM, the rest decoded
+        // ---- every unit in order: the parked ones from TMEM (MMAs only),
+        // a partly parked one quad by quad, the rest decoded
         const int xrow = g < B ? g : 0;  // batch column of this lane's B fragment (n = g)
         float d0[4], d1[4];
         int tile = wfirst, sg = wu0 - wfirst * nsg;
-        auto start_tile = [&]() {
-            load_tabs(tile);
+        int vw = warp * RG;                    // current virtual warp (the first non-empty one)
+        int vend = vbeg(vw + 1) - wu0;         // its end (relative unit index)
+        while (vend <= 0 && vw + 1 < (warp + 1) * RG) vend = vbeg(++vw + 1) - wu0;
+        int vfirst = wfirst;                   // first tile of the current virtual warp
+        auto zero_acc = [&]() {
 #pragma unroll
             for (int q = 0; q < 4; ++q) d0[q] = d1[q] = 0.f;
         };
-        auto out = [&](int row, int col, float v) {
-            if (row < p.n_out && col < B) p.y[col * p.ldy + row] = f2h_rn(v + csr_row_sum(row - ra, col));
-        };
+        // the current virtual warp's part of `tile`: the tile's sum when the
+        // virtual warp holds it whole, else its slot (first or last tile it shares)
         auto flush_tile = [&]() {
             float rr[4];
 #pragma unroll
             for (int q = 0; q < 4; ++q) rr[q] = d0[q] + d1[q];
             const int tl = tile - t_first;
-            const int row0 = tile * kTileRows;
             const int mask = s_tinfo[tl];
-            if ((mask & (mask - 1)) == 0) {
-                if constexpr (SB) {
-                    if (t4 == 0) {
-                        out(row0 + g, 0, rr[0]);
-                        out(row0 + g + 8, 0, rr[2]);
-                    }
-                } else {
-                    const int col = 2 * t4;
-                    out(row0 + g, col, rr[0]);
-                    out(row0 + g, col + 1, rr[1]);
-                    out(row0 + g + 8, col, rr[2]);
-                    out(row0 + g + 8, col + 1, rr[3]);
-                }
-                return;
-            }
-            float* dst = s_slots + (warp * 2 + (tile == wfirst ? 0 : 1)) * TE;
+            float* dst = (mask & (mask - 1)) == 0 ? s_tsum + tl * TE
+                                                  : s_slots + (vw * 2 + (tile == vfirst ? 0 : 1)) * TE;
             if constexpr (SB) {
                 if (t4 == 0) {
                     dst[g] = rr[0];
@@ -567,75 +584,157 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_pd_kernel(const __grid_const
                 dst[(g + 8) * CM + col + 1] = rr[3];
             }
         };
-        start_tile();
-#pragma unroll 1
-        for (int u = 0; u < nwu; ++u) {
-            const int tq = min(4, max(0, qp - 4 * u));  // quads of this unit parked in TMEM
-            uint32_t w[4 * V];
-            if (tq < 4) {
-                tc::cp_async_wait<S - 2>();
-                read_stage(s_read, w);
-                issue(s_fill);
-                s_read = s_read + 1 == S ? 0 : s_read + 1;
-                s_fill = s_fill + 1 == S ? 0 : s_fill + 1;
-            } else {
+        auto mma_quad = [&](const uint16_t* xb, int q, const uint32_t (&a)[16]) {
 #pragma unroll
-                for (int i = 0; i < 4 * V; ++i) w[i] = 0u;
+            for (int j = 0; j < 4; ++j) {
+                const uint2 xv = *reinterpret_cast<const uint2*>(xb + (4 * q + j) * 16);
+                if (j & 1)
+                    tc::mma16816(d1, a[4 * j], a[4 * j + 1], a[4 * j + 2], a[4 * j + 3], xv.x, xv.y);
+                else
+                    tc::mma16816(d0, a[4 * j], a[4 * j + 1], a[4 * j + 2], a[4 * j + 3], xv.x, xv.y);
             }
+        };
+        auto next_stage = [&](uint32_t (&w)[4 * V]) {
+            tc::cp_async_wait<S - 2>();
+            read_stage(s_read, w);
+            issue(s_fill);
+            s_read = s_read + 1 == S ? 0 : s_read + 1;
+            s_fill = s_fill + 1 == S ? 0 : s_fill + 1;
+        };
+        const int nfull = qp >> 2, tq_part = qp & 3;
+        // after a unit: the accumulators go to the tile's slot at the end of a
+        // tile or of a virtual warp
+        auto unit_done = [&](int u) {
+            const bool tile_end = ++sg == nsg;
+            const bool v_end = u + 1 == vend;
+            if (tile_end || v_end) {
+                flush_tile();
+                __syncwarp();  // the tcgen05 loads that follow need the whole warp
+                zero_acc();
+                if (v_end && u + 1 < nwu) {  // the next virtual warp
+                    ++vw;
+                    vend = vbeg(vw + 1) - wu0;
+                    vfirst = (wu0 + u + 1) / nsg;
+                }
+                if (tile_end && u + 1 < nwu) {
+                    ++tile;
+                    sg = 0;
+                    load_tabs(tile);
+                }
+            }
+        };
+        if (nwu > 0) {
+            load_tabs(tile);
+            zero_acc();
+        }
+        int u = 0;
+        // parked whole: MMAs only
+#pragma unroll 1
+        for (; u < nfull; ++u) {
             const uint16_t* xb = xs + xrow * P.x_stride + sg * kSgCols + 4 * t4;
             const uint32_t tcol = tw + (uint32_t)(64 * u);
+            uint32_t a[16], b[16];
+            tmem_ld16(tcol, a);
+            tmem_ld16(tcol + 16, b);
+            tmem_wait_ld(a, b);
+            mma_quad(xb, 0, a);
+            tmem_ld16(tcol + 32, a);
+            mma_quad(xb, 1, b);
+            tmem_wait_ld(a);
+            tmem_ld16(tcol + 48, b);
+            mma_quad(xb, 2, a);
+            tmem_wait_ld(b);
+            mma_quad(xb, 3, b);
+            unit_done(u);
+        }
+        // parked in part: quad by quad
+        if (tq_part > 0 && u < nwu) {
+            const uint16_t* xb = xs + xrow * P.x_stride + sg * kSgCols + 4 * t4;
+            const uint32_t tcol = tw + (uint32_t)(64 * u);
+            uint32_t w[4 * V];
+            next_stage(w);
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 uint32_t a[16];
-                if (q < tq) {
+                if (q < tq_part) {
                     tmem_ld16(tcol + 16 * q, a);
-                    tmem_wait_ld();
+                    tmem_wait_ld(a);
                 } else {
                     decode_quad<BITS>(tg, tg8, w, q, a);
                 }
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const uint2 xv = *reinterpret_cast<const uint2*>(xb + (4 * q + j) * 16);
-                    if (j & 1)
-                        tc::mma16816(d1, a[4 * j], a[4 * j + 1], a[4 * j + 2], a[4 * j + 3], xv.x, xv.y);
-                    else
-                        tc::mma16816(d0, a[4 * j], a[4 * j + 1], a[4 * j + 2], a[4 * j + 3], xv.x, xv.y);
-                }
+                mma_quad(xb, q, a);
             }
-            if (++sg == nsg || u + 1 == nwu) {
-                flush_tile();
-                __syncwarp();  // the tcgen05 loads that follow need the whole warp
-                if (u + 1 < nwu) {
-                    ++tile;
-                    sg = 0;
-                    start_tile();
-                }
-            }
+            unit_done(u);
+            ++u;
         }
+        // the sparse shares: the warps of the lower half before their decode
+        // loop, the others after it, so that every sub-partition has a warp
+        // decoding while another waits on the shares' loads
+        const bool sparse_first = warp < (NW / 2);
+        auto run_shares = [&]() {
+            if (has_csr)
+#pragma unroll
+                for (int r = 0; r < RG; ++r) sparse_share((warp * RG + r) * 32 + lane, srow[r]);
+            __syncwarp();
+        };
+        if (sparse_first) run_shares();
+        // the rest: decoded here
+#pragma unroll 1
+        for (; u < nwu; ++u) {
+            const uint16_t* xb = xs + xrow * P.x_stride + sg * kSgCols + 4 * t4;
+            uint32_t w[4 * V];
+            next_stage(w);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                uint32_t a[16];
+                decode_quad<BITS>(tg, tg8, w, q, a);
+                mma_quad(xb, q, a);
+            }
+            unit_done(u);
+        }
+        if (!sparse_first) run_shares();
     }
+    if (!waits_ok) atomicOr(p.status, tc::kStatusWaitTimeout);
 
-    // ---- tiles shared by several warps: once every warp has left its loop,
-    // the warps' parts are added in warp order and the rows get their sparse
-    // sums; the control warp frees TMEM (every tcgen05.ld has completed)
+    // ---- once every warp has left its loop: each output is the tile's sum
+    // (or the virtual warps' parts of a shared tile, in order) plus the row's
+    // sparse sum (interior sum, then the pieces of the shares that cut the
+    // row, in share order); the control warp frees TMEM (every tcgen05.ld
+    // has completed)
     tmem_fence_before();
     __syncthreads();
     tmem_fence_after();
     if (ctrl) tmem_dealloc(taddr, kTmemCols);
-    csr_ready = true;  // the control warp wrote the sparse sums before the barrier
     for (int idx = tid; idx < ctiles * TE; idx += kThreads) {
         const int tl = idx / TE, e = idx - tl * TE;
-        const int mask = s_tinfo[tl];
-        if ((mask & (mask - 1)) == 0) continue;  // one warp: already written
         const int row_l = e / CM, col = e - row_l * CM;
         const int tile = t_first + tl;
-        float sum = 0.f;
-        for (int mm = mask; mm; mm &= mm - 1) {
-            const int wv = __ffs(mm) - 1;
-            const int wfirst_v = (u0 + cn * wv / kDenseWarps) / nsg;
-            sum += s_slots[(wv * 2 + (tile == wfirst_v ? 0 : 1)) * TE + e];
-        }
         const int row = tile * kTileRows + row_l;
-        if (row < p.n_out && col < B) p.y[col * p.ldy + row] = f2h_rn(sum + csr_row_sum(row - ra, col));
+        if (row >= p.n_out || col >= B) continue;
+        const int mask = s_tinfo[tl];
+        float sum = 0.f;
+        if ((mask & (mask - 1)) == 0) {
+            sum = s_tsum[idx];
+        } else {
+            for (int mm = mask; mm; mm &= mm - 1) {
+                const int v = __ffs(mm) - 1;
+                const int vfirst_v = vbeg(v) / nsg;
+                sum += s_slots[(v * 2 + (tile == vfirst_v ? 0 : 1)) * TE + e];
+            }
+        }
+        if (has_csr) {
+            const int i = row - ra, rs = s_rp[i], re = s_rp[i + 1];
+            if (re > rs) {
+                float cs = s_rowsum[i * CM + col];
+                const int tau_a = (rs - q0) / e_per, tau_b = min(kVThreads - 1, (re - 1 - q0) / e_per);
+                for (int tau = tau_a; tau <= tau_b; ++tau) {
+                    if (s_headrow[tau] == i) cs += s_head[tau * CM + col];
+                    if (s_tailrow[tau] == i) cs += s_tail[tau * CM + col];
+                }
+                sum += cs;
+            }
+        }
+        p.y[col * p.ldy + row] = f2h_rn(sum);
     }
 }
 

@@ -76,7 +76,7 @@ struct sqz_layer {
     int smem_budget = 232448;  // shared memory of one fused CTA (kCtasPerSm of them share an SM)
     int mac = SQZ_MAC_TENSOR_CORES;
     int csr_mode = SQZ_CSR_BALANCED;
-    int predecode = 1;  // batches of 1..8: the kernel that decodes ahead of x into TMEM
+    int predecode = 0;  // batches of 1..8: 1/8/16 take the kernel that decodes ahead of x into TMEM
     // The fused kernel serves every layer with N > 0 and K > 0 (columns past
     // K are padded inside the kernel-native layout).
     bool fused_ok = false;
@@ -233,25 +233,45 @@ sqz_status prepare_fused_kernels(int optin) {
     sqz_status st = prepare_fused_bits<3>(optin);
     if (st != SQZ_OK) return st;
     if ((st = prepare_fused_bits<4>(optin)) != SQZ_OK) return st;
-    SQZ_CUDA_TRY(cudaFuncSetAttribute(sqz::pd::gemv_pd_kernel<3, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      optin), "cudaFuncSetAttribute");
-    SQZ_CUDA_TRY(cudaFuncSetAttribute(sqz::pd::gemv_pd_kernel<3, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      optin), "cudaFuncSetAttribute");
-    SQZ_CUDA_TRY(cudaFuncSetAttribute(sqz::pd::gemv_pd_kernel<4, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      optin), "cudaFuncSetAttribute");
-    SQZ_CUDA_TRY(cudaFuncSetAttribute(sqz::pd::gemv_pd_kernel<4, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      optin), "cudaFuncSetAttribute");
+#define SQZ_PD_ATTR(BITS, SB, NW)                                                                            \
+    SQZ_CUDA_TRY(cudaFuncSetAttribute(sqz::pd::gemv_pd_kernel<BITS, SB, NW>,                                 \
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, optin),                   \
+                 "cudaFuncSetAttribute")
+    SQZ_PD_ATTR(3, true, 8);
+    SQZ_PD_ATTR(3, false, 8);
+    SQZ_PD_ATTR(4, true, 8);
+    SQZ_PD_ATTR(4, false, 8);
+    SQZ_PD_ATTR(3, true, 16);
+    SQZ_PD_ATTR(3, false, 16);
+    SQZ_PD_ATTR(4, true, 16);
+    SQZ_PD_ATTR(4, false, 16);
+#undef SQZ_PD_ATTR
     return SQZ_OK;
 }
 
+bool tc_grid_too_large(int n_out, int sm_count) { return sqz::tc::grid_size(n_out, sm_count) > sqz::tc::kMaxCtas; }
+
 // The decode-ahead kernel's plan for a call, or false when it does not serve
-// it (batch above 8, or x and the rings do not fit in one CTA's shared
-// memory).
-bool pd_plan_for(int bits, int n_out, int k_in, int sm_count, int smem_optin, int batch, sqz::pd::Plan* out) {
+// it (batch above 8, or x and the rings do not fit one CTA's shared memory).
+// Two CTAs of 8 dense warps per SM when they fit in half an SM (`smem_half`),
+// else one CTA of 16 dense warps; `force_nw` (8 or 16) asks for one shape.
+bool pd_plan_for(int bits, int n_out, int k_in, int sm_count, int smem_half, int smem_optin, int batch, int force_nw,
+                 sqz::pd::Plan* out, int* nw) {
     if (batch < 1 || batch > 8 || n_out < 1 || k_in < 1) return false;
-    const sqz::pd::Plan P = sqz::pd::make_plan(bits, n_out, k_in, batch, sm_count, smem_optin);
-    if (P.total > smem_optin || P.grid > sqz::tc::kMaxCtas) return false;
+    if (tc_grid_too_large(n_out, sm_count)) return false;
+    if (force_nw != 16) {
+        const sqz::pd::Plan P = sqz::pd::make_plan(bits, n_out, k_in, batch, sm_count, smem_half, 8);
+        if (P.total <= smem_half) {
+            *out = P;
+            *nw = 8;
+            return true;
+        }
+        if (force_nw == 8) return false;
+    }
+    const sqz::pd::Plan P = sqz::pd::make_plan(bits, n_out, k_in, batch, sm_count, smem_optin, 16);
+    if (P.total > smem_optin) return false;
     *out = P;
+    *nw = 16;
     return true;
 }
 
@@ -363,11 +383,11 @@ cudaError_t launch_fused_bits(const sqz::tc::Params& prm, int batch, int mac, in
     return launch_fused<BITS, 1, kMacTensor, true>(prm, s);
 }
 
-template <int BITS>
+template <int BITS, int NW>
 cudaError_t launch_pd(const sqz::pd::Params& prm, bool single, cudaStream_t s) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)prm.plan.grid);
-    cfg.blockDim = dim3(sqz::pd::kThreads);
+    cfg.blockDim = dim3(sqz::pd::Shape<NW>::kThreads);
     cfg.dynamicSmemBytes = (size_t)prm.plan.total;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
@@ -375,22 +395,25 @@ cudaError_t launch_pd(const sqz::pd::Params& prm, bool single, cudaStream_t s) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return single ? cudaLaunchKernelEx(&cfg, sqz::pd::gemv_pd_kernel<BITS, true>, prm)
-                  : cudaLaunchKernelEx(&cfg, sqz::pd::gemv_pd_kernel<BITS, false>, prm);
+    return single ? cudaLaunchKernelEx(&cfg, sqz::pd::gemv_pd_kernel<BITS, true, NW>, prm)
+                  : cudaLaunchKernelEx(&cfg, sqz::pd::gemv_pd_kernel<BITS, false, NW>, prm);
 }
 
 // Whether a call takes the decode-ahead kernel: the handle's default options
 // (tensor cores, balanced outliers), batch 1..8 and a plan that fits.
-bool pd_serves(const sqz_layer* L, int32_t batch, sqz::pd::Plan* P) {
+bool pd_serves(const sqz_layer* L, int32_t batch, sqz::pd::Plan* P, int* nw) {
     return L->fused_ok && L->predecode && L->mac == SQZ_MAC_TENSOR_CORES && L->csr_mode == SQZ_CSR_BALANCED &&
-           pd_plan_for(L->bits, L->n_out, L->k_in, L->sm_count, L->smem_optin, batch, P) && P->grid == L->grid;
+           pd_plan_for(L->bits, L->n_out, L->k_in, L->sm_count, L->smem_budget, L->smem_optin, batch,
+                       L->predecode == 1 ? 0 : L->predecode, P, nw) &&
+           P->grid == L->grid;
 }
 
 sqz_status gemv_impl(const sqz_layer* L, const uint16_t* x, int32_t batch, int64_t ldx, uint16_t* y, int64_t ldy,
                      cudaStream_t s) {
     if (L->n_out == 0) return SQZ_OK;
     sqz::pd::Plan PP;
-    if (pd_serves(L, batch, &PP)) {
+    int nw = 0;
+    if (pd_serves(L, batch, &PP, &nw)) {
         sqz::pd::Params prm{};
         prm.codes = L->codes_native;
         prm.lutp = L->lut_native;
@@ -411,7 +434,9 @@ sqz_status gemv_impl(const sqz_layer* L, const uint16_t* x, int32_t batch, int64
         prm.x_bulk = (reinterpret_cast<uintptr_t>(x) % 16 == 0) && (ldx % 8 == 0) && (L->k_in % 8 == 0);
         prm.plan = PP;
         prm.csr_cta = L->csr_cta;
-        const cudaError_t e = L->bits == 3 ? launch_pd<3>(prm, batch == 1, s) : launch_pd<4>(prm, batch == 1, s);
+        const bool one = batch == 1;
+        const cudaError_t e = L->bits == 3 ? (nw == 8 ? launch_pd<3, 8>(prm, one, s) : launch_pd<3, 16>(prm, one, s))
+                                           : (nw == 8 ? launch_pd<4, 8>(prm, one, s) : launch_pd<4, 16>(prm, one, s));
         SQZ_CUDA_TRY(e, "fused gemv launch");
         return SQZ_OK;
     }
@@ -733,7 +758,7 @@ sqz_status sqz_gemv_host(sqz_layer_t layer, const uint16_t* x_host, int32_t batc
 }
 
 sqz_status sqz_plan_query(int32_t n_out, int32_t k_in, int32_t bits, int32_t batch, int32_t sm_count,
-                          int32_t smem_per_sm, int32_t smem_optin, sqz_plan_info* out) {
+                          int32_t smem_per_sm, int32_t smem_optin, int32_t predecode, sqz_plan_info* out) {
     if (!out) return fail(SQZ_ERR_INVALID_ARG, "out is NULL");
     *out = sqz_plan_info{};
     if (bits != 3 && bits != 4) return fail(SQZ_ERR_INVALID_ARG, "bits must be 3 or 4 (got %d)", bits);
@@ -745,15 +770,20 @@ sqz_status sqz_plan_query(int32_t n_out, int32_t k_in, int32_t bits, int32_t bat
     const DeviceShape d{sm_count, share < smem_optin ? share : smem_optin, smem_optin};
     const int grid = sqz::tc::grid_size(n_out, sm_count);
     sqz::pd::Plan PP;
-    if (grid <= sqz::tc::kMaxCtas && pd_plan_for(bits, n_out, k_in, sm_count, smem_optin, batch, &PP)) {
+    int nw = 0;
+    if (predecode != 0 && predecode != 1 && predecode != 8 && predecode != 16)
+        return fail(SQZ_ERR_INVALID_ARG, "predecode must be 0, 1, 8 or 16 (got %d)", predecode);
+    if (predecode &&
+        pd_plan_for(bits, n_out, k_in, sm_count, d.smem_half, smem_optin, batch, predecode == 1 ? 0 : predecode, &PP,
+                    &nw)) {
         out->fused = 1;
         out->predecode = 1;
         out->columns_per_launch = batch;
         out->launches = 1;
         out->grid = PP.grid;
-        out->threads = sqz::pd::kThreads;
+        out->threads = (nw + 1) * 32;
         out->smem_bytes = PP.total;
-        out->ctas_per_sm = 1;
+        out->ctas_per_sm = nw == 8 ? 2 : 1;
         out->passes = 1;
         out->ring_stages = sqz::pd::kStages;
         out->csr_stage_entries = PP.csr_cap;
@@ -827,7 +857,8 @@ sqz_status sqz_layer_set_csr_mode(sqz_layer_t layer, int32_t mode) {
 
 sqz_status sqz_layer_set_predecode(sqz_layer_t layer, int32_t enable) {
     if (!layer) return fail(SQZ_ERR_INVALID_ARG, "layer is NULL");
-    if (enable != 0 && enable != 1) return fail(SQZ_ERR_INVALID_ARG, "enable must be 0 or 1 (got %d)", enable);
+    if (enable != 0 && enable != 1 && enable != 8 && enable != 16)
+        return fail(SQZ_ERR_INVALID_ARG, "enable must be 0, 1, 8 or 16 (got %d)", enable);
     layer->predecode = enable;
     drop_host_graphs(layer);
     return SQZ_OK;

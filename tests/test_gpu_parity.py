@@ -469,25 +469,60 @@ def test_layer_holds_the_compressed_weights_once(B, wl):
     (300, 4096, 3, 5000, 1), (257, 1032, 4, 1000, 3), (2000, 3072, 3, 30000, 8), (5000, 512, 4, 0, 2),
     (33, 96, 3, 10, 1), (4100, 2048, 4, 9000, 5), (150, 20000, 3, 400, 1)])
 def test_decode_ahead_and_plain_kernels_match_oracle(B, orc, n_out, k_in, bits, nnz, batch):
-    """Batches of 1..8 take by default the kernel that decodes ahead of x
-    into tensor memory; the kernel without that step must agree with the
-    oracle on the same inputs too, and the decode-ahead results must not
-    depend on how many quads a warp parked before x arrived (the same MMAs
-    run in the same order either way): repeated calls are bit-identical."""
+    """The kernel that decodes ahead of x into tensor memory (an option of
+    the handle, batches of 1..8) and the default kernel agree with the oracle
+    on the same inputs; the two CTA shapes of the decode-ahead kernel give the
+    same bits, and its results do not depend on how many quads a warp parked
+    before x arrived (the same MMAs run in the same order either way)."""
     L = make_small(90 + n_out % 17, n_out, k_in, bits, nnz)
     x = synth.make_x(batch, k_in, seed=3, key="pd")
     layer = upload(B, L)
     y_ref, bound = orc.gemv_layer(L, x)
-    plan = B.sqz_plan_query(n_out, k_in, bits, batch)
-    assert plan["predecode"] == 1
+    y_plain = gpu_gemv(B, layer, x)
+    assert_close(y_plain, y_ref, bound, "default kernel")
+    assert B.sqz_plan_query(n_out, k_in, bits, batch, predecode=1)["predecode"] == 1
+    B.sqz_layer_set_predecode(layer, 1)
     y_pd = gpu_gemv(B, layer, x)
     assert_close(y_pd, y_ref, bound, "decode-ahead")
     for _ in range(3):
         assert np.array_equal(gpu_gemv(B, layer, x), y_pd)
-    B.sqz_layer_set_predecode(layer, False)
-    y_plain = gpu_gemv(B, layer, x)
-    assert_close(y_plain, y_ref, bound, "plain")
-    B.sqz_layer_set_predecode(layer, True)
-    assert np.array_equal(gpu_gemv(B, layer, x), y_pd)
+    for shape_nw in (8, 16):
+        plan = B.sqz_plan_query(n_out, k_in, bits, batch, predecode=shape_nw)
+        if not plan["predecode"]:
+            continue  # that CTA shape does not fit this call
+        assert plan["threads"] == (shape_nw + 1) * 32
+        B.sqz_layer_set_predecode(layer, shape_nw)
+        assert np.array_equal(gpu_gemv(B, layer, x), y_pd), f"decode-ahead with {shape_nw} dense warps"
+    B.sqz_layer_set_predecode(layer, 0)
+    assert np.array_equal(gpu_gemv(B, layer, x), y_plain)
     assert B.sqz_layer_status(layer) == 0
     layer.close()
+
+
+def test_decode_ahead_chained_calls_read_the_previous_output(B, orc):
+    """The decode-ahead kernel starts decoding before the previous kernel of
+    the stream has finished; x must still be read only after it has."""
+    dims = [4096, 1024, 2048, 4096, 512]
+    layers, hosts = [], []
+    for i in range(len(dims) - 1):
+        L = make_small(170 + i, dims[i + 1], dims[i], 3 if i % 2 == 0 else 4, dims[i + 1] * 3)
+        hosts.append(L)
+        layers.append(upload(B, L))
+        B.sqz_layer_set_predecode(layers[-1], 1)
+    x0 = synth.make_x(1, dims[0], seed=14)
+    bufs = [torch.from_numpy(x0.view(np.int16)).cuda()]
+    for d in dims[1:]:
+        bufs.append(torch.full((1, d), 0x7E00, dtype=torch.int16, device="cuda"))
+    torch.cuda.synchronize()
+    for rep in range(3):
+        for i, layer in enumerate(layers):
+            B.sqz_gemv(layer, bufs[i], bufs[i + 1])
+        torch.cuda.synchronize()
+        x = x0
+        for i, L in enumerate(hosts):
+            y = bufs[i + 1].cpu().numpy().view(np.uint16)
+            y_ref, bound = orc.gemv_layer(L, x)
+            assert_close(y, y_ref, bound, f"rep {rep} layer {i}")
+            x = y
+        for b in bufs[1:]:
+            b.fill_(0x7E00)

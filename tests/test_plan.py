@@ -1,8 +1,9 @@
 """The launch plan (host logic, no GPU): for every workload shape and every
 batch size a fused kernel serves the call with a plan that fits the shared
-memory it claims.  Batches of 1..8 whose x fits take the decode-ahead kernel
-(one CTA of 17 warps per SM, more than half the SM's shared memory so that
-no second CTA of it can be resident and wait for its tensor memory); the
+memory it claims.  With the decode-ahead option, batches of 1..8 whose x
+fits take that kernel (two CTAs of 9 warps per SM, each within half the SM,
+or one CTA of 17 warps taking more than half of it, so that at most two of
+its CTAs share an SM's tensor memory); by default, and otherwise, the
 others take the 12-warp kernel, whose single-pass launches use the fixed 3-
 or 4-stage code ring (its compile-time waits depend on it), and whose
 batches above 8 run as one-pass launches of 8 columns when those fit while
@@ -34,12 +35,7 @@ def test_every_batch_gets_a_fitting_fused_plan(shape):
         assert p["launches"] * p["columns_per_launch"] >= batch
         assert (p["launches"] - 1) * p["columns_per_launch"] < batch
         assert p["csr_stage_entries"] >= 0 and p["csr_stage_entries"] % 8 == 0
-        if p["predecode"]:
-            assert batch <= 8
-            assert p["threads"] == 17 * 32 and p["ctas_per_sm"] == 1
-            assert DEV["smem_per_sm"] // 2 < p["smem_bytes"] <= DEV["smem_optin"]
-            assert (p["launches"], p["passes"], p["ring_stages"]) == (1, 1, 4)
-            continue
+        assert p["predecode"] == 0  # the default: the 12-warp kernel
         assert p["threads"] == 384
         budget = HALF if p["ctas_per_sm"] == 2 else DEV["smem_optin"]
         assert 0 < p["smem_bytes"] <= budget
@@ -47,18 +43,42 @@ def test_every_batch_gets_a_fitting_fused_plan(shape):
             assert p["ring_stages"] in (3, 4)
         else:
             assert p["ring_stages"] >= 2
-        assert batch > 1, "batch 1 of every workload shape takes the decode-ahead kernel"
+        if batch == 1:
+            assert p["passes"] == 1 and p["launches"] == 1
+            assert p["ctas_per_sm"] == 2, "batch 1 must leave room for the next call's CTA"
 
 
-def test_decode_ahead_kernel_serves_batches_up_to_eight_whose_x_fits():
-    x_fits = lambda k, b: b * (((k + 255) // 256 * 512 + 127) // 128 * 128 + 32)
+@pytest.mark.parametrize("shape", list(shapes()), ids=lambda s: f"{s.n_out}x{s.k_in}b{s.bits}")
+def test_decode_ahead_plans_fit(shape):
+    for batch in range(1, 17):
+        p = B.sqz_plan_query(shape.n_out, shape.k_in, shape.bits, batch, **DEV, predecode=1)
+        assert p["fused"] == 1, (shape.key, batch)
+        if not p["predecode"]:
+            continue
+        assert batch <= 8
+        assert (p["launches"], p["passes"], p["ring_stages"]) == (1, 1, 4)
+        assert p["grid"] == min(DEV["sm_count"], (shape.n_out + 15) // 16)
+        if p["threads"] == 9 * 32:  # two CTAs of 8 dense warps per SM, half the SM each
+            assert p["ctas_per_sm"] == 2 and 0 < p["smem_bytes"] <= HALF
+        else:  # one CTA of 16 dense warps, more than half the SM: no second one fits
+            assert p["threads"] == 17 * 32 and p["ctas_per_sm"] == 1
+            assert DEV["smem_per_sm"] // 2 < p["smem_bytes"] <= DEV["smem_optin"]
+
+
+def test_decode_ahead_kernel_serves_small_batches_and_never_above_eight():
     for n, k, bits in ((11008, 4096, 3), (4096, 4096, 4), (5120, 13824, 3), (8192, 22016, 3)):
         for batch in range(1, 17):
-            p = B.sqz_plan_query(n, k, bits, batch, **DEV)
+            p = B.sqz_plan_query(n, k, bits, batch, **DEV, predecode=1)
             if batch > 8:
                 assert p["predecode"] == 0
-            elif x_fits(k, batch) <= 64 * 1024:
+            elif batch == 1 or (batch == 2 and k <= 13824):
                 assert p["predecode"] == 1, (n, k, batch)
+
+
+def test_batch_one_of_every_workload_shape_shares_the_sm_with_the_next_call():
+    for shape in shapes():
+        p = B.sqz_plan_query(shape.n_out, shape.k_in, shape.bits, 1, **DEV, predecode=1)
+        assert p["predecode"] == 1 and p["ctas_per_sm"] == 2, shape.key
 
 
 def test_large_batches_split_into_single_pass_launches_of_eight():
