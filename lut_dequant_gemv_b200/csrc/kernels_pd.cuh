@@ -174,6 +174,31 @@ struct Params {
     const int32_t* csr_cta;  // [grid + 1]: CSR entry range of each CTA's rows
 };
 
+// ------------------------------------------------------- per-SM hand-over
+// Decoding ahead pays only while the SM has nothing else to do: in a chain of
+// calls the next call's CTA is resident long before the current one has
+// finished its dense loop, and decoding then would only take integer issue
+// from it.  So every CTA of this kernel takes a ticket from its SM's start
+// counter and, once its dense warps are done, bumps its SM's "loop done"
+// counter; a CTA starts decoding ahead once every CTA of this kernel that
+// started on its SM before it has finished its dense loop (or once its x has
+// arrived).  The counters are hints only: the wait ends on either condition
+// and is bounded, and it never orders anything that results depend on.
+constexpr int kSmSlots = 256;
+__device__ unsigned int g_pd_started[kSmSlots];
+__device__ unsigned int g_pd_looped[kSmSlots];
+__device__ __forceinline__ unsigned int sm_id() {
+    unsigned int r;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ unsigned int ld_relaxed(const unsigned int* p) {
+    unsigned int v;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+constexpr int kGatePolls = 20000;  // x 256 ns: the gate gives up after about 5 ms
+
 // ---------------------------------------------------------------- helpers
 __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
     uint32_t ok;
@@ -305,8 +330,11 @@ __global__ void __launch_bounds__(Shape<NW>::kThreads, Shape<NW>::kCtasPerSm)
 
     // ---- control warp: barriers, copies of the weights (independent of the
     // previous kernel), the L2 prefetch of the CTA's codes, TMEM
+    const unsigned int smslot = sm_id() % kSmSlots;
+    unsigned int* s_ticket = reinterpret_cast<unsigned int*>(smem + P.off_taddr + 4);
     if (ctrl) {
         if (lane == 0) {
+            *s_ticket = atomicAdd(&g_pd_started[smslot], 1u);
             tc::mbar_init(lbar, 1);
             tc::mbar_init(xbar, p.x_bulk ? 1 : 32);  // bulk: one expect_tx; else every lane after its stores
             tc::mbar_init(cbar, 1);
@@ -365,6 +393,7 @@ __global__ void __launch_bounds__(Shape<NW>::kThreads, Shape<NW>::kCtasPerSm)
     __syncthreads();
     tmem_fence_after();
     const uint32_t taddr = *s_taddr;
+    const unsigned int ticket = *s_ticket;
 
     if (ctrl) {
         // ---- x may be written by the previous kernel of the stream: wait
@@ -512,6 +541,16 @@ __global__ void __launch_bounds__(Shape<NW>::kThreads, Shape<NW>::kCtasPerSm)
         // is in shared memory (checked before every quad)
         int qp = 0;  // quads parked
         int s_read = 0, s_fill = D;
+        // the SM's earlier CTAs of this kernel first (see g_pd_looped)
+        if (nwu > 0) {
+            bool go = false;
+            for (int i = 0; i < kGatePolls && !go; ++i) {
+                bool t = false;
+                if (lane == 0) t = mbar_test(xbar, 0) || (int)(ld_relaxed(&g_pd_looped[smslot]) - ticket) >= 0;
+                go = __shfl_sync(0xffffffffu, t, 0);
+                if (!go) __nanosleep(256);
+            }
+        }
         if (nwu > 0) {
             const int pre = min(nwu, kPreUnits);
             int tab_tile = -1;
@@ -705,6 +744,7 @@ __global__ void __launch_bounds__(Shape<NW>::kThreads, Shape<NW>::kCtasPerSm)
     __syncthreads();
     tmem_fence_after();
     if (ctrl) tmem_dealloc(taddr, kTmemCols);
+    if (tid == 0) atomicAdd(&g_pd_looped[smslot], 1u);  // this CTA's dense loops are done
     for (int idx = tid; idx < ctiles * TE; idx += kThreads) {
         const int tl = idx / TE, e = idx - tl * TE;
         const int row_l = e / CM, col = e - row_l * CM;
