@@ -64,7 +64,6 @@ using tc::kSgCols;
 using tc::kSgSteps;
 using tc::kTileRows;
 using tc::round_up;
-using tc::tile_begin;
 
 // Two shapes of CTA (template argument NW, the dense warps):
 //   NW = 8:  8 dense warps + the control warp, two CTAs per SM, each with half
@@ -105,7 +104,8 @@ struct Plan {
 };
 
 // Shared-memory plan of a launch; total > budget when it does not fit.
-__host__ __device__ inline Plan make_plan(int bits, int n_out, int k_in, int batch, int sms, int budget, int nw) {
+__host__ __device__ inline Plan make_plan(int bits, int n_out, int k_in, int batch, int sms, int budget, int nw,
+                                          int ctiles_max = 0) {
     Plan P{};
     const int min_smem = nw == 8 ? Shape<8>::kMinSmem : Shape<16>::kMinSmem;
     const int ntiles = (n_out + kTileRows - 1) / kTileRows;
@@ -114,6 +114,7 @@ __host__ __device__ inline Plan make_plan(int bits, int n_out, int k_in, int bat
     const int sg_bytes = bits == 3 ? 1536 : 2048;
     P.grid = tc::grid_size(n_out, sms);
     P.ctiles_max = (ntiles + P.grid - 1) / P.grid;
+    if (ctiles_max > P.ctiles_max) P.ctiles_max = ctiles_max;
     P.cm = batch == 1 ? 1 : 8;
     // x rows: stride = 32 (mod 128) bytes keeps the batch rows of one
     // fragment load in different banks
@@ -172,6 +173,7 @@ struct Params {
     int64_t ldy;
     int* status;
     const int32_t* csr_cta;  // [grid + 1]: CSR entry range of each CTA's rows
+    const int32_t* cta_tiles;  // [grid + 1]: first tile of each CTA, or nullptr (the even split)
 };
 
 // ------------------------------------------------------- per-SM hand-over
@@ -296,7 +298,8 @@ __global__ void __launch_bounds__(Shape<NW>::kThreads, Shape<NW>::kCtasPerSm)
     const bool ctrl = warp == kCtrlWarp;
     const int G = gridDim.x, c = blockIdx.x;
     const int nsg = p.nsg;
-    const int t_first = tile_begin(p.ntiles, G, c), t_end = tile_begin(p.ntiles, G, c + 1);
+    int t_first, t_end;
+    tc::cta_tile_range(p.cta_tiles, p.ntiles, G, c, t_first, t_end);
     const int ctiles = t_end - t_first;
     const int u0 = t_first * nsg, cn = ctiles * nsg;
     // virtual warp v: units [vbeg(v), vbeg(v + 1)) of the CTA; dense warp w

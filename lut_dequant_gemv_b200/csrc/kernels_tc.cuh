@@ -172,8 +172,9 @@ __host__ __device__ inline int grid_size(int n_out, int sms) {
 // rest; total > budget when not even kMinStages fit.
 // `passes` > 1 stages x in K chunks of chunk_sg super-groups (two buffers)
 // and keeps per-tile sums in shared memory between passes.
+// `ctiles_max`: the most tiles one CTA owns (0: the even split's).
 __host__ __device__ inline Plan make_plan(int bits, int n_out, int k_in, int batch, int nt, bool single, int sms,
-                                          int budget, int passes = 1) {
+                                          int budget, int passes = 1, int ctiles_max = 0) {
     Plan P{};
     const int ntiles = (n_out + kTileRows - 1) / kTileRows;
     const int nsteps = (k_in + 15) / 16;
@@ -181,6 +182,7 @@ __host__ __device__ inline Plan make_plan(int bits, int n_out, int k_in, int bat
     const int lut_bytes = bits == 3 ? 16 : 32;
     P.grid = grid_size(n_out, sms);
     P.ctiles_max = (ntiles + P.grid - 1) / P.grid;
+    if (ctiles_max > P.ctiles_max) P.ctiles_max = ctiles_max;
     P.cm = single ? 1 : 8 * nt;
     P.passes = passes < 1 ? 1 : (passes > nsg ? nsg : passes);
     P.chunk_sg = (nsg + P.passes - 1) / P.passes;
@@ -266,7 +268,23 @@ struct Params {
     // out of the parameters: a small parameter block stays in the constant
     // cache, whose misses cost hundreds of cycles wherever a field is reread.
     const int32_t* csr_cta;
+    // First tile of CTA c: cta_tiles[c] (grid + 1 values) when the layer's
+    // outliers are skewed enough for a split by weight (tiles + nonzeros);
+    // nullptr: the even split of tile_begin.
+    const int32_t* cta_tiles;
 };
+
+// Tiles [first, end) of CTA c.
+__device__ __forceinline__ void cta_tile_range(const int32_t* cta_tiles, int ntiles, int grid, int c, int& first,
+                                               int& end) {
+    if (cta_tiles) {
+        first = __ldg(cta_tiles + c);
+        end = __ldg(cta_tiles + c + 1);
+    } else {
+        first = tile_begin(ntiles, grid, c);
+        end = tile_begin(ntiles, grid, c + 1);
+    }
+}
 
 // ------------------------------------------------------------- PTX helpers
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
@@ -511,10 +529,10 @@ __global__ void repack_lut_kernel(const uint16_t* __restrict__ lut, int32_t n_ou
 
 // CSR entry range of each CTA's rows: out[c] = rowptr[first row of CTA c],
 // c = 0..grid (the last value is rowptr[n_out]).
-__global__ void csr_cta_bounds_kernel(const int32_t* __restrict__ rowptr, int32_t n_out, int ntiles, int grid,
-                                      int32_t* __restrict__ out) {
+__global__ void csr_cta_bounds_kernel(const int32_t* __restrict__ rowptr, const int32_t* __restrict__ cta_tiles,
+                                      int32_t n_out, int ntiles, int grid, int32_t* __restrict__ out) {
     for (int c = blockIdx.x * blockDim.x + threadIdx.x; c <= grid; c += gridDim.x * blockDim.x) {
-        const int64_t r = (int64_t)tile_begin(ntiles, grid, c) * kTileRows;
+        const int64_t r = (int64_t)(cta_tiles ? cta_tiles[c] : tile_begin(ntiles, grid, c)) * kTileRows;
         out[c] = rowptr[r < n_out ? r : n_out];
     }
 }
@@ -588,7 +606,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_fused_kernel(const 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t4 = lane & 3;
     const int G = gridDim.x, c = blockIdx.x;
     const int nsg = p.nsg;
-    const int t_first = tile_begin(p.ntiles, G, c), t_end = tile_begin(p.ntiles, G, c + 1);
+    int t_first, t_end;
+    cta_tile_range(p.cta_tiles, p.ntiles, G, c, t_first, t_end);
     const int ctiles = t_end - t_first;
     const int u0 = t_first * nsg, cn = ctiles * nsg;  // the CTA's units: [u0, u0 + cn)
     const int shift = p.has_csr ? kCsrUnitShift : 0;

@@ -9,6 +9,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <algorithm>
 #include <new>
 #include <string>
 #include <vector>
@@ -95,6 +96,8 @@ struct sqz_layer {
     int64_t units = 0;
     int grid = 0;                     // CTAs of a fused launch (one per SM)
     int32_t* csr_cta = nullptr;       // [grid + 1] (device): CSR entry range of each CTA's rows
+    int32_t* cta_tiles = nullptr;     // [grid + 1] (device): first tile of each CTA, or nullptr (even split)
+    int ctiles_max = 0;               // the most tiles one CTA owns
     uint8_t* codes_native = nullptr;  // [ntiles][nsg][sg_bytes]
     uint8_t* lut_native = nullptr;    // [ntiles*16][2 << bits] byte planes
     int* status = nullptr;            // [1]
@@ -135,6 +138,7 @@ void free_layer(sqz_layer* L) {
     cudaFree(L->lut_native);
     cudaFree(L->status);
     cudaFree(L->csr_cta);
+    cudaFree(L->cta_tiles);
     cudaFree(L->x_stage);
     cudaFree(L->y_stage);
     delete L;
@@ -256,11 +260,11 @@ bool tc_grid_too_large(int n_out, int sm_count) { return sqz::tc::grid_size(n_ou
 // Two CTAs of 8 dense warps per SM when they fit in half an SM (`smem_half`),
 // else one CTA of 16 dense warps; `force_nw` (8 or 16) asks for one shape.
 bool pd_plan_for(int bits, int n_out, int k_in, int sm_count, int smem_half, int smem_optin, int batch, int force_nw,
-                 sqz::pd::Plan* out, int* nw) {
+                 sqz::pd::Plan* out, int* nw, int ctiles_max = 0) {
     if (batch < 1 || batch > 8 || n_out < 1 || k_in < 1) return false;
     if (tc_grid_too_large(n_out, sm_count)) return false;
     if (force_nw != 16) {
-        const sqz::pd::Plan P = sqz::pd::make_plan(bits, n_out, k_in, batch, sm_count, smem_half, 8);
+        const sqz::pd::Plan P = sqz::pd::make_plan(bits, n_out, k_in, batch, sm_count, smem_half, 8, ctiles_max);
         if (P.total <= smem_half) {
             *out = P;
             *nw = 8;
@@ -268,7 +272,7 @@ bool pd_plan_for(int bits, int n_out, int k_in, int sm_count, int smem_half, int
         }
         if (force_nw == 8) return false;
     }
-    const sqz::pd::Plan P = sqz::pd::make_plan(bits, n_out, k_in, batch, sm_count, smem_optin, 16);
+    const sqz::pd::Plan P = sqz::pd::make_plan(bits, n_out, k_in, batch, sm_count, smem_optin, 16, ctiles_max);
     if (P.total > smem_optin) return false;
     *out = P;
     *nw = 16;
@@ -286,12 +290,13 @@ struct DeviceShape {
     int sm_count, smem_half, smem_optin;
 };
 
-bool plan_for(int bits, int n_out, int k_in, const DeviceShape& d, int batch, sqz::tc::Plan* out) {
+bool plan_for(int bits, int n_out, int k_in, const DeviceShape& d, int batch, sqz::tc::Plan* out, int ctiles_max = 0) {
     const int nt = batch > 8 ? 2 : 1;
     const int grid = sqz::tc::grid_size(n_out, d.sm_count);
     const int nsg = ((k_in + 15) / 16 + sqz::tc::kSgSteps - 1) / sqz::tc::kSgSteps;
     for (int budget : {d.smem_half, d.smem_optin}) {
-        sqz::tc::Plan P = sqz::tc::make_plan(bits, n_out, k_in, batch, nt, batch == 1, d.sm_count, budget);
+        sqz::tc::Plan P =
+            sqz::tc::make_plan(bits, n_out, k_in, batch, nt, batch == 1, d.sm_count, budget, 1, ctiles_max);
         if (P.total <= budget && P.grid == grid) {
             *out = P;
             return true;
@@ -303,7 +308,7 @@ bool plan_for(int bits, int n_out, int k_in, const DeviceShape& d, int batch, sq
         bool have = false;
         for (int passes = 2; passes <= nsg; ++passes) {
             sqz::tc::Plan P =
-                sqz::tc::make_plan(bits, n_out, k_in, batch, nt, false, d.sm_count, d.smem_optin, passes);
+                sqz::tc::make_plan(bits, n_out, k_in, batch, nt, false, d.sm_count, d.smem_optin, passes, ctiles_max);
             if (P.passes != passes || P.total > d.smem_optin || P.grid != grid) continue;
             if (!have) {
                 *out = P;
@@ -320,7 +325,8 @@ bool plan_for(int bits, int n_out, int k_in, const DeviceShape& d, int batch, sq
 }
 
 bool fused_plan(const sqz_layer* L, int batch, sqz::tc::Plan* out) {
-    return plan_for(L->bits, L->n_out, L->k_in, DeviceShape{L->sm_count, L->smem_budget, L->smem_optin}, batch, out);
+    return plan_for(L->bits, L->n_out, L->k_in, DeviceShape{L->sm_count, L->smem_budget, L->smem_optin}, batch, out,
+                    L->ctiles_max);
 }
 
 // Columns per launch and the plan of the first launch: the whole batch when
@@ -330,19 +336,32 @@ bool fused_plan(const sqz_layer* L, int batch, sqz::tc::Plan* out) {
 // gives each warp about one unit per tile, and the passes' barriers then
 // cost more than decoding the weights twice.  Returns 0 when no fused plan
 // exists (the row-per-warp kernel serves the call).
-int launch_columns(int bits, int n_out, int k_in, const DeviceShape& d, int batch, sqz::tc::Plan* P) {
+int launch_columns(int bits, int n_out, int k_in, const DeviceShape& d, int batch, sqz::tc::Plan* P,
+                   int ctiles_max = 0) {
     int chunk = batch;
-    bool fits = plan_for(bits, n_out, k_in, d, chunk, P);
-    if (fits && batch > 8 && P->passes > 1) {
-        sqz::tc::Plan P8;
-        if (plan_for(bits, n_out, k_in, d, 8, &P8) && P8.passes == 1) {
-            chunk = 8;
-            *P = P8;
+    bool fits = plan_for(bits, n_out, k_in, d, chunk, P, ctiles_max);
+    if (fits && P->passes > 1) {
+        // x staged in K chunks: the passes' barriers cost more than decoding
+        // the weights again (from L2) in another launch once there are more
+        // passes than launches -- take the widest single-pass column chunk
+        // whose launches are fewer than the passes (measured on B200:
+        // 5120x13824 at 8 columns, 55 us in 4 passes, 37 us as two launches
+        // of 4).  Above 8 columns, launches of 8 whenever 8 fit one pass.
+        for (int c : {8, 4, 2, 1}) {
+            if (c >= batch) continue;
+            sqz::tc::Plan Pc;
+            if (!plan_for(bits, n_out, k_in, d, c, &Pc, ctiles_max) || Pc.passes != 1) continue;
+            const int launches = (batch + c - 1) / c;
+            if ((batch > 8 && c == 8) || launches < P->passes) {
+                chunk = c;
+                *P = Pc;
+            }
+            break;
         }
     }
     while (!fits && chunk > 1) {
         chunk = chunk > 8 ? 8 : chunk / 2;
-        fits = plan_for(bits, n_out, k_in, d, chunk, P);
+        fits = plan_for(bits, n_out, k_in, d, chunk, P, ctiles_max);
     }
     return fits ? chunk : 0;
 }
@@ -404,7 +423,7 @@ cudaError_t launch_pd(const sqz::pd::Params& prm, bool single, cudaStream_t s) {
 bool pd_serves(const sqz_layer* L, int32_t batch, sqz::pd::Plan* P, int* nw) {
     return L->fused_ok && L->predecode && L->mac == SQZ_MAC_TENSOR_CORES && L->csr_mode == SQZ_CSR_BALANCED &&
            pd_plan_for(L->bits, L->n_out, L->k_in, L->sm_count, L->smem_budget, L->smem_optin, batch,
-                       L->predecode == 1 ? 0 : L->predecode, P, nw) &&
+                       L->predecode == 1 ? 0 : L->predecode, P, nw, L->ctiles_max) &&
            P->grid == L->grid;
 }
 
@@ -434,6 +453,7 @@ sqz_status gemv_impl(const sqz_layer* L, const uint16_t* x, int32_t batch, int64
         prm.x_bulk = (reinterpret_cast<uintptr_t>(x) % 16 == 0) && (ldx % 8 == 0) && (L->k_in % 8 == 0);
         prm.plan = PP;
         prm.csr_cta = L->csr_cta;
+        prm.cta_tiles = L->cta_tiles;
         const bool one = batch == 1;
         const cudaError_t e = L->bits == 3 ? (nw == 8 ? launch_pd<3, 8>(prm, one, s) : launch_pd<3, 16>(prm, one, s))
                                            : (nw == 8 ? launch_pd<4, 8>(prm, one, s) : launch_pd<4, 16>(prm, one, s));
@@ -442,7 +462,8 @@ sqz_status gemv_impl(const sqz_layer* L, const uint16_t* x, int32_t batch, int64
     }
     sqz::tc::Plan P;
     const int chunk = L->fused_ok ? launch_columns(L->bits, L->n_out, L->k_in,
-                                                   DeviceShape{L->sm_count, L->smem_budget, L->smem_optin}, batch, &P)
+                                                   DeviceShape{L->sm_count, L->smem_budget, L->smem_optin}, batch, &P,
+                                                   L->ctiles_max)
                                   : 0;
     const bool fits = chunk > 0;
     if (fits) {
@@ -470,6 +491,7 @@ sqz_status gemv_impl(const sqz_layer* L, const uint16_t* x, int32_t batch, int64
             prm.x_bulk = (reinterpret_cast<uintptr_t>(xc) % 16 == 0) && (ldx % 8 == 0) && (L->k_in % 8 == 0);
             prm.plan = P;
             prm.csr_cta = L->csr_cta;
+            prm.cta_tiles = L->cta_tiles;
             const cudaError_t e = L->bits == 3 ? launch_fused_bits<3>(prm, nb, L->mac, L->csr_mode, s)
                                                : launch_fused_bits<4>(prm, nb, L->mac, L->csr_mode, s);
             SQZ_CUDA_TRY(e, "fused gemv launch");
@@ -483,6 +505,56 @@ sqz_status gemv_impl(const sqz_layer* L, const uint16_t* x, int32_t batch, int64
     }
     SQZ_CUDA_TRY(cudaGetLastError(), "gemv launch");
     return SQZ_OK;
+}
+
+// A split of the tiles over the CTAs by weight, for layers whose outliers
+// are skewed: a CTA's time is its dense units (one per tile and 256-column
+// super-group) plus its share of the sparse part, and a CTA whose rows hold
+// many outliers should own fewer tiles.  Weight of a tile = its units x
+// kNnzPerUnit + its nonzeros (kNnzPerUnit: the nonzeros that cost about as
+// much as one unit's decode, measured on B200); CTA c starts at the first
+// tile whose weight prefix reaches c/grid of the total, every CTA keeping at
+// least one tile and at most twice the even split's count.  Used only when it
+// lowers the heaviest CTA's weight by more than 5 %; otherwise (uniform
+// outliers) the even split stays and `first` is left empty.
+constexpr int64_t kNnzPerUnit = 100;
+bool split_tiles_by_weight(const std::vector<int32_t>& rp, int n_out, int ntiles, int nsg, int grid,
+                           std::vector<int32_t>* first, int* ctiles_max) {
+    std::vector<int64_t> w((size_t)ntiles), pre((size_t)ntiles + 1, 0);
+    for (int t = 0; t < ntiles; ++t) {
+        const int r0 = t * sqz::tc::kTileRows, r1 = std::min(n_out, r0 + sqz::tc::kTileRows);
+        w[t] = (int64_t)nsg * kNnzPerUnit + (rp[r1] - rp[r0]);
+        pre[t + 1] = pre[t] + w[t];
+    }
+    const int even_max = (ntiles + grid - 1) / grid, cap = 2 * even_max;
+    auto heaviest = [&](const std::vector<int32_t>& f) {
+        int64_t m = 0;
+        for (int c = 0; c < grid; ++c) m = std::max(m, pre[f[c + 1]] - pre[f[c]]);
+        return m;
+    };
+    std::vector<int32_t> even((size_t)grid + 1), split((size_t)grid + 1);
+    for (int c = 0; c <= grid; ++c) even[c] = sqz::tc::tile_begin(ntiles, grid, c);
+    split[0] = 0;
+    split[grid] = ntiles;
+    for (int c = 1; c < grid; ++c) {
+        const int64_t target = pre[ntiles] * c / grid;
+        int t = (int)(std::lower_bound(pre.begin(), pre.end(), target) - pre.begin());
+        t = std::max(t, split[c - 1] + 1);              // at least one tile for CTA c - 1
+        t = std::min(t, split[c - 1] + cap);            // at most `cap` tiles for CTA c - 1
+        t = std::min(t, ntiles - (grid - c));           // one tile left for each CTA after it
+        t = std::max(t, ntiles - (grid - c) * cap);     // no CTA after it above `cap`
+        split[c] = t;
+    }
+    int m = 0;
+    for (int c = 0; c < grid; ++c) {
+        const int n = split[c + 1] - split[c];
+        if (n < 1 || n > cap) return false;  // the bounds could not all be met: keep the even split
+        m = std::max(m, n);
+    }
+    if (!(heaviest(split) * 100 < heaviest(even) * 95)) return false;
+    *first = split;
+    *ctiles_max = m;
+    return true;
 }
 
 // Kernel-native copies of codes and LUT and the fused kernel's status word.
@@ -521,11 +593,26 @@ sqz_status build_native(sqz_layer* L, cudaStream_t s) {
             sqz::tc::repack_lut_kernel<4><<<blocks, 256, 0, s>>>(L->lut, L->n_out, rows, L->lut_native);
         SQZ_CUDA_TRY(cudaGetLastError(), "repack lut");
     }
+    // Tiles of every CTA: the even split, or -- when the outliers are skewed
+    // enough -- a split by weight (see split_tiles_by_weight)
+    L->ctiles_max = (L->ntiles + L->grid - 1) / L->grid;
+    if (L->nnz > 0 && L->grid > 1) {
+        std::vector<int32_t> rp((size_t)L->n_out + 1), first;
+        SQZ_CUDA_TRY(cudaMemcpyAsync(rp.data(), L->rowptr, rp.size() * 4, cudaMemcpyDeviceToHost, s), "rowptr read");
+        SQZ_CUDA_TRY(cudaStreamSynchronize(s), "rowptr read");
+        if (split_tiles_by_weight(rp, L->n_out, L->ntiles, L->nsg, L->grid, &first, &L->ctiles_max)) {
+            if ((st = alloc(&L->cta_tiles, (size_t)L->grid + 1, L, "CTA tiles")) != SQZ_OK) return st;
+            SQZ_CUDA_TRY(cudaMemcpyAsync(L->cta_tiles, first.data(), first.size() * 4, cudaMemcpyHostToDevice, s),
+                         "CTA tiles copy");
+            SQZ_CUDA_TRY(cudaStreamSynchronize(s), "CTA tiles copy");  // `first` is a host temporary
+        }
+    }
     // CSR entry range of every CTA's rows (device array read by each launch)
     if ((st = alloc(&L->csr_cta, (size_t)L->grid + 1, L, "CTA bounds")) != SQZ_OK) return st;
     if (L->nnz > 0) {
         if (L->grid > kMaxCtas) return fail(SQZ_ERR_UNSUPPORTED, "%d CTAs exceed the fused kernel's %d", L->grid, kMaxCtas);
-        csr_cta_bounds_kernel<<<(L->grid + 256) / 256, 256, 0, s>>>(L->rowptr, L->n_out, L->ntiles, L->grid, L->csr_cta);
+        csr_cta_bounds_kernel<<<(L->grid + 256) / 256, 256, 0, s>>>(L->rowptr, L->cta_tiles, L->n_out, L->ntiles,
+                                                                    L->grid, L->csr_cta);
         SQZ_CUDA_TRY(cudaGetLastError(), "CTA bounds");
     } else {
         SQZ_CUDA_TRY(cudaMemsetAsync(L->csr_cta, 0, sizeof(int32_t) * ((size_t)L->grid + 1), s), "memset");

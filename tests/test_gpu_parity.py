@@ -357,13 +357,15 @@ def test_padded_columns_with_nonfinite_lut_entries(B, orc, bits, k_in, mac):
     (300, 6144, 4, 16, 0),
     (64, 16384, 3, 8, 0),    # 8 columns that need several passes
     (40, 20000, 4, 16, 0),   # 16 columns, several passes even in launches of 8
+    (300, 18432, 3, 5, 0),   # as many passes as launches of 2 would be: x in K chunks
+    (300, 18432, 3, 5, 3),
 ])
 def test_batches_whose_x_is_staged_in_chunks(B, orc, n_out, k_in, bits, batch, ldx_pad):
-    """Batches whose activations do not fit in shared memory at once: x is
-    staged chunk by chunk over several passes and per-tile sums are kept
-    between them, or (above 8 columns, when 8 fit in one pass) the batch
-    runs as launches of 8 columns.  Same tolerance, and bit-identical from
-    run to run."""
+    """Batches whose activations do not fit in shared memory at once: the
+    batch runs as single-pass launches of fewer columns when those are fewer
+    than the passes the whole batch would need, else x is staged chunk by
+    chunk over several passes with per-tile sums kept between them.  Same
+    tolerance, and bit-identical from run to run."""
     L = make_small(90 + k_in, n_out, k_in, bits, n_out * 12)
     x = synth.make_x(batch, k_in, seed=batch)
     layer = upload(B, L)

@@ -86,9 +86,14 @@ def test_large_batches_split_into_single_pass_launches_of_eight():
     for n, k in ((5120, 5120), (13824, 5120), (4096, 4096)):
         p = B.sqz_plan_query(n, k, 3, 16, **DEV)
         assert (p["launches"], p["columns_per_launch"], p["passes"]) == (2, 8, 1), (n, k, p)
-    # 8 columns of K = 13824 do not fit one pass: one launch of 16 in several passes
-    p = B.sqz_plan_query(5120, 13824, 3, 16, **DEV)
-    assert p["launches"] == 1 and p["passes"] > 1
+    # 8 columns of K = 13824 do not fit one pass: launches of 4 in one pass each
+    # (fewer launches than the passes the whole batch would need)
+    for batch, launches in ((16, 4), (8, 2)):
+        p = B.sqz_plan_query(5120, 13824, 3, batch, **DEV)
+        assert (p["launches"], p["columns_per_launch"], p["passes"]) == (launches, 4, 1), (batch, p)
+    # as many launches as passes: x staged in K chunks in one launch
+    p = B.sqz_plan_query(300, 18432, 3, 5, **DEV)
+    assert p["launches"] == 1 and p["passes"] == 3
 
 
 def test_plan_query_rejects_bad_arguments():
