@@ -62,6 +62,8 @@ def parse():
     p.add_argument("--predecode", type=int, choices=(0, 1, 8, 16), default=0,
                    help="batches of 1..8: the kernel that decodes ahead of x into tensor memory (1; 8 or 16 dense "
                         "warps per CTA) instead of the default 12-warp kernel (0)")
+    p.add_argument("--mac", choices=("tensor", "cuda", "mixed"), default="tensor",
+                   help="batch-1 multiply-accumulate unit of the 12-warp kernel (sqz_layer_set_mac)")
     p.add_argument("--csr", choices=("balanced", "rowwise"), default="balanced",
                    help="sparse scheme of the fused kernel (rowwise: the plain CSR comparison)")
     p.add_argument("--encode", action="store_true",
@@ -225,7 +227,7 @@ def config_for(args, shape, instances, inst_bytes):
         "workload": f"{args.workload}: " + WORKLOAD_DESC.get(
             args.workload, f"{shape.n_out}x{shape.k_in}, {shape.bits}-bit, {shape.density:.2%} CSR, batch {shape.batch}"),
         "n_out": shape.n_out, "k_in": shape.k_in, "bits": shape.bits, "density": shape.density,
-        "batch": shape.batch, "outliers": shape.dist, "csr_scheme": args.csr,
+        "batch": shape.batch, "outliers": shape.dist, "csr_scheme": args.csr, "mac": getattr(args, "mac", "tensor"),
         "kernel": "decode-ahead (TMEM)" if getattr(args, "predecode", 0) and shape.batch <= 8 else "12-warp fused",
         "step": f"one token through a stack of {instances} distinct layers of this shape ({instances} calls)",
         "l2": f"inputs larger than L2: the stack holds {instances * inst_bytes / 1e6:.0f} MB",
@@ -378,6 +380,8 @@ def run_ours(args):
             B.sqz_layer_set_csr_mode(layers[-1], B.SQZ_CSR_ROWWISE)
         if args.predecode:
             B.sqz_layer_set_predecode(layers[-1], args.predecode)
+        if args.mac != "tensor":
+            B.sqz_layer_set_mac(layers[-1], {"cuda": B.SQZ_MAC_CUDA_CORES, "mixed": B.SQZ_MAC_MIXED}[args.mac])
         xs.append(torch.from_numpy(synth.x_for(shape, seed=args.seed, instance=instance_id(rank, i)).view(np.int16))
                   .to(dev))
         ys.append(torch.empty((shape.batch, shape.n_out), dtype=torch.int16, device=dev))
