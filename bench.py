@@ -57,6 +57,8 @@ def parse():
     p.add_argument("--shape-index", type=int, default=0)
     p.add_argument("--impl", choices=("ours", "reference"), default="ours")
     p.add_argument("--sweep", action="store_true", help="one JSON line per workload shape")
+    p.add_argument("--stack", type=int, default=0,
+                   help="layers per step (default: at least 32 and at least 4x L2; never below 4x L2)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--seed", type=int, default=0)
     p.add_argument("--predecode", type=int, choices=(0, 1, 8, 16), default=0,
@@ -147,7 +149,7 @@ def recorded_traffic(workload: str, shape_key: str, batch: int = 1):
                 continue
             kv = dict(tok.split("=", 1) for tok in line.split())
             if (kv.get("shape") == shape_key and kv.get("batch", "1") == str(batch)
-                    and kv.get("source_hash") == want):
+                    and kv.get("source_hash") == want and "bytes_per_launch" in kv):
                 return int(kv["bytes_per_launch"])
     return None
 
@@ -342,9 +344,10 @@ MIN_STACK = 32          # layers per step: at least LLaMA-7B's decoder depth
 CALLS_PER_GRAPH = 512   # about this many kernel nodes per captured graph
 
 
-def stack_depth(l2_bytes: int, layer_bytes: int) -> int:
-    """Layers per step: at least MIN_STACK and at least 4x L2 in total."""
-    return max(MIN_STACK, math.ceil(4 * l2_bytes / layer_bytes))
+def stack_depth(l2_bytes: int, layer_bytes: int, requested: int = 0) -> int:
+    """Layers per step: at least 4x L2 in total, and MIN_STACK unless another
+    depth is requested."""
+    return max(requested if requested > 0 else MIN_STACK, math.ceil(4 * l2_bytes / layer_bytes))
 
 
 def graph_plan(steps: int, per_graph: int):
@@ -370,7 +373,7 @@ def run_ours(args):
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     L0 = synth.layer_for(shape, seed=args.seed, instance=instance_id(rank, 0))
     inst_bytes = L0.nbytes()
-    R = stack_depth(l2, inst_bytes)
+    R = stack_depth(l2, inst_bytes, args.stack)
     layers, xs, ys = [], [], []
     for i in range(R):
         L = L0 if i == 0 else synth.layer_for(shape, seed=args.seed, instance=instance_id(rank, i))
@@ -441,7 +444,7 @@ def run_ours(args):
     value = whole_job_gbs(world, bytes_per_step, args.steps, ms)
     per_launch_gbs = bytes_per_call / (us_per_call * 1e-6) / 1e9
 
-    e2e = e2e_measure(B, torch, dist, shape, layers, R, args, world, rank, dev, stream, bytes_per_step,
+    e2e = e2e_measure(B, torch, dist, shape, layers, xs, R, args, world, rank, dev, stream, bytes_per_step,
                       us_per_call)
 
     # ---- fp16 dense yardstick (same shape, uncompressed weights)
@@ -481,7 +484,7 @@ def run_ours(args):
     return 0
 
 
-def e2e_measure(B, torch, dist, shape, layers, R, args, world, rank, dev, stream, bytes_per_step, us_kernel):
+def e2e_measure(B, torch, dist, shape, layers, xs_dev, R, args, world, rank, dev, stream, bytes_per_step, us_kernel):
     """End to end through the host entry point: every call copies its
     layer's x in from pinned host memory, runs the product, copies y back
     and synchronises.  One step = R calls (the same stack as the device
@@ -511,29 +514,29 @@ def e2e_measure(B, torch, dist, shape, layers, R, args, world, rank, dev, stream
     calls = steps * R
     us_call = ms * 1e3 / calls
 
-    # ---- where a call's time goes: the device time of a call's copies and
-    # kernel (the same copy-in, product, copy-out captured back to back for
-    # the whole stack, replayed, CUDA events), the ctypes round trip of a
-    # call that does nothing, and the rest (graph launch, synchronisation,
-    # Python)
-    xd = [torch.empty((shape.batch, shape.k_in), dtype=torch.int16, device=dev) for _ in range(R)]
+    # ---- where a call's time goes, each part timed alone with CUDA events on
+    # an idle stream: the kernel of one call (no neighbour to overlap with),
+    # the copy of x in and of y out (pinned host memory), the ctypes round
+    # trip of a call that does nothing; the rest is the graph launch, the
+    # synchronisation and Python
+    xd = torch.empty((shape.batch, shape.k_in), dtype=torch.int16, device=dev)
     yd = torch.empty((shape.batch, shape.n_out), dtype=torch.int16, device=dev)
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g, stream=stream):
-        for i in range(R):
-            xd[i].copy_(xh[i], non_blocking=True)
-            B.sqz_gemv(layers[i], xd[i], yd, stream=stream)
-            yh.copy_(yd, non_blocking=True)
-    with torch.cuda.stream(stream):
-        g.replay()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(5):
-            g.replay()
-        b.record(stream)
-    torch.cuda.synchronize(dev)
-    dev_us = a.elapsed_time(b) * 1e3 / (5 * R)
-    del g
+
+    def timed(fn, n=50):
+        out = []
+        with torch.cuda.stream(stream):
+            for i in range(n):
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                fn(i)
+                b.record(stream)
+                b.synchronize()
+                out.append(a.elapsed_time(b) * 1e3)
+        return statistics.median(out)
+
+    kern_us = timed(lambda i: B.sqz_gemv(layers[i % R], xs_dev[i % R], yd, stream=stream))
+    h2d_us = timed(lambda i: xd.copy_(xh[i % R], non_blocking=True))
+    d2h_us = timed(lambda i: yh.copy_(yd, non_blocking=True))
     lib = B.lib()
     n = 20000
     t0 = time.perf_counter()
@@ -545,9 +548,9 @@ def e2e_measure(B, torch, dist, shape, layers, R, args, world, rank, dev, stream
             "d2h_bytes_per_step": R * 2 * shape.batch * shape.n_out,
             "us_per_call": us_call, "wall_us_per_call": wall * 1e6 / calls, "steps": steps, "calls_per_step": R,
             "api": "sqz_gemv_host (pinned host x/y)",
-            "breakdown_us": {"device_copies_and_kernel_back_to_back": dev_us, "kernel_alone": us_kernel,
-                             "ctypes_round_trip": ctypes_us,
-                             "launch_sync_python_rest": us_call - dev_us - ctypes_us}}
+            "breakdown_us": {"kernel_one_call_alone": kern_us, "kernel_in_a_chain_of_calls": us_kernel,
+                             "h2d_copy": h2d_us, "d2h_copy": d2h_us, "ctypes_round_trip": ctypes_us,
+                             "graph_launch_sync_python_rest": us_call - kern_us - h2d_us - d2h_us - ctypes_us}}
 
 
 def fp16_yardstick(B, torch, shape, dev, stream, l2):
@@ -587,7 +590,7 @@ def run_sweep(args):
     for name, shapes in synth.workloads().items():
         for i in range(len(shapes)):
             cmd = [sys.executable, __file__, "--workload", name, "--shape-index", str(i), "--steps",
-                   str(args.steps), "--warmup", str(args.warmup), "--no-cpu-baseline"]
+                   str(args.steps), "--warmup", str(args.warmup), "--no-cpu-baseline", "--stack", str(args.stack or 1)]
             subprocess.run(cmd, check=True)
     return 0
 
