@@ -23,32 +23,39 @@
 //   * Rows in tiles of 16 (the M of an m16n8k16 MMA), columns in
 //     super-groups of 256 (16 k16-steps); a unit = (tile, super-group).  The
 //     code layout and decoder are those of kernels_tc.cuh.
-//   * One CTA per SM (the whole register file): 16 dense warps and one
-//     control warp.  A CTA owns a contiguous run of whole tiles; its dense
-//     warps split the CTA's units into 16 contiguous, equal ranges.
+//   * A CTA owns a contiguous run of whole tiles (the even split, or the
+//     split by weight of the layer's tile array for skewed outliers).  It has
+//     NW dense warps (8: two CTAs per SM; 16: one CTA per SM, see Shape) and
+//     one control warp.  Its units are split into 16 contiguous, equal ranges
+//     ("virtual warps"); with NW = 8 a warp runs two adjacent ranges.
 //   * The control warp requests the LUT planes, the rowptr slice and the
-//     CSR entries of the CTA (bulk copies), allocates TMEM, waits for the
-//     previous kernel and copies x in.
+//     CSR entries of the CTA (bulk copies), asks L2 for the CTA's codes,
+//     allocates TMEM, waits for the previous kernel and copies x in.
+//   * Decoding ahead starts only once the SM's earlier CTAs of this kernel
+//     have finished their dense loops (or x has arrived): see g_pd_looped.
 //   * Sparse part (the balanced scheme): the CTA's nonzeros are split evenly
-//     over the 512 dense threads.  Before x arrives a thread finds the row of
-//     its first entry and loads its first entries; once x is there it sums
-//     its share per row (head piece, rows it holds whole, tail piece), then
-//     starts its dense work.
-//   * Every warp stores its part of each tile it touches in shared memory
-//     (one slot for a tile it holds whole, per-warp slots for the first and
-//     last tiles it shares); after one CTA barrier the threads add the
-//     parts in warp order and each row's sparse sum (the interior sum plus
-//     the pieces of the threads whose shares cut the row, in thread order)
-//     and write y once.  Every summation order is fixed: results are bitwise
-//     reproducible, and a column of a batch equals the batch-1 call on it.
+//     into 512 shares (two per thread with NW = 8).  Before x arrives a
+//     thread finds the row of its first entry and loads its first entries;
+//     once x is there it sums its share per row (head piece, rows it holds
+//     whole, tail piece).  Warps in the first half run their shares before
+//     their decode loop, the others after it.
+//   * Every virtual warp stores its part of each tile it touches in shared
+//     memory (one slot for a tile it holds whole, its own slots for the
+//     first and last tiles it shares); after one CTA barrier the threads add
+//     the parts in virtual-warp order and each row's sparse sum (the
+//     interior sum plus the pieces of the shares that cut the row, in share
+//     order) and write y once.  Every summation order is fixed and does not
+//     depend on NW: results are bitwise reproducible, both shapes give the
+//     same bits, and a column of a batch equals the batch-1 call on it.
 //
-// TMEM: warp w reaches the 32 lanes of quarter w % 4 (lane = the warp's
-// lane); its columns are [(w / 4) * 128, +128): two units of 64 columns (a
-// quad of 4 k16-steps = 16 columns of A fragments).  The control warp
-// allocates all 512 columns at the start and frees them after the last
-// tcgen05.ld, on every path.  A CTA takes the whole register file and more
-// than half of the shared memory, so no second CTA of this kernel can be
-// resident on the SM and wait for its TMEM.
+// TMEM: dense warp w reaches the 32 lanes of quarter w % 4 (lane = the
+// warp's lane); its columns are [(w / 4) * 128, +128) of its CTA's
+// allocation: two units of 64 columns (a quad of 4 k16-steps = 16 columns of
+// A fragments).  The control warp allocates the CTA's columns (256 with
+// NW = 8, 512 with NW = 16) at the start and frees them after the last
+// tcgen05.ld, on every path; the resident CTAs of an SM never ask for more
+// than its 512 columns together, so no allocation waits on a CTA that waits
+// for it.
 //
 // Every wait on a copy or mbarrier is bounded and records a status bit
 // instead of hanging.
