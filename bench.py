@@ -514,33 +514,24 @@ def e2e_measure(B, torch, dist, shape, layers, xs_dev, R, args, world, rank, dev
     calls = steps * R
     us_call = ms * 1e3 / calls
 
-    # ---- where a call's time goes.  Device side: the same work (copy of x
-    # in from pinned memory, the product, copy of y out) for the R layers of
-    # a step, captured as one graph and replayed back to back, timed with
-    # CUDA events; per call that is what the GPU does.  Host side: the rest
-    # of a synchronous call (graph launch, synchronisation, Python).  For
-    # reference, each device part on its own on an idle stream (these carry
-    # the start-from-idle cost, so they do not add up to the device time).
-    xd = [torch.empty((shape.batch, shape.k_in), dtype=torch.int16, device=dev) for _ in range(R)]
+    # ---- where a call's time goes: the same call without moving x and y
+    # (sqz_gemv on device buffers, then a stream synchronise; wall clock, the
+    # same layer rotation) is the cost of a lone synchronous product; the
+    # rest of the e2e call is bringing x in and taking y out.  The kernel in a
+    # chain of calls and the parts alone on an idle stream (CUDA events; they
+    # carry the start-from-idle cost) are listed for reference.
     yd = torch.empty((shape.batch, shape.n_out), dtype=torch.int16, device=dev)
-    g = torch.cuda.CUDAGraph()
+    xd0 = torch.empty((shape.batch, shape.k_in), dtype=torch.int16, device=dev)
     with torch.cuda.stream(stream):
-        with torch.cuda.graph(g, stream=stream):
-            for i in range(R):
-                xd[i].copy_(xh[i], non_blocking=True)
-                B.sqz_gemv(layers[i], xd[i], yd, stream=stream)
-                yh.copy_(yd, non_blocking=True)
-        for _ in range(3):
-            g.replay()
-        reps = max(2, min(steps, 50))
-        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a0.record(stream)
-        for _ in range(reps):
-            g.replay()
-        a1.record(stream)
-    torch.cuda.synchronize(dev)
-    dev_us = a0.elapsed_time(a1) * 1e3 / (reps * R)
-    del g
+        for i in range(R):
+            B.sqz_gemv(layers[i], xs_dev[i], yd, stream=stream)
+            stream.synchronize()
+        n_sync = max(R, min(calls, 2000))
+        t0 = time.perf_counter()
+        for j in range(n_sync):
+            B.sqz_gemv(layers[j % R], xs_dev[j % R], yd, stream=stream)
+            stream.synchronize()
+        sync_us = (time.perf_counter() - t0) / n_sync * 1e6
 
     def timed(fn, n=50):
         out = []
@@ -555,7 +546,7 @@ def e2e_measure(B, torch, dist, shape, layers, xs_dev, R, args, world, rank, dev
         return statistics.median(out)
 
     kern_us = timed(lambda i: B.sqz_gemv(layers[i % R], xs_dev[i % R], yd, stream=stream))
-    h2d_us = timed(lambda i: xd[0].copy_(xh[i % R], non_blocking=True))
+    h2d_us = timed(lambda i: xd0.copy_(xh[i % R], non_blocking=True))
     d2h_us = timed(lambda i: yh.copy_(yd, non_blocking=True))
     lib = B.lib()
     n = 20000
@@ -568,11 +559,12 @@ def e2e_measure(B, torch, dist, shape, layers, xs_dev, R, args, world, rank, dev
             "d2h_bytes_per_step": R * 2 * shape.batch * shape.n_out,
             "us_per_call": us_call, "wall_us_per_call": wall * 1e6 / calls, "steps": steps, "calls_per_step": R,
             "api": "sqz_gemv_host (pinned host x/y)",
-            "breakdown_us": {"device_copy_in_kernel_copy_out_per_call": dev_us,
-                             "host_launch_sync_python_per_call": us_call - dev_us,
-                             "of_which_ctypes_round_trip": ctypes_us,
+            "breakdown_us": {"synchronous_product_without_io": sync_us,
+                             "moving_x_in_and_y_out": us_call - sync_us,
+                             "ctypes_round_trip": ctypes_us,
                              "kernel_in_a_chain_of_calls": us_kernel,
-                             "alone_from_idle": {"kernel": kern_us, "h2d_copy": h2d_us, "d2h_copy": d2h_us}}}
+                             "alone_from_idle_events": {"kernel": kern_us, "h2d_copy_engine": h2d_us,
+                                                        "d2h_copy_engine": d2h_us}}}
 
 
 def fp16_yardstick(B, torch, shape, dev, stream, l2):

@@ -127,16 +127,23 @@ SQZ_API sqz_status sqz_gemv(sqz_layer_t layer, const uint16_t* x, int32_t batch,
 
 /*
  * The same product for callers whose activations live in HOST memory:
- * copies x (host, [batch][ldx]) to the handle's device staging buffer,
- * runs sqz_gemv, copies y back to host memory ([batch][ldy]) and
- * synchronises `stream` before returning.  Pinned host buffers give
- * asynchronous copies; pageable ones work but copy synchronously.  With
- * pinned buffers on a created (non-default) stream, the copy-in, product
- * and copy-out are captured as a CUDA graph on first use and replayed by
- * later calls with the same buffers, shape and stream (up to 64 per handle,
- * least recently used dropped; released by sqz_destroy and by a change of
- * the handle's MAC unit or CSR mode).  Not thread-safe against other calls
- * on the same handle.  Errors as sqz_gemv.
+ * x (host, [batch][ldx]) in, y (host, [batch][ldy]) out; synchronises
+ * `stream` before returning.
+ *   - Page-locked buffers (cudaHostAlloc / cudaMallocHost / cudaHostRegister,
+ *     including torch's pin_memory): the kernels read x and write y through
+ *     the buffers' device mapping -- a small copy kernel brings x into the
+ *     handle's device staging buffer (the product kernel is its programmatic
+ *     dependent, so it starts loading weights meanwhile) and the product
+ *     kernel stores y straight into the host buffer.  No copy-engine
+ *     transfer.  On a created (non-default) stream the two launches are
+ *     captured as a CUDA graph on first use and replayed by later calls with
+ *     the same buffers, shape and stream (up to 64 per handle, least
+ *     recently used dropped; released by sqz_destroy and by a change of the
+ *     handle's MAC unit, CSR mode or decode-ahead setting).
+ *   - Pageable buffers: copied through the staging buffers with
+ *     cudaMemcpyAsync (synchronous for pageable memory).
+ * Elements of y beyond column N of each row are not written.  Not
+ * thread-safe against other calls on the same handle.  Errors as sqz_gemv.
  */
 SQZ_API sqz_status sqz_gemv_host(sqz_layer_t layer, const uint16_t* x_host, int32_t batch, int64_t ldx,
                          uint16_t* y_host, int64_t ldy, void* stream);

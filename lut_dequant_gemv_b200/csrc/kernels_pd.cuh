@@ -748,13 +748,20 @@ __global__ void __launch_bounds__(Shape<NW>::kThreads, Shape<NW>::kCtasPerSm)
     // ---- once every warp has left its loop: each output is the tile's sum
     // (or the virtual warps' parts of a shared tile, in order) plus the row's
     // sparse sum (interior sum, then the pieces of the shares that cut the
-    // row, in share order); the control warp frees TMEM (every tcgen05.ld
-    // has completed)
+    // row: in share order, or by a warp for a long row); the control warp
+    // frees TMEM (every tcgen05.ld has completed)
     tmem_fence_before();
     __syncthreads();
     tmem_fence_after();
     if (ctrl) tmem_dealloc(taddr, kTmemCols);
     if (tid == 0) atomicAdd(&g_pd_looped[smslot], 1u);  // this CTA's dense loops are done
+    // rows cut into more than kLongPieces shares: their pieces are added into
+    // the interior sum by a warp first (the loop below skips them)
+    if (has_csr) {
+        tc::add_long_rows<CM>(nrows, warp, kThreads / 32, lane, s_rp, q0, e_per, kVThreads, s_rowsum, s_headrow,
+                              s_head, s_tailrow, s_tail);
+        __syncthreads();
+    }
     for (int idx = tid; idx < ctiles * TE; idx += kThreads) {
         const int tl = idx / TE, e = idx - tl * TE;
         const int row_l = e / CM, col = e - row_l * CM;
@@ -777,7 +784,7 @@ __global__ void __launch_bounds__(Shape<NW>::kThreads, Shape<NW>::kCtasPerSm)
             if (re > rs) {
                 float cs = s_rowsum[i * CM + col];
                 const int tau_a = (rs - q0) / e_per, tau_b = min(kVThreads - 1, (re - 1 - q0) / e_per);
-                for (int tau = tau_a; tau <= tau_b; ++tau) {
+                for (int tau = tau_a; tau <= tau_b && tau_b - tau_a < tc::kLongPieces; ++tau) {
                     if (s_headrow[tau] == i) cs += s_head[tau * CM + col];
                     if (s_tailrow[tau] == i) cs += s_tail[tau * CM + col];
                 }

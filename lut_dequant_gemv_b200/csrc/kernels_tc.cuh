@@ -95,6 +95,10 @@ constexpr int kSbStages = 4;      // one pass over K: the ring depth, 4 stages (
 constexpr int kPreWait = 2;       // code units per warp requested before waiting for the previous kernel;
                                   // the rest of the first ring follows once x has landed
 constexpr int kCsrCap = 4096;     // CSR entries per CTA staged in shared memory, at most (more: read from global)
+// A row whose nonzeros are cut into more than kLongPieces shares (a long
+// row of skewed outliers spans up to every share of its CTA) has its pieces
+// added by a whole warp instead of one thread walking them in order.
+constexpr int kLongPieces = 16;
 constexpr uint32_t kSuspendNs = 1000000u;  // 1 ms per poll
 constexpr uint32_t kWaitLimit = 2000u;
 
@@ -441,6 +445,66 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
         "{%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// The sparse pieces of row i held by shares [tau_a, tau_b] (a head piece
+// where the share's first row is i, a tail piece where its last row is),
+// added by the 32 lanes of a warp: lane l sums shares tau_a + l, + 32, ...
+// in order, then a fixed shuffle tree brings the lanes' sums to lane 0,
+// which adds them to the row's interior sum.  The order depends only on the
+// split of the nonzeros into shares, never on the batch size.
+template <int CM>
+__device__ __forceinline__ void add_long_row_pieces(int i, int tau_a, int tau_b, int lane, float* s_rowsum,
+                                                    const int* s_headrow, const float* s_head,
+                                                    const int* s_tailrow, const float* s_tail) {
+    float part[CM];
+#pragma unroll
+    for (int b = 0; b < CM; ++b) part[b] = 0.f;
+    for (int tau = tau_a + lane; tau <= tau_b; tau += 32) {
+        if (s_headrow[tau] == i) {
+#pragma unroll
+            for (int b = 0; b < CM; ++b) part[b] += s_head[tau * CM + b];
+        }
+        if (s_tailrow[tau] == i) {
+#pragma unroll
+            for (int b = 0; b < CM; ++b) part[b] += s_tail[tau * CM + b];
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+        for (int b = 0; b < CM; ++b) part[b] += __shfl_down_sync(0xffffffffu, part[b], off);
+    if (lane == 0) {
+#pragma unroll
+        for (int b = 0; b < CM; ++b) s_rowsum[i * CM + b] += part[b];
+    }
+}
+
+// Long rows of rows [0, nrows): warp w of the nw warps that call this scans
+// rows w*32 + lane, + nw*32, ... and adds the pieces of each long row with
+// the whole warp.  Warp-uniform: every lane of the calling warps enters.
+template <int CM>
+__device__ __forceinline__ void add_long_rows(int nrows, int warp, int nw, int lane, const int* s_rp, int q0,
+                                              int e_per, int nshares, float* s_rowsum, const int* s_headrow,
+                                              const float* s_head, const int* s_tailrow, const float* s_tail) {
+    for (int i0 = warp * 32; i0 < nrows; i0 += nw * 32) {
+        const int i = i0 + lane;
+        int ta = 0, tb = -1;
+        if (i < nrows) {
+            const int rs = s_rp[i], re = s_rp[i + 1];
+            if (re > rs) {
+                ta = (rs - q0) / e_per;
+                tb = min(nshares - 1, (re - 1 - q0) / e_per);
+            }
+        }
+        unsigned int m = __ballot_sync(0xffffffffu, tb - ta >= kLongPieces);
+        while (m) {
+            const int l = __ffs(m) - 1;
+            m &= m - 1;
+            const int a = __shfl_sync(0xffffffffu, ta, l), b = __shfl_sync(0xffffffffu, tb, l);
+            add_long_row_pieces<CM>(i0 + l, a, b, lane, s_rowsum, s_headrow, s_head, s_tailrow, s_tail);
+        }
+    }
 }
 
 // acc += w.lo * x.lo + w.hi * x.hi with fp16 operands and an fp32
@@ -906,29 +970,46 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_fused_kernel(const 
     }
     // Balanced mode: once every share is written (a barrier of the CT sparse
     // threads), each row's interior sum and the pieces of the threads whose
-    // shares cut it are added, in thread order, into s_rowsum -- so a row's
-    // sparse sum is one shared-memory read wherever y is written.
+    // shares cut it are added into s_rowsum -- in thread order by one thread,
+    // or by a warp for a row cut into more than kLongPieces shares -- so a
+    // row's sparse sum is one shared-memory read wherever y is written.
     if (!RW && has_csr && tid < CT) {
         asm volatile("bar.sync 1, %0;" ::"n"(CT) : "memory");
-        for (int i = tid; i < nrows; i += CT) {
-            const int rs = s_rp[i], re = s_rp[i + 1];
-            if (re <= rs) continue;
-            float cs[CM];
-#pragma unroll
-            for (int b = 0; b < CM; ++b) cs[b] = s_rowsum[i * CM + b];
-            const int tau_a = (rs - q0) / e_per, tau_b = min(CT - 1, (re - 1 - q0) / e_per);
-            for (int tau = tau_a; tau <= tau_b; ++tau) {
-                if (s_headrow[tau] == i) {
-#pragma unroll
-                    for (int b = 0; b < CM; ++b) cs[b] += s_head[tau * CM + b];
-                }
-                if (s_tailrow[tau] == i) {
-#pragma unroll
-                    for (int b = 0; b < CM; ++b) cs[b] += s_tail[tau * CM + b];
+        // thread tid takes rows tid, tid + CT, ...; the loop runs warp by warp
+        // so that the long rows of a 32-row group can be handed to the warp
+        for (int i0 = warp * 32; i0 < nrows; i0 += CT) {
+            const int i = i0 + lane;
+            int tau_a = 0, tau_b = -1;
+            if (i < nrows) {
+                const int rs = s_rp[i], re = s_rp[i + 1];
+                if (re > rs) {
+                    tau_a = (rs - q0) / e_per;
+                    tau_b = min(CT - 1, (re - 1 - q0) / e_per);
                 }
             }
+            const bool long_row = tau_b - tau_a >= kLongPieces;
+            if (tau_b >= tau_a && !long_row) {
+                float cs[CM];
 #pragma unroll
-            for (int b = 0; b < CM; ++b) s_rowsum[i * CM + b] = cs[b];
+                for (int b = 0; b < CM; ++b) cs[b] = s_rowsum[i * CM + b];
+                for (int tau = tau_a; tau <= tau_b; ++tau) {
+                    if (s_headrow[tau] == i) {
+#pragma unroll
+                        for (int b = 0; b < CM; ++b) cs[b] += s_head[tau * CM + b];
+                    }
+                    if (s_tailrow[tau] == i) {
+#pragma unroll
+                        for (int b = 0; b < CM; ++b) cs[b] += s_tail[tau * CM + b];
+                    }
+                }
+#pragma unroll
+                for (int b = 0; b < CM; ++b) s_rowsum[i * CM + b] = cs[b];
+            }
+            for (unsigned int m = __ballot_sync(0xffffffffu, long_row); m; m &= m - 1) {
+                const int l = __ffs(m) - 1;
+                const int a = __shfl_sync(0xffffffffu, tau_a, l), b = __shfl_sync(0xffffffffu, tau_b, l);
+                add_long_row_pieces<CM>(i0 + l, a, b, lane, s_rowsum, s_headrow, s_head, s_tailrow, s_tail);
+            }
         }
     }
     if (has_csr && tid < CT) mbar_arrive(rbar);

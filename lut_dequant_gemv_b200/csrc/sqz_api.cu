@@ -755,12 +755,39 @@ sqz_status sqz_gemv(sqz_layer_t layer, const uint16_t* x, int32_t batch, int64_t
 
 namespace {
 
-// Copy x in, run the product, copy y out, all on stream s.
+// Device addresses of page-locked host buffers (nullptr: pageable memory,
+// which only the copy engines can move).
+struct HostMaps {
+    const uint16_t* x = nullptr;
+    uint16_t* y = nullptr;
+};
+HostMaps host_maps(const uint16_t* x_host, uint16_t* y_host) {
+    HostMaps m;
+    cudaPointerAttributes a{};
+    if (cudaPointerGetAttributes(&a, x_host) == cudaSuccess && a.type == cudaMemoryTypeHost && a.devicePointer)
+        m.x = static_cast<const uint16_t*>(a.devicePointer);
+    a = cudaPointerAttributes{};
+    if (cudaPointerGetAttributes(&a, y_host) == cudaSuccess && a.type == cudaMemoryTypeHost && a.devicePointer)
+        m.y = static_cast<uint16_t*>(a.devicePointer);
+    (void)cudaGetLastError();
+    return m;
+}
+
+// Bring x in, run the product, take y out, all on stream s.  Page-locked
+// buffers are read and written by the kernels through their device mapping:
+// x by fetch_x_kernel into the staging buffer (the product follows as a
+// programmatic dependent), y by the product's own stores.  Pageable buffers
+// go through the staging buffers with copy-engine transfers.
 sqz_status enqueue_host_call(const sqz_layer* L, const uint16_t* x_host, int32_t batch, int64_t ldx, uint16_t* y_host,
-                             int64_t ldy, cudaStream_t s) {
+                             int64_t ldy, cudaStream_t s, const HostMaps& m) {
     sqz_status st;
-    // one flat copy each way when the rows are packed (a 2-D copy otherwise)
-    if (L->k_in > 0) {
+    if (L->k_in > 0 && m.x) {
+        const bool vec = reinterpret_cast<uintptr_t>(m.x) % 16 == 0 && ldx % 8 == 0 && L->k_in % 8 == 0;
+        const int64_t items = vec ? (int64_t)batch * (L->k_in / 8) : (int64_t)batch * L->k_in;
+        const int64_t ctas = std::min<int64_t>((items + 255) / 256, 4 * (int64_t)L->sm_count);
+        sqz::fetch_x_kernel<<<(unsigned)ctas, 256, 0, s>>>(m.x, ldx, L->k_in, batch, L->x_stage, vec ? 1 : 0);
+        SQZ_CUDA_TRY(cudaGetLastError(), "x fetch launch");
+    } else if (L->k_in > 0) {
         const size_t row = (size_t)L->k_in * 2;
         const cudaError_t e = (ldx == L->k_in || batch == 1)
                                   ? cudaMemcpyAsync(L->x_stage, x_host, row * batch, cudaMemcpyHostToDevice, s)
@@ -768,6 +795,7 @@ sqz_status enqueue_host_call(const sqz_layer* L, const uint16_t* x_host, int32_t
                                                       cudaMemcpyHostToDevice, s);
         SQZ_CUDA_TRY(e, "x host-to-device copy");
     }
+    if (m.y) return gemv_impl(L, L->x_stage, batch, L->k_in, m.y, ldy, s);
     st = gemv_impl(L, L->x_stage, batch, L->k_in, L->y_stage, L->n_out, s);
     if (st != SQZ_OK) return st;
     if (L->n_out > 0) {
@@ -787,15 +815,9 @@ constexpr size_t kHostGraphsPerLayer = 64;
 // call cannot be captured (the legacy default stream, or a stream that is
 // already being captured), in which case the caller enqueues it directly.
 cudaGraphExec_t host_graph(sqz_layer* L, const uint16_t* x_host, int32_t batch, int64_t ldx, uint16_t* y_host,
-                           int64_t ldy, cudaStream_t s) {
+                           int64_t ldy, cudaStream_t s, const HostMaps& m) {
     if (s == nullptr || s == cudaStreamLegacy || s == cudaStreamPerThread) return nullptr;
-    for (const void* p : {static_cast<const void*>(x_host), static_cast<const void*>(y_host)}) {
-        cudaPointerAttributes a{};
-        if (cudaPointerGetAttributes(&a, p) != cudaSuccess || a.type != cudaMemoryTypeHost) {
-            (void)cudaGetLastError();
-            return nullptr;  // pageable memory: copied directly, not captured
-        }
-    }
+    if (!m.x || !m.y) return nullptr;  // pageable memory: copied directly, not captured
     cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
     if (cudaStreamIsCapturing(s, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) return nullptr;
     for (auto& g : L->host_graphs)
@@ -807,7 +829,7 @@ cudaGraphExec_t host_graph(sqz_layer* L, const uint16_t* x_host, int32_t batch, 
         (void)cudaGetLastError();
         return nullptr;
     }
-    const sqz_status st = enqueue_host_call(L, x_host, batch, ldx, y_host, ldy, s);
+    const sqz_status st = enqueue_host_call(L, x_host, batch, ldx, y_host, ldy, s, m);
     cudaGraph_t graph = nullptr;
     const cudaError_t e = cudaStreamEndCapture(s, &graph);
     cudaGraphExec_t exec = nullptr;
@@ -835,9 +857,10 @@ sqz_status sqz_gemv_host(sqz_layer_t layer, const uint16_t* x_host, int32_t batc
     sqz_status st = check_gemv_args(layer, x_host, batch, ldx, y_host, ldy);
     if (st != SQZ_OK) return st;
     cudaStream_t s = as_stream(stream);
-    if (cudaGraphExec_t exec = host_graph(layer, x_host, batch, ldx, y_host, ldy, s)) {
+    const HostMaps m = host_maps(x_host, y_host);
+    if (cudaGraphExec_t exec = host_graph(layer, x_host, batch, ldx, y_host, ldy, s, m)) {
         SQZ_CUDA_TRY(cudaGraphLaunch(exec, s), "graph launch");
-    } else if ((st = enqueue_host_call(layer, x_host, batch, ldx, y_host, ldy, s)) != SQZ_OK) {
+    } else if ((st = enqueue_host_call(layer, x_host, batch, ldx, y_host, ldy, s, m)) != SQZ_OK) {
         return st;
     }
     SQZ_CUDA_TRY(cudaStreamSynchronize(s), "stream synchronize");

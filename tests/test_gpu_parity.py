@@ -190,6 +190,32 @@ def test_deterministic_and_batch_independent(B):
     assert np.array_equal(y16, gpu_gemv(B, layer, x16))
 
 
+def test_long_rows_deterministic_and_batch_independent(B, orc):
+    """Skewed outliers: rows cut into many sparse shares have their pieces
+    added by a warp in a fixed order.  Results match the oracle on sampled
+    rows (the longest rows among them), repeat bit for bit, and each column
+    of a batch equals the batch-1 call on it -- with the default kernel and
+    with the decode-ahead kernel."""
+    shape = synth.workloads()["llama7b-skew"][0]
+    L = synth.layer_for(shape)
+    counts = np.diff(L.rowptr)
+    longest = np.argsort(counts)[-24:]
+    rows = np.unique(np.concatenate([longest, np.arange(0, shape.n_out, 97)])).astype(np.int32)
+    x = synth.make_x(8, shape.k_in, seed=12, key="long-rows")
+    for predecode in (0, 1):
+        layer = upload(B, L)
+        if predecode:
+            B.sqz_layer_set_predecode(layer, 1)
+        y8 = gpu_gemv(B, layer, x)
+        assert np.array_equal(y8, gpu_gemv(B, layer, x))
+        for b in (0, 5):
+            y1 = gpu_gemv(B, layer, x[b:b + 1])
+            assert np.array_equal(y1[0], y8[b]), (predecode, b)
+        y_ref, bound = orc.gemv_layer(L, x, rows=rows)
+        assert_close(y8[:, rows], y_ref, bound, f"predecode={predecode}")
+        layer.close()
+
+
 def test_host_entry_point_matches_device(B):
     shape = synth.workloads()["llama7b-q-4bit"][0]
     L = synth.layer_for(shape)
@@ -225,6 +251,35 @@ def test_host_entry_point_replays_read_new_inputs(B, orc):
     B.sqz_gemv_host(layer, xp, yp, stream=s)
     y_ref, bound = orc.gemv_layer(L, xp.numpy().view(np.uint16))
     assert_close(yp.numpy().view(np.uint16), y_ref, bound, "host pageable")
+
+
+def test_host_entry_point_strided_and_unaligned_pinned_buffers(B, orc):
+    """Page-locked x and y read and written by the kernels through their
+    device mapping: row strides that are not multiples of 8 elements and a
+    start 2 bytes past a 16-byte boundary take the element-wise copy of x;
+    y's padding columns stay untouched; captured and direct (legacy
+    stream) calls agree."""
+    L = make_small(61, 200, 512, 4, 300)
+    layer = upload(B, L)
+    s = torch.cuda.Stream()
+    ldx, ldy = 512 + 3, 200 + 5
+    xbuf = torch.zeros(3 * ldx + 1, dtype=torch.int16).pin_memory()
+    ybuf = torch.full((3 * ldy + 1,), 0x7E00, dtype=torch.int16).pin_memory()
+    xh = xbuf[1:1 + 3 * ldx].view(3, ldx)  # 2 bytes past the allocation's start
+    yh = ybuf[1:1 + 3 * ldy].view(3, ldy)
+    for trial, stream in enumerate((s, s, None)):
+        x = synth.make_x(3, 512, seed=70 + trial)
+        xh[:, :512].copy_(torch.from_numpy(x.view(np.int16)))
+        xh[:, 512:].fill_(0x7C00)  # +inf past K must never be read
+        B.sqz_gemv_host(layer, xh, yh, stream=stream)
+        y_ref, bound = orc.gemv_layer(L, x)
+        assert_close(yh[:, :200].numpy().view(np.uint16), y_ref, bound, f"pinned strided {trial}")
+        assert np.all(yh[:, 200:].numpy() == 0x7E00)
+    aligned_x = torch.from_numpy(synth.make_x(2, 512, seed=80).view(np.int16).copy()).pin_memory()
+    aligned_y = torch.zeros((2, 200), dtype=torch.int16).pin_memory()
+    B.sqz_gemv_host(layer, aligned_x, aligned_y, stream=s)
+    y_ref, bound = orc.gemv_layer(L, aligned_x.numpy().view(np.uint16))
+    assert_close(aligned_y.numpy().view(np.uint16), y_ref, bound, "pinned packed")
 
 
 def test_non_default_stream(B, orc):
