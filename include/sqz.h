@@ -128,22 +128,19 @@ SQZ_API sqz_status sqz_gemv(sqz_layer_t layer, const uint16_t* x, int32_t batch,
 /*
  * The same product for callers whose activations live in HOST memory:
  * x (host, [batch][ldx]) in, y (host, [batch][ldy]) out; synchronises
- * `stream` before returning.
- *   - Page-locked buffers (cudaHostAlloc / cudaMallocHost / cudaHostRegister,
- *     including torch's pin_memory): the kernels read x and write y through
- *     the buffers' device mapping -- a small copy kernel brings x into the
- *     handle's device staging buffer (the product kernel is its programmatic
- *     dependent, so it starts loading weights meanwhile) and the product
- *     kernel stores y straight into the host buffer.  No copy-engine
- *     transfer.  On a created (non-default) stream the two launches are
- *     captured as a CUDA graph on first use and replayed by later calls with
- *     the same buffers, shape and stream (up to 64 per handle, least
- *     recently used dropped; released by sqz_destroy and by a change of the
- *     handle's MAC unit, CSR mode or decode-ahead setting).
- *   - Pageable buffers: copied through the staging buffers with
- *     cudaMemcpyAsync (synchronous for pageable memory).
- * Elements of y beyond column N of each row are not written.  Not
- * thread-safe against other calls on the same handle.  Errors as sqz_gemv.
+ * `stream` before returning.  x is copied to the handle's device staging
+ * buffer with cudaMemcpyAsync (asynchronous when x is page-locked).  A
+ * page-locked y (cudaHostAlloc / cudaMallocHost / cudaHostRegister,
+ * including torch's pin_memory) is written by the product kernel's own
+ * stores through the buffer's device mapping, without a copy back; a
+ * pageable y is written to a staging buffer and copied back.  With both
+ * buffers page-locked on a created (non-default) stream, the copy and the
+ * product are captured as a CUDA graph on first use and replayed by later
+ * calls with the same buffers, shape and stream (up to 64 per handle, least
+ * recently used dropped; released by sqz_destroy and by a change of the
+ * handle's MAC unit, CSR mode or decode-ahead setting).  Elements of y
+ * beyond column N of each row are not written.  Not thread-safe against
+ * other calls on the same handle.  Errors as sqz_gemv.
  */
 SQZ_API sqz_status sqz_gemv_host(sqz_layer_t layer, const uint16_t* x_host, int32_t batch, int64_t ldx,
                          uint16_t* y_host, int64_t ldy, void* stream);

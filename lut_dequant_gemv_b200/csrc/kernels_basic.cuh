@@ -37,37 +37,6 @@ static __global__ void validate_csr_kernel(const int32_t* __restrict__ rowptr, c
     if (bad) atomicOr(flag, bad);
 }
 
-// ------------------------------------------- x from page-locked host memory
-// Copies x (batch rows of k_in halves, row stride ldx) from page-locked host
-// memory, read through its device mapping, into a device buffer with row
-// stride k_in: the host entry point's copy of x without a copy-engine
-// transfer.  vec: the source address, ldx and k_in all allow 16-byte loads;
-// else 2-byte loads.  Loads are cache-volatile (.cv): host memory may have
-// changed since an earlier call read the same lines.  The product kernel
-// launched after it is a programmatic dependent: its weight loads start while
-// this kernel waits on the host link, and it reads x only after this grid
-// has finished.
-static __global__ void __launch_bounds__(256) fetch_x_kernel(const uint16_t* __restrict__ xh, int64_t ldx,
-                                                             int32_t k_in, int32_t batch, uint16_t* __restrict__ xd,
-                                                             int vec) {
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    const int64_t t0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (vec) {
-        const int64_t per = k_in / 8;  // 16-byte pieces per row
-        for (int64_t i = t0; i < (int64_t)batch * per; i += stride) {
-            const int64_t b = i / per, j = i - b * per;
-            const uint4 v = __ldcv(reinterpret_cast<const uint4*>(xh + b * ldx) + j);
-            reinterpret_cast<uint4*>(xd + b * (int64_t)k_in)[j] = v;
-        }
-    } else {
-        for (int64_t i = t0; i < (int64_t)batch * k_in; i += stride) {
-            const int64_t b = i / k_in, k = i - b * k_in;
-            xd[i] = __ldcv(xh + b * ldx + k);
-        }
-    }
-}
-
 // ------------------------------------------------------- canonical decoding
 // Code j (0..31) of a 3-word, 32-code group of a 3-bit row: bits 3j..3j+2 of
 // the 96-bit little-endian integer w0 + w1*2^32 + w2*2^64.

@@ -755,17 +755,15 @@ sqz_status sqz_gemv(sqz_layer_t layer, const uint16_t* x, int32_t batch, int64_t
 
 namespace {
 
-// Device addresses of page-locked host buffers (nullptr: pageable memory,
-// which only the copy engines can move).
+// Device addresses of page-locked host buffers (nullptr: pageable memory).
 struct HostMaps {
-    const uint16_t* x = nullptr;
+    bool x_pinned = false;
     uint16_t* y = nullptr;
 };
 HostMaps host_maps(const uint16_t* x_host, uint16_t* y_host) {
     HostMaps m;
     cudaPointerAttributes a{};
-    if (cudaPointerGetAttributes(&a, x_host) == cudaSuccess && a.type == cudaMemoryTypeHost && a.devicePointer)
-        m.x = static_cast<const uint16_t*>(a.devicePointer);
+    m.x_pinned = cudaPointerGetAttributes(&a, x_host) == cudaSuccess && a.type == cudaMemoryTypeHost;
     a = cudaPointerAttributes{};
     if (cudaPointerGetAttributes(&a, y_host) == cudaSuccess && a.type == cudaMemoryTypeHost && a.devicePointer)
         m.y = static_cast<uint16_t*>(a.devicePointer);
@@ -773,21 +771,15 @@ HostMaps host_maps(const uint16_t* x_host, uint16_t* y_host) {
     return m;
 }
 
-// Bring x in, run the product, take y out, all on stream s.  Page-locked
-// buffers are read and written by the kernels through their device mapping:
-// x by fetch_x_kernel into the staging buffer (the product follows as a
-// programmatic dependent), y by the product's own stores.  Pageable buffers
-// go through the staging buffers with copy-engine transfers.
+// Bring x in, run the product, take y out, all on stream s.  x goes to the
+// handle's staging buffer by a copy-engine transfer.  A page-locked y is
+// written by the product kernel's own stores through its device mapping (a
+// copy-engine transfer after the kernel took 2-4 us longer per call); a
+// pageable y goes through the staging buffer and a copy back.
 sqz_status enqueue_host_call(const sqz_layer* L, const uint16_t* x_host, int32_t batch, int64_t ldx, uint16_t* y_host,
                              int64_t ldy, cudaStream_t s, const HostMaps& m) {
     sqz_status st;
-    if (L->k_in > 0 && m.x) {
-        const bool vec = reinterpret_cast<uintptr_t>(m.x) % 16 == 0 && ldx % 8 == 0 && L->k_in % 8 == 0;
-        const int64_t items = vec ? (int64_t)batch * (L->k_in / 8) : (int64_t)batch * L->k_in;
-        const int64_t ctas = std::min<int64_t>((items + 255) / 256, 4 * (int64_t)L->sm_count);
-        sqz::fetch_x_kernel<<<(unsigned)ctas, 256, 0, s>>>(m.x, ldx, L->k_in, batch, L->x_stage, vec ? 1 : 0);
-        SQZ_CUDA_TRY(cudaGetLastError(), "x fetch launch");
-    } else if (L->k_in > 0) {
+    if (L->k_in > 0) {
         const size_t row = (size_t)L->k_in * 2;
         const cudaError_t e = (ldx == L->k_in || batch == 1)
                                   ? cudaMemcpyAsync(L->x_stage, x_host, row * batch, cudaMemcpyHostToDevice, s)
@@ -817,7 +809,7 @@ constexpr size_t kHostGraphsPerLayer = 64;
 cudaGraphExec_t host_graph(sqz_layer* L, const uint16_t* x_host, int32_t batch, int64_t ldx, uint16_t* y_host,
                            int64_t ldy, cudaStream_t s, const HostMaps& m) {
     if (s == nullptr || s == cudaStreamLegacy || s == cudaStreamPerThread) return nullptr;
-    if (!m.x || !m.y) return nullptr;  // pageable memory: copied directly, not captured
+    if (!m.x_pinned || !m.y) return nullptr;  // pageable memory: copied directly, not captured
     cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
     if (cudaStreamIsCapturing(s, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) return nullptr;
     for (auto& g : L->host_graphs)

@@ -254,10 +254,10 @@ def test_host_entry_point_replays_read_new_inputs(B, orc):
 
 
 def test_host_entry_point_strided_and_unaligned_pinned_buffers(B, orc):
-    """Page-locked x and y read and written by the kernels through their
-    device mapping: row strides that are not multiples of 8 elements and a
-    start 2 bytes past a 16-byte boundary take the element-wise copy of x;
-    y's padding columns stay untouched; captured and direct (legacy
+    """Page-locked y written by the product kernel through its device
+    mapping, with row strides that are not multiples of 8 elements and
+    buffers starting 2 bytes past a 16-byte boundary (x then takes a 2-D
+    copy); y's padding columns stay untouched; captured and direct (legacy
     stream) calls agree."""
     L = make_small(61, 200, 512, 4, 300)
     layer = upload(B, L)
