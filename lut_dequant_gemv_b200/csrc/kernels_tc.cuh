@@ -10,7 +10,9 @@
 //   * One CTA of 12 warps per SM and call; its registers and shared memory
 //     fit two CTAs on an SM, so the next call's CTA (programmatic dependent
 //     launch) is resident while this one computes.  Each CTA owns a
-//     contiguous run of whole tiles (runs differ by at most one tile) and its
+//     contiguous run of whole tiles (runs differ by at most one tile, or,
+//     for skewed outliers, follow a split by weight that the layer computed
+//     at creation: cta_tile_range) and its
 //     warps split the CTA's units into contiguous ranges (equal, except that
 //     the eight warps that also sum the sparse part give one unit each to the
 //     other warps when the layer has outliers), so a tile is finished inside
@@ -59,9 +61,10 @@
 // pages.  Each thread sums its share per row (head piece, rows it holds
 // whole, tail piece) after x has arrived and before its dense loop; after a
 // barrier of those 256 threads, each row's interior sum and the pieces of the
-// threads whose shares cut the row are added in thread order (deterministic)
-// into the row's slot, and the threads arrive on an mbarrier that the
-// writers of y wait on.
+// threads whose shares cut the row are added into the row's slot -- in
+// thread order by one thread, or, for a row cut into more than kLongPieces
+// shares, by a warp in a fixed order (deterministic either way) -- and the
+// threads arrive on an mbarrier that the writers of y wait on.
 #pragma once
 
 #include <type_traits>
