@@ -512,9 +512,9 @@ sqz_status gemv_impl(const sqz_layer* L, const uint16_t* x, int32_t batch, int64
 // super-group) plus its share of the sparse part, and a CTA whose rows hold
 // many outliers should own fewer tiles.  Weight of a tile = its units x
 // kNnzPerUnit + its nonzeros (kNnzPerUnit: the nonzeros that cost about as
-// much as one unit's decode, measured on B200); CTA c starts at the first
-// tile whose weight prefix reaches c/grid of the total, every CTA keeping at
-// least one tile and at most twice the even split's count.  Used only when it
+// much as one unit's decode, measured on B200).  The CTAs take consecutive
+// runs of at least one tile and at most twice the even split's count, split
+// so that the heaviest run is as light as possible.  Used only when it
 // lowers the heaviest CTA's weight by more than 5 %; otherwise (uniform
 // outliers) the even split stays and `first` is left empty.
 constexpr int64_t kNnzPerUnit = 100;
@@ -532,18 +532,42 @@ bool split_tiles_by_weight(const std::vector<int32_t>& rp, int n_out, int ntiles
         for (int c = 0; c < grid; ++c) m = std::max(m, pre[f[c + 1]] - pre[f[c]]);
         return m;
     };
-    std::vector<int32_t> even((size_t)grid + 1), split((size_t)grid + 1);
+    std::vector<int32_t> even((size_t)grid + 1);
     for (int c = 0; c <= grid; ++c) even[c] = sqz::tc::tile_begin(ntiles, grid, c);
-    split[0] = 0;
-    split[grid] = ntiles;
-    for (int c = 1; c < grid; ++c) {
-        const int64_t target = pre[ntiles] * c / grid;
-        int t = (int)(std::lower_bound(pre.begin(), pre.end(), target) - pre.begin());
-        t = std::max(t, split[c - 1] + 1);              // at least one tile for CTA c - 1
-        t = std::min(t, split[c - 1] + cap);            // at most `cap` tiles for CTA c - 1
-        t = std::min(t, ntiles - (grid - c));           // one tile left for each CTA after it
-        t = std::max(t, ntiles - (grid - c) * cap);     // no CTA after it above `cap`
-        split[c] = t;
+    // The split into `grid` runs of 1..cap consecutive tiles whose heaviest
+    // run is lightest: the least bound W (binary search) for which runs packed
+    // greedily up to W and `cap` tiles number at most `grid`; then, while there
+    // are fewer runs than CTAs, the heaviest run of two or more tiles (the
+    // first on ties) gives its last tile to a run of its own.
+    auto pack = [&](int64_t W, std::vector<int32_t>* starts) {
+        starts->clear();
+        for (int t = 0; t < ntiles;) {
+            if (w[t] > W) return false;
+            starts->push_back(t);
+            int64_t sum = 0;
+            for (int k = 0; t < ntiles && k < cap && sum + w[t] <= W; ++k) sum += w[t++];
+        }
+        return (int)starts->size() <= grid;
+    };
+    std::vector<int32_t> split;
+    int64_t lo = *std::max_element(w.begin(), w.end()), hi = pre[ntiles];
+    while (lo < hi) {
+        const int64_t mid = lo + (hi - lo) / 2;
+        if (pack(mid, &split)) hi = mid;
+        else lo = mid + 1;
+    }
+    if (!pack(lo, &split)) return false;
+    split.push_back(ntiles);
+    while ((int)split.size() - 1 < grid) {
+        int best = -1;
+        int64_t best_w = -1;
+        for (int r = 0; r + 1 < (int)split.size(); ++r)
+            if (split[r + 1] - split[r] >= 2 && pre[split[r + 1]] - pre[split[r]] > best_w) {
+                best = r;
+                best_w = pre[split[r + 1]] - pre[split[r]];
+            }
+        if (best < 0) return false;  // fewer tiles than CTAs: cannot happen (grid <= ntiles)
+        split.insert(split.begin() + best + 1, split[best + 1] - 1);
     }
     int m = 0;
     for (int c = 0; c < grid; ++c) {
