@@ -511,19 +511,20 @@ sqz_status gemv_impl(const sqz_layer* L, const uint16_t* x, int32_t batch, int64
 // are skewed: a CTA's time is its dense units (one per tile and 256-column
 // super-group) plus its share of the sparse part, and a CTA whose rows hold
 // many outliers should own fewer tiles.  Weight of a tile = its units x
-// kNnzPerUnit + its nonzeros (kNnzPerUnit: the nonzeros that cost about as
-// much as one unit's decode, measured on B200).  The CTAs take consecutive
+// nnz_per_unit(bits) + its nonzeros (the nonzeros that cost about as much as
+// one unit's decode, measured on B200: 100 at 3 bits; a 4-bit unit takes
+// about 1.5x as long to decode, 150).  The CTAs take consecutive
 // runs of at least one tile and at most twice the even split's count, split
 // so that the heaviest run is as light as possible.  Used only when it
 // lowers the heaviest CTA's weight by more than 5 %; otherwise (uniform
 // outliers) the even split stays and `first` is left empty.
-constexpr int64_t kNnzPerUnit = 100;
-bool split_tiles_by_weight(const std::vector<int32_t>& rp, int n_out, int ntiles, int nsg, int grid,
+inline int64_t nnz_per_unit(int bits) { return bits == 3 ? 100 : 150; }
+bool split_tiles_by_weight(const std::vector<int32_t>& rp, int n_out, int bits, int ntiles, int nsg, int grid,
                            std::vector<int32_t>* first, int* ctiles_max) {
     std::vector<int64_t> w((size_t)ntiles), pre((size_t)ntiles + 1, 0);
     for (int t = 0; t < ntiles; ++t) {
         const int r0 = t * sqz::tc::kTileRows, r1 = std::min(n_out, r0 + sqz::tc::kTileRows);
-        w[t] = (int64_t)nsg * kNnzPerUnit + (rp[r1] - rp[r0]);
+        w[t] = (int64_t)nsg * nnz_per_unit(bits) + (rp[r1] - rp[r0]);
         pre[t + 1] = pre[t] + w[t];
     }
     const int even_max = (ntiles + grid - 1) / grid, cap = 2 * even_max;
@@ -624,7 +625,7 @@ sqz_status build_native(sqz_layer* L, cudaStream_t s) {
         std::vector<int32_t> rp((size_t)L->n_out + 1), first;
         SQZ_CUDA_TRY(cudaMemcpyAsync(rp.data(), L->rowptr, rp.size() * 4, cudaMemcpyDeviceToHost, s), "rowptr read");
         SQZ_CUDA_TRY(cudaStreamSynchronize(s), "rowptr read");
-        if (split_tiles_by_weight(rp, L->n_out, L->ntiles, L->nsg, L->grid, &first, &L->ctiles_max)) {
+        if (split_tiles_by_weight(rp, L->n_out, L->bits, L->ntiles, L->nsg, L->grid, &first, &L->ctiles_max)) {
             if ((st = alloc(&L->cta_tiles, (size_t)L->grid + 1, L, "CTA tiles")) != SQZ_OK) return st;
             SQZ_CUDA_TRY(cudaMemcpyAsync(L->cta_tiles, first.data(), first.size() * 4, cudaMemcpyHostToDevice, s),
                          "CTA tiles copy");
