@@ -138,7 +138,7 @@ struct Plan {
     int passes;      // passes over K (1, or more when x is staged in K chunks)
     int chunk_sg;    // super-groups of x per pass
     int xbufs;       // x buffers (2 when passes > 1: the next chunk loads during a pass)
-    int cm;          // batch columns carried by the sparse part and the combine (1 or 8*NT)
+    int cm;          // batch columns carried by the sparse part and the combine (carried_columns)
     int stages;      // shared-memory stages of each warp's code ring
     int csr_cap;     // CSR entries of a CTA that are staged in shared memory (more: read from global)
     // byte offsets
@@ -147,6 +147,17 @@ struct Plan {
 };
 
 __host__ __device__ inline int round_up(int v, int m) { return (v + m - 1) / m * m; }
+
+// Batch columns a launch carries through the sparse part, the warps' slots
+// and the combine: 1 for batch 1, else the batch rounded up to 2, 4 or 8
+// (one n-tile) or 16 (two).  The MMA always computes 8 columns per n-tile;
+// carrying fewer keeps the shared memory of batches 2-4 small enough for
+// two CTAs per SM.
+__host__ __device__ inline int carried_columns(int batch, int nt, bool single) {
+    if (single) return 1;
+    if (nt == 2) return 16;
+    return batch <= 2 ? 2 : batch <= 4 ? 4 : 8;
+}
 
 // First tile of CTA c when `ntiles` tiles are split over `grid` CTAs: the
 // first ntiles % grid CTAs take one tile more (32-bit arithmetic only).
@@ -190,7 +201,7 @@ __host__ __device__ inline Plan make_plan(int bits, int n_out, int k_in, int bat
     P.grid = grid_size(n_out, sms);
     P.ctiles_max = (ntiles + P.grid - 1) / P.grid;
     if (ctiles_max > P.ctiles_max) P.ctiles_max = ctiles_max;
-    P.cm = single ? 1 : 8 * nt;
+    P.cm = carried_columns(batch, nt, single);
     P.passes = passes < 1 ? 1 : (passes > nsg ? nsg : passes);
     P.chunk_sg = (nsg + P.passes - 1) / P.passes;
     P.passes = (nsg + P.chunk_sg - 1) / P.chunk_sg;
@@ -652,13 +663,16 @@ __global__ void dequant_native_kernel(const uint8_t* __restrict__ codes, const u
 
 // ------------------------------------------------------------ main kernel
 // MAC: kMacTensor / kMacCuda / kMacMixed.  SB: batch 1 (one column carried
-// through the sparse part and the combine).
-template <int BITS, int NT, int MAC, bool SB, bool RW>
+// through the sparse part and the combine).  CMX: the batch columns carried
+// (the plan's cm, carried_columns); it equals the launch's batch rounded up.
+template <int BITS, int NT, int MAC, bool SB, bool RW, int CMX = (SB ? 1 : 8 * NT)>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_fused_kernel(const __grid_constant__ Params p) {
     using F = Fmt<BITS>;
     using TAB = typename std::conditional<BITS == 3, Tab3, Tab4>::type;
     constexpr int BM = 8 * NT;              // batch columns of the MMA accumulators
-    constexpr int CM = SB ? 1 : BM;         // batch columns carried after the dense loop
+    constexpr int CM = CMX;                 // batch columns carried after the dense loop
+    static_assert(SB ? CMX == 1 : (CMX % 2 == 0 && CMX >= 2 && CMX <= BM && (NT == 1 || CMX > 8)),
+                  "carried columns: 1 for batch 1, else an even count within the n-tiles");
     constexpr int TE = kTileRows * CM;      // elements of one tile's result
     constexpr int V = F::kVecs;
     constexpr int CT = kCsrThreads;
@@ -1114,11 +1128,13 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_fused_kernel(const 
         } else {
 #pragma unroll
             for (int n = 0; n < NT; ++n) {
-                const int col = 8 * n + 2 * t4;
-                dst[g * CM + col] = rr[n][0];
-                dst[g * CM + col + 1] = rr[n][1];
-                dst[(g + 8) * CM + col] = rr[n][2];
-                dst[(g + 8) * CM + col + 1] = rr[n][3];
+                const int col = 8 * n + 2 * t4;  // even, like CM: col < CM covers col + 1
+                if (col < CM) {
+                    dst[g * CM + col] = rr[n][0];
+                    dst[g * CM + col + 1] = rr[n][1];
+                    dst[(g + 8) * CM + col] = rr[n][2];
+                    dst[(g + 8) * CM + col + 1] = rr[n][3];
+                }
             }
         }
         // shared tiles are combined after the loop (one CTA barrier)
@@ -1212,6 +1228,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) gemv_fused_kernel(const 
 #pragma unroll
                 for (int n = 0; n < NT; ++n) {
                     const int col = 8 * n + 2 * t4;
+                    if (col >= CM) continue;  // columns past the carried ones are never written out
                     if (whole) {
                         dst[g * CM + col] += rr[n][0];
                         dst[g * CM + col + 1] += rr[n][1];

@@ -210,9 +210,9 @@ void dispatch_rowwarp(const sqz_layer* L, const uint16_t* x, int32_t batch, int6
 }
 
 // ------------------------------------------------------------ fused kernel
-template <int BITS, int NT, int MAC, bool SB, bool RW = false>
+template <int BITS, int NT, int MAC, bool SB, bool RW = false, int CM = (SB ? 1 : 8 * NT)>
 sqz_status set_smem_attr(int bytes) {
-    SQZ_CUDA_TRY(cudaFuncSetAttribute(sqz::tc::gemv_fused_kernel<BITS, NT, MAC, SB, RW>,
+    SQZ_CUDA_TRY(cudaFuncSetAttribute(sqz::tc::gemv_fused_kernel<BITS, NT, MAC, SB, RW, CM>,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, bytes),
                  "cudaFuncSetAttribute");
     return SQZ_OK;
@@ -223,12 +223,16 @@ sqz_status prepare_fused_bits(int optin) {
     using namespace sqz::tc;
     sqz_status st;
     if ((st = set_smem_attr<BITS, 1, kMacTensor, true>(optin)) != SQZ_OK) return st;
-    if ((st = set_smem_attr<BITS, 1, kMacTensor, false>(optin)) != SQZ_OK) return st;
+    if ((st = set_smem_attr<BITS, 1, kMacTensor, false, false, 2>(optin)) != SQZ_OK) return st;
+    if ((st = set_smem_attr<BITS, 1, kMacTensor, false, false, 4>(optin)) != SQZ_OK) return st;
+    if ((st = set_smem_attr<BITS, 1, kMacTensor, false, false, 8>(optin)) != SQZ_OK) return st;
     if ((st = set_smem_attr<BITS, 2, kMacTensor, false>(optin)) != SQZ_OK) return st;
     if ((st = set_smem_attr<BITS, 1, kMacCuda, true>(optin)) != SQZ_OK) return st;
     if ((st = set_smem_attr<BITS, 1, kMacMixed, true>(optin)) != SQZ_OK) return st;
     if ((st = set_smem_attr<BITS, 1, kMacTensor, true, true>(optin)) != SQZ_OK) return st;
-    if ((st = set_smem_attr<BITS, 1, kMacTensor, false, true>(optin)) != SQZ_OK) return st;
+    if ((st = set_smem_attr<BITS, 1, kMacTensor, false, true, 2>(optin)) != SQZ_OK) return st;
+    if ((st = set_smem_attr<BITS, 1, kMacTensor, false, true, 4>(optin)) != SQZ_OK) return st;
+    if ((st = set_smem_attr<BITS, 1, kMacTensor, false, true, 8>(optin)) != SQZ_OK) return st;
     if ((st = set_smem_attr<BITS, 2, kMacTensor, false, true>(optin)) != SQZ_OK) return st;
     return SQZ_OK;
 }
@@ -369,7 +373,7 @@ int launch_columns(int bits, int n_out, int k_in, const DeviceShape& d, int batc
 // Launch with programmatic stream serialization: the kernel may start while
 // the previous kernel of the stream is still running; it prefetches only
 // weights before it waits for that kernel (griddepcontrol.wait).
-template <int BITS, int NT, int MAC, bool SB, bool RW = false>
+template <int BITS, int NT, int MAC, bool SB, bool RW = false, int CM = (SB ? 1 : 8 * NT)>
 cudaError_t launch_fused(const sqz::tc::Params& prm, cudaStream_t s) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)prm.plan.grid);
@@ -381,7 +385,20 @@ cudaError_t launch_fused(const sqz::tc::Params& prm, cudaStream_t s) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, sqz::tc::gemv_fused_kernel<BITS, NT, MAC, SB, RW>, prm);
+    return cudaLaunchKernelEx(&cfg, sqz::tc::gemv_fused_kernel<BITS, NT, MAC, SB, RW, CM>, prm);
+}
+
+// Batches 2..8 (one n-tile): the instantiation that carries the plan's
+// number of batch columns (2, 4 or 8; the plan sized shared memory for it).
+template <int BITS, bool RW>
+cudaError_t launch_fused_one_tile(const sqz::tc::Params& prm, cudaStream_t s) {
+    using namespace sqz::tc;
+    switch (prm.plan.cm) {
+        case 2: return launch_fused<BITS, 1, kMacTensor, false, RW, 2>(prm, s);
+        case 4: return launch_fused<BITS, 1, kMacTensor, false, RW, 4>(prm, s);
+        case 8: return launch_fused<BITS, 1, kMacTensor, false, RW, 8>(prm, s);
+        default: return cudaErrorInvalidValue;
+    }
 }
 
 // Batch 1 takes the requested multiply-accumulate unit; larger batches the
@@ -392,11 +409,11 @@ cudaError_t launch_fused_bits(const sqz::tc::Params& prm, int batch, int mac, in
     using namespace sqz::tc;
     if (csr_mode == SQZ_CSR_ROWWISE) {
         if (batch > 8) return launch_fused<BITS, 2, kMacTensor, false, true>(prm, s);
-        if (batch > 1) return launch_fused<BITS, 1, kMacTensor, false, true>(prm, s);
+        if (batch > 1) return launch_fused_one_tile<BITS, true>(prm, s);
         return launch_fused<BITS, 1, kMacTensor, true, true>(prm, s);
     }
     if (batch > 8) return launch_fused<BITS, 2, kMacTensor, false>(prm, s);
-    if (batch > 1) return launch_fused<BITS, 1, kMacTensor, false>(prm, s);
+    if (batch > 1) return launch_fused_one_tile<BITS, false>(prm, s);
     if (mac == SQZ_MAC_CUDA_CORES) return launch_fused<BITS, 1, kMacCuda, true>(prm, s);
     if (mac == SQZ_MAC_MIXED) return launch_fused<BITS, 1, kMacMixed, true>(prm, s);
     return launch_fused<BITS, 1, kMacTensor, true>(prm, s);

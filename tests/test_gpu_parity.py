@@ -412,8 +412,10 @@ def test_padded_columns_with_nonfinite_lut_entries(B, orc, bits, k_in, mac):
     (300, 6144, 4, 16, 0),
     (64, 16384, 3, 8, 0),    # 8 columns that need several passes
     (40, 20000, 4, 16, 0),   # 16 columns, several passes even in launches of 8
-    (300, 18432, 3, 5, 0),   # as many passes as launches of 2 would be: x in K chunks
+    (300, 18432, 3, 5, 0),   # launches of 4 columns (4 carried) and 1
     (300, 18432, 3, 5, 3),
+    (40, 98304, 4, 2, 0),    # one column does not fit at all: x in K chunks (7 passes, 2 carried)
+    (24, 98304, 3, 3, 1),    # 9 passes, 4 carried, x rows copied by the threads
 ])
 def test_batches_whose_x_is_staged_in_chunks(B, orc, n_out, k_in, bits, batch, ldx_pad):
     """Batches whose activations do not fit in shared memory at once: the

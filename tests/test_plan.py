@@ -91,9 +91,25 @@ def test_large_batches_split_into_single_pass_launches_of_eight():
     for batch, launches in ((16, 4), (8, 2)):
         p = B.sqz_plan_query(5120, 13824, 3, batch, **DEV)
         assert (p["launches"], p["columns_per_launch"], p["passes"]) == (launches, 4, 1), (batch, p)
-    # as many launches as passes: x staged in K chunks in one launch
+    # 4 columns carry 4 (not 8) batch columns and fit one pass: launches of 4
+    # and 1 instead of 3 passes
     p = B.sqz_plan_query(300, 18432, 3, 5, **DEV)
-    assert p["launches"] == 1 and p["passes"] == 3
+    assert (p["launches"], p["columns_per_launch"], p["passes"]) == (2, 4, 1), p
+    # not even one column fits one pass: x staged in K chunks in one launch
+    p = B.sqz_plan_query(40, 98304, 4, 2, **DEV)
+    assert (p["launches"], p["columns_per_launch"], p["passes"]) == (1, 2, 7), p
+    assert B.sqz_plan_query(40, 98304, 4, 1, **DEV)["fused"] == 0
+
+
+def test_small_batches_keep_two_ctas_per_sm():
+    # batches of 2-4 carry 2 or 4 batch columns through the sparse part and the
+    # combine (not 8), so their shared memory fits half an SM where x does
+    for n, k, batches in ((5120, 5120, (2, 3, 4)), (11008, 4096, (2, 3, 4)), (4096, 4096, (2, 3, 4)),
+                          (13824, 5120, (2, 3))):
+        for batch in batches:
+            p = B.sqz_plan_query(n, k, 3, batch, **DEV)
+            assert (p["launches"], p["passes"], p["ctas_per_sm"]) == (1, 1, 2), (n, k, batch, p)
+            assert p["smem_bytes"] <= HALF
 
 
 def test_plan_query_rejects_bad_arguments():
