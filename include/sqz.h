@@ -245,6 +245,28 @@ typedef struct {
 SQZ_API sqz_status sqz_plan_query(int32_t n_out, int32_t k_in, int32_t bits, int32_t batch, int32_t sm_count,
                                   int32_t smem_per_sm, int32_t smem_optin, int32_t predecode, sqz_plan_info* out);
 
+/*
+ * The split of a layer's row tiles (16 rows each) over the fused kernel's
+ * CTAs that sqz_create_layer computes from the outlier matrix, computed on
+ * the host from a HOST copy of rowptr ([n_out + 1] int32, rowptr[0] = 0,
+ * non-decreasing) -- no device needed.  The balanced sparse kernel of the
+ * summary page (§3.4 "Kernel Implementation", "Balanced sparse kernel")
+ * gives each thread an equal share of nonzeros; when the outliers are skewed
+ * over the rows, this library also balances across CTAs: each tile weighs
+ * w x its 256-column units + its nonzeros (w = 100 at 3 bits, 150 at 4),
+ * and the CTAs take consecutive runs of 1 to twice the even count of tiles,
+ * cut so that the heaviest run is as light as possible.  That split is
+ * used only when it lowers the heaviest CTA's weight by more than 5 %.
+ * On return first[c] (c = 0..grid, grid = min(sm_count, tiles)) is the first
+ * tile of CTA c and first[grid] the tile count; *weighted = 1 when the split
+ * by weight is used, 0 for the even split (runs differing by at most one
+ * tile).  `first` is caller-owned host memory of at least grid + 1 entries.
+ * Errors: SQZ_ERR_INVALID_ARG for NULL pointers, bits not in {3,4}, n_out,
+ * k_in or sm_count < 1, or a rowptr that does not start at 0 or decreases.
+ */
+SQZ_API sqz_status sqz_tile_split_query(const int32_t* rowptr, int32_t n_out, int32_t k_in, int32_t bits,
+                                        int32_t sm_count, int32_t* first, int32_t* weighted);
+
 /* Release a handle and its device memory.  NULL is accepted.  The caller
  * must make sure no work that uses the handle is still in flight. */
 SQZ_API sqz_status sqz_destroy(sqz_layer_t layer);

@@ -13,6 +13,7 @@ import ctypes
 import os
 from typing import Optional
 
+import numpy as np
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -38,7 +39,7 @@ STATUS_NAMES = {0: "SQZ_OK", 1: "SQZ_ERR_INVALID_ARG", 2: "SQZ_ERR_UNSUPPORTED",
 EXPORTED = ("sqz_create_layer", "sqz_gemv", "sqz_gemv_host", "sqz_debug_dequant", "sqz_layer_info",
             "sqz_destroy", "sqz_fp16_gemv", "sqz_last_error", "sqz_version", "sqz_check_csr_static",
             "sqz_layer_set_mac", "sqz_layer_set_csr_mode", "sqz_layer_status", "sqz_encode",
-            "sqz_encode_outliers", "sqz_plan_query", "sqz_layer_set_predecode")
+            "sqz_encode_outliers", "sqz_plan_query", "sqz_layer_set_predecode", "sqz_tile_split_query")
 
 
 class SqzError(RuntimeError):
@@ -104,6 +105,8 @@ def lib() -> ctypes.CDLL:
         L.sqz_encode.restype = ctypes.c_int
         L.sqz_plan_query.argtypes = [i32, i32, i32, i32, i32, i32, i32, i32, ctypes.POINTER(sqz_plan_info)]
         L.sqz_plan_query.restype = ctypes.c_int
+        L.sqz_tile_split_query.argtypes = [P, i32, i32, i32, i32, P, ctypes.POINTER(i32)]
+        L.sqz_tile_split_query.restype = ctypes.c_int
         L.sqz_encode_outliers.argtypes = [i64, ctypes.c_double]
         L.sqz_encode_outliers.restype = i64
         L.sqz_last_error.argtypes = []
@@ -317,6 +320,21 @@ def sqz_plan_query(n_out: int, k_in: int, bits: int, batch: int, sm_count: int =
     _check(lib().sqz_plan_query(n_out, k_in, bits, batch, sm_count, smem_per_sm, smem_optin, int(predecode),
                                 ctypes.byref(info)), "sqz_plan_query")
     return {name: int(getattr(info, name)) for name, _ in sqz_plan_info._fields_}
+
+
+def sqz_tile_split_query(rowptr, n_out: int, k_in: int, bits: int, sm_count: int = 148):
+    """The CTA -> tile split sqz_create_layer would use for this host rowptr
+    (host computation): (first tile of every CTA plus the tile count as an
+    int32 array of grid + 1 entries, True when the split by weight is used)."""
+    rp = np.ascontiguousarray(rowptr, dtype=np.int32)
+    if rp.shape != (n_out + 1,):
+        raise ValueError(f"rowptr must have n_out + 1 = {n_out + 1} entries")
+    ntiles = (max(n_out, 0) + 15) // 16
+    first = np.zeros(max(1, min(sm_count, ntiles)) + 1, dtype=np.int32)
+    weighted = ctypes.c_int32(0)
+    _check(lib().sqz_tile_split_query(rp.ctypes.data, n_out, k_in, bits, sm_count, first.ctypes.data,
+                                      ctypes.byref(weighted)), "sqz_tile_split_query")
+    return first, bool(weighted.value)
 
 
 def sqz_encode_outliers(n_weights: int, outlier_fraction: float) -> int:

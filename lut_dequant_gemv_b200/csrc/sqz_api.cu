@@ -949,6 +949,32 @@ sqz_status sqz_plan_query(int32_t n_out, int32_t k_in, int32_t bits, int32_t bat
     return SQZ_OK;
 }
 
+sqz_status sqz_tile_split_query(const int32_t* rowptr, int32_t n_out, int32_t k_in, int32_t bits, int32_t sm_count,
+                                int32_t* first, int32_t* weighted) {
+    if (!rowptr || !first || !weighted) return fail(SQZ_ERR_INVALID_ARG, "rowptr, first and weighted must not be NULL");
+    *weighted = 0;
+    if (bits != 3 && bits != 4) return fail(SQZ_ERR_INVALID_ARG, "bits must be 3 or 4 (got %d)", bits);
+    if (n_out < 1 || k_in < 1) return fail(SQZ_ERR_INVALID_ARG, "n_out and k_in must be positive");
+    if (sm_count < 1) return fail(SQZ_ERR_INVALID_ARG, "sm_count must be positive");
+    if (rowptr[0] != 0) return fail(SQZ_ERR_INVALID_ARG, "rowptr[0] must be 0");
+    for (int32_t i = 0; i < n_out; ++i)
+        if (rowptr[i + 1] < rowptr[i]) return fail(SQZ_ERR_INVALID_ARG, "rowptr decreases at row %d", i);
+    using namespace sqz::tc;
+    const int ntiles = (n_out + kTileRows - 1) / kTileRows;
+    const int grid = grid_size(n_out, sm_count);
+    const int nsg = ((k_in + 15) / 16 + kSgSteps - 1) / kSgSteps;
+    std::vector<int32_t> rp(rowptr, rowptr + (size_t)n_out + 1), split;
+    int ctiles_max = 0;
+    // the same condition and function as layer creation
+    if (rp[(size_t)n_out] > 0 && grid > 1 && split_tiles_by_weight(rp, n_out, bits, ntiles, nsg, grid, &split, &ctiles_max)) {
+        std::copy(split.begin(), split.end(), first);
+        *weighted = 1;
+    } else {
+        for (int c = 0; c <= grid; ++c) first[c] = tile_begin(ntiles, grid, c);
+    }
+    return SQZ_OK;
+}
+
 sqz_status sqz_debug_dequant(sqz_layer_t layer, uint16_t* w_out, void* stream) {
     if (!layer) return fail(SQZ_ERR_INVALID_ARG, "layer is NULL");
     const sqz_layer* L = layer;
