@@ -161,7 +161,7 @@ class ClockSampler:
                0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
                0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
 
-    def __init__(self, device_index: int, period_s: float = 0.0002):
+    def __init__(self, device_index: int, period_s: float = 0.0):
         self.ok = False
         self.samples, self.reasons = [], 0
         self.period = period_s
@@ -188,6 +188,9 @@ class ClockSampler:
         return i
 
     def _run(self):
+        # back to back (sleep(0) only yields to the launching thread): the
+        # NVML queries themselves set the pace, a fraction of a millisecond
+        # per sample, so even a timed region of a few ms gets ten or more
         nv = self.nv
         while not self._stop.is_set():
             try:
