@@ -125,3 +125,35 @@ def test_very_long_rows_fall_back_to_the_row_kernel():
     # one batch column of x beyond the shared memory of a CTA
     p = B.sqz_plan_query(64, 1 << 17, 4, 1, **DEV)
     assert p["fused"] == 0 and p["launches"] == 0
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_random_shapes_get_plans_within_their_shared_memory(seed):
+    """Random layer shapes and batches, beyond the workloads: a fused plan,
+    when there is one, covers the batch, fits the shared memory it claims
+    (half an SM when two CTAs share one) and keeps the ring bounds; only a
+    batch-1 call whose single column of x cannot fit falls back to the
+    row-per-warp kernel, and then so do no larger batches of a shorter K."""
+    import numpy as np
+
+    rng = np.random.default_rng(seed)
+    for _ in range(40):
+        bits = int(rng.choice([3, 4]))
+        step = 32 if bits == 3 else 8
+        k_in = step * int(rng.integers(1, 120000 // step))
+        n_out = int(rng.integers(1, 30000))
+        batch = int(rng.integers(1, 17))
+        p = B.sqz_plan_query(n_out, k_in, bits, batch, **DEV)
+        if not p["fused"]:
+            assert batch == 1 and k_in > 40000, (n_out, k_in, bits, batch)
+            continue
+        assert p["grid"] == min(DEV["sm_count"], (n_out + 15) // 16)
+        assert (p["launches"] - 1) * p["columns_per_launch"] < batch <= p["launches"] * p["columns_per_launch"]
+        budget = HALF if p["ctas_per_sm"] == 2 else DEV["smem_optin"]
+        assert 0 < p["smem_bytes"] <= budget, (n_out, k_in, bits, batch, p)
+        assert p["ring_stages"] in (3, 4) if p["passes"] == 1 else p["ring_stages"] >= 2
+        assert p["csr_stage_entries"] >= 0 and p["csr_stage_entries"] % 8 == 0
+        if batch == 1:
+            assert p["passes"] == 1 and p["launches"] == 1, (n_out, k_in, bits)
+            if k_in <= 8192:  # x of 16 KB or less: always room for the next call's CTA
+                assert p["ctas_per_sm"] == 2, (n_out, k_in, bits)
