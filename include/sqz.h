@@ -223,7 +223,10 @@ SQZ_API sqz_status sqz_layer_info(sqz_layer_t layer, int32_t* n_out, int32_t* k_
 /*
  * The launch plan sqz_gemv would use for a layer shape and batch on a device
  * with the given SM count and shared memory (per SM, and the opt-in maximum
- * of one CTA) -- computed on the host, no device needed.  fused = 0 means the
+ * of one CTA) -- computed on the host, no device needed -- for the even split
+ * of row tiles over the CTAs (a layer whose outliers are skewed enough to be
+ * split by weight, see sqz_tile_split_query, gives some CTAs up to twice the
+ * tiles, and its plan sizes their shared memory for that).  fused = 0 means the
  * row-per-warp kernel serves the call (all other fields 0).  Otherwise the
  * batch runs as `launches` launches of up to columns_per_launch columns,
  * each a grid of `grid` CTAs of `threads` threads with smem_bytes of dynamic
