@@ -157,3 +157,34 @@ def test_random_shapes_get_plans_within_their_shared_memory(seed):
             assert p["passes"] == 1 and p["launches"] == 1, (n_out, k_in, bits)
             if k_in <= 8192:  # x of 16 KB or less: always room for the next call's CTA
                 assert p["ctas_per_sm"] == 2, (n_out, k_in, bits)
+
+
+def test_x_in_k_chunks_only_when_no_column_launches_are_fewer():
+    """The planner stages x in K chunks (several passes) only when no split
+    of the batch into single-pass launches of 8, 4, 2 or 1 columns gives
+    fewer launches than those passes (and, above 8 columns, when 8 columns
+    do not fit one pass)."""
+    import numpy as np
+
+    rng = np.random.default_rng(7)
+    multi = 0
+    for _ in range(300):
+        bits = int(rng.choice([3, 4]))
+        step = 32 if bits == 3 else 8
+        k_in = step * int(rng.integers(60000 // step, 140000 // step))
+        n_out = int(rng.integers(1, 20000))
+        batch = int(rng.integers(2, 17))
+        p = B.sqz_plan_query(n_out, k_in, bits, batch, **DEV)
+        if not p["fused"] or p["passes"] == 1:
+            continue
+        multi += 1
+        assert p["launches"] == 1 and p["columns_per_launch"] == batch
+        for c in (8, 4, 2, 1):
+            if c >= batch:
+                continue
+            q = B.sqz_plan_query(n_out, k_in, bits, c, **DEV)
+            one_pass = q["fused"] and q["launches"] == 1 and q["passes"] == 1
+            if one_pass:
+                assert not (batch > 8 and c == 8), (n_out, k_in, bits, batch)
+                assert -(-batch // c) >= p["passes"], (n_out, k_in, bits, batch, c, p)
+    assert multi > 20
